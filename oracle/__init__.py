@@ -1,0 +1,159 @@
+"""CPU oracle for the NVFP4 verify GEMM: Python bindings to ``nvfp4_oracle.c``.
+
+TEST INFRASTRUCTURE ONLY. Only the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg may import this package. The GPU library never
+imports it and shares no code with it.
+
+The C source computes everything in fp64 from the format definitions:
+E2M1 codes (two per byte, low nibble = even k), one E4M3 scale per 16-element
+K block, one FP32 tensor scale; Y = X . dequant(W)^T. See the header of
+``nvfp4_oracle.c`` for the definitions and their sources.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "nvfp4_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle_nvfp4.so")
+
+OR_OK = 0
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into a host shared library (gcc, OpenMP, strict IEEE fp64)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
+               "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB)
+        p = ctypes.c_void_p
+        i64 = ctypes.c_int64
+        L.or_e2m1_decode.restype = ctypes.c_double
+        L.or_e2m1_decode.argtypes = [ctypes.c_uint32]
+        L.or_e4m3_decode.restype = ctypes.c_double
+        L.or_e4m3_decode.argtypes = [ctypes.c_uint32]
+        L.or_e4m3_encode.restype = ctypes.c_uint32
+        L.or_e4m3_encode.argtypes = [ctypes.c_double]
+        L.or_e2m1_encode.restype = ctypes.c_uint32
+        L.or_e2m1_encode.argtypes = [ctypes.c_double]
+        L.or_quantize.restype = ctypes.c_int
+        L.or_quantize.argtypes = [p, i64, i64, p, p, p]
+        L.or_dequant.restype = ctypes.c_int
+        L.or_dequant.argtypes = [p, p, ctypes.c_float, i64, i64, p, p]
+        L.or_gemm.restype = ctypes.c_int
+        L.or_gemm.argtypes = [p, i64, p, p, ctypes.c_float, i64, i64, p, p]
+        L.or_gemm_sampled.restype = ctypes.c_int
+        L.or_gemm_sampled.argtypes = [p, i64, p, p, ctypes.c_float, i64, i64, p, p, i64, p, p]
+        L.or_num_threads.restype = ctypes.c_int
+        L.or_set_num_threads.argtypes = [ctypes.c_int]
+        _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def e2m1_decode(code: int) -> float:
+    return lib().or_e2m1_decode(code)
+
+
+def e4m3_decode(byte: int) -> float:
+    return lib().or_e4m3_decode(byte)
+
+
+def e4m3_encode(t: float) -> int:
+    return lib().or_e4m3_encode(float(t))
+
+
+def e2m1_encode(q: float) -> int:
+    return lib().or_e2m1_encode(float(q))
+
+
+def quantize(w: np.ndarray):
+    """fp32 W[N, K] -> (codes uint8[N, K/2], scales uint8[N, K/16], g float)."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    N, K = w.shape
+    codes = np.zeros((N, K // 2), dtype=np.uint8)
+    scales = np.zeros((N, K // 16), dtype=np.uint8)
+    g = np.zeros(1, dtype=np.float32)
+    rc = lib().or_quantize(_ptr(w), N, K, _ptr(codes), _ptr(scales), _ptr(g))
+    if rc != OR_OK:
+        raise ValueError(f"or_quantize failed with code {rc}")
+    return codes, scales, float(g[0])
+
+
+def dequant(codes: np.ndarray, scales: np.ndarray, g: float, want_wq: bool = False):
+    """-> w32 float32[N, K] = fp32(e2m1*e4m3*g), and optionally wq float64[N, K] = e2m1*e4m3."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    N, K = codes.shape[0], codes.shape[1] * 2
+    w32 = np.zeros((N, K), dtype=np.float32)
+    wq = np.zeros((N, K), dtype=np.float64) if want_wq else None
+    rc = lib().or_dequant(_ptr(codes), _ptr(scales), ctypes.c_float(g), N, K, _ptr(w32),
+                          _ptr(wq) if wq is not None else None)
+    if rc != OR_OK:
+        raise ValueError(f"or_dequant failed with code {rc}")
+    return (w32, wq) if want_wq else w32
+
+
+def gemm(x_bits: np.ndarray, codes: np.ndarray, scales: np.ndarray, g: float):
+    """x_bits: bf16 bits uint16[M, K]. -> (y_ref float64[M, N], a_ref float64[M, N])."""
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    M, K = x_bits.shape
+    N = codes.shape[0]
+    if codes.shape[1] * 2 != K:
+        raise ValueError("K of X and W differ")
+    y = np.zeros((M, N), dtype=np.float64)
+    a = np.zeros((M, N), dtype=np.float64)
+    rc = lib().or_gemm(_ptr(x_bits), M, _ptr(codes), _ptr(scales), ctypes.c_float(g), N, K,
+                       _ptr(y), _ptr(a))
+    if rc != OR_OK:
+        raise ValueError(f"or_gemm failed with code {rc}")
+    return y, a
+
+
+def gemm_sampled(x_bits, codes, scales, g, m_idx, n_idx):
+    """Oracle outputs at the (m_idx[i], n_idx[i]) positions only."""
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    m_idx = np.ascontiguousarray(m_idx, dtype=np.int64)
+    n_idx = np.ascontiguousarray(n_idx, dtype=np.int64)
+    M, K = x_bits.shape
+    N = codes.shape[0]
+    y = np.zeros(len(m_idx), dtype=np.float64)
+    a = np.zeros(len(m_idx), dtype=np.float64)
+    rc = lib().or_gemm_sampled(_ptr(x_bits), M, _ptr(codes), _ptr(scales), ctypes.c_float(g), N, K,
+                               _ptr(m_idx), _ptr(n_idx), len(m_idx), _ptr(y), _ptr(a))
+    if rc != OR_OK:
+        raise ValueError(f"or_gemm_sampled failed with code {rc}")
+    return y, a
+
+
+def num_threads() -> int:
+    return lib().or_num_threads()
+
+
+def set_num_threads(n: int) -> None:
+    lib().or_set_num_threads(int(n))

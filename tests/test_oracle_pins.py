@@ -1,0 +1,339 @@
+"""Pins for the CPU oracle: checks against facts that do not come from the oracle itself.
+
+Each test pins one part of the oracle to something independent of its code:
+hand-worked values from the format definitions (tests/golden), library
+decoders/encoders (torch float8_e4m3fn, ml_dtypes float4_e2m1fn), closed forms,
+brute force with exact rationals, and special cases whose result is known
+exactly (identity, one-hot and small-integer weights, M-invariance).
+A plausible mistake (a dropped term, a wrong sign or nibble order, a transposed
+operand, a tie broken the wrong way) fails at least one of them.
+"""
+
+import math
+from fractions import Fraction
+
+import ml_dtypes
+import numpy as np
+import pytest
+import torch
+
+import synth
+from conftest import read_golden
+
+
+def _f(s):
+    return float("nan") if s == "nan" else float(s)
+
+
+def _same(a, b):
+    if math.isnan(b):
+        return math.isnan(a)
+    return a == b and math.copysign(1.0, a) == math.copysign(1.0, b)
+
+
+# ---------------------------------------------------------------- E2M1 / E4M3 decode
+
+def test_e2m1_decode_hand_worked(orc):
+    rows = read_golden("e2m1_decode.txt")
+    assert len(rows) == 16
+    for code, val in rows:
+        assert _same(orc.e2m1_decode(int(code, 16)), _f(val)), code
+
+
+def test_e2m1_decode_matches_ml_dtypes(orc):
+    lib_vals = np.arange(16, dtype=np.uint8).view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    for c in range(16):
+        assert _same(orc.e2m1_decode(c), float(lib_vals[c])), c
+
+
+def test_e4m3_decode_hand_worked(orc):
+    for byte, val in read_golden("e4m3_decode.txt"):
+        assert _same(orc.e4m3_decode(int(byte, 16)), _f(val)), byte
+
+
+def test_e4m3_decode_all_bytes_match_torch(orc):
+    lib_vals = torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).to(torch.float64)
+    for b in range(256):
+        assert _same(orc.e4m3_decode(b), float(lib_vals[b])), hex(b)
+
+
+def test_e4m3_decode_invariants(orc):
+    pos = [orc.e4m3_decode(b) for b in range(0x7F)]
+    assert all(pos[i] < pos[i + 1] for i in range(len(pos) - 1))  # strictly increasing
+    assert pos[-1] == 448.0 and pos[1] == 2.0 ** -9
+    for b in range(0x7F):
+        assert orc.e4m3_decode(0x80 | b) == -orc.e4m3_decode(b)
+
+
+# ---------------------------------------------------------------- encoders
+
+def test_e2m1_round_hand_worked(orc):
+    for q, code in read_golden("e2m1_round.txt"):
+        assert orc.e2m1_encode(float(q)) == int(code, 16), q
+
+
+def test_e2m1_round_matches_ml_dtypes(orc):
+    # Every multiple of 1/64 in [-6, 6]: ml_dtypes rounds to nearest even (it is a library RNE).
+    qs = np.arange(-384, 385, dtype=np.float64) / 64.0
+    lib = qs.astype(np.float32).astype(ml_dtypes.float4_e2m1fn).view(np.uint8)
+    for q, c in zip(qs, lib):
+        want = int(c) & 0xF
+        if want == 0x8:
+            want = 0x0  # the weight format never stores -0
+        assert orc.e2m1_encode(float(q)) == want, q
+
+
+def test_e2m1_round_brute_force_nearest(orc):
+    grid = [Fraction(v) for v in (0, 0.5, 1, 1.5, 2, 3, 4, 6)]
+    for i in range(-900, 901):
+        q = Fraction(i, 128)
+        a = min(abs(q), Fraction(6))
+        d = [abs(a - g) for g in grid]
+        best = min(d)
+        cands = [c for c in range(8) if d[c] == best]
+        c = cands[0] if len(cands) == 1 else [c for c in cands if c % 2 == 0][0]
+        if c and q < 0:
+            c |= 8
+        assert orc.e2m1_encode(float(q)) == c, q
+
+
+def test_e4m3_round_hand_worked(orc):
+    for t, b in read_golden("e4m3_round.txt"):
+        assert orc.e4m3_encode(float(t)) == int(b, 16), t
+
+
+def test_e4m3_round_matches_torch(orc):
+    rng = np.random.default_rng(1)
+    ts = np.concatenate([
+        rng.uniform(0, 448, 3000), np.exp(rng.uniform(math.log(2.0 ** -12), math.log(448.0), 3000)),
+    ]).astype(np.float32)
+    # every midpoint between adjacent finite codes is a tie; all are exact in fp32
+    vals = [float(v) for v in torch.arange(0x7F, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).to(torch.float64)]
+    mids = np.array([(vals[i] + vals[i + 1]) / 2 for i in range(len(vals) - 1)], dtype=np.float32)
+    ts = np.concatenate([ts, mids])
+    lib = torch.from_numpy(ts).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    for t, b in zip(ts, lib):
+        assert orc.e4m3_encode(float(t)) == int(b), float(t)
+
+
+def test_e4m3_round_saturates(orc):
+    for t in (448.0, 448.5, 464.0, 480.0, 1e30, float("inf")):
+        assert orc.e4m3_encode(t) == 0x7E
+
+
+# ---------------------------------------------------------------- packed decode
+
+def test_dequant_hand_worked_bytes(orc):
+    for cb, sb, g, w0, w1 in read_golden("nvfp4_packed.txt"):
+        codes = np.zeros((1, 8), dtype=np.uint8)
+        codes[0, 0] = int(cb, 16)
+        scales = np.array([[int(sb, 16)]], dtype=np.uint8)
+        w32 = orc.dequant(codes, scales, float(g))
+        assert _same(float(w32[0, 0]), float(w0)), (cb, sb, g)
+        assert _same(float(w32[0, 1]), float(w1)), (cb, sb, g)
+
+
+def test_dequant_scale_index_per_16_block(orc):
+    # scale b covers k in [16b, 16b+16): give each block a distinct power-of-two scale
+    K = 64
+    codes = np.full((1, K // 2), 0x22, dtype=np.uint8)  # every weight code 2 -> 1.0
+    scales = np.array([[0x38, 0x40, 0x48, 0x30]], dtype=np.uint8)  # 1, 2, 4, 0.5
+    w = orc.dequant(codes, scales, 1.0)[0]
+    want = np.repeat([1.0, 2.0, 4.0, 0.5], 16)
+    assert np.array_equal(w, want)
+
+
+def test_dequant_fp32_single_rounding(orc):
+    # g with a full 24-bit mantissa: the fp32 result must be the correctly rounded exact product
+    rng = np.random.default_rng(5)
+    codes = rng.integers(0, 256, (4, 32), dtype=np.uint8)
+    scales = rng.integers(0, 0x7F, (4, 4), dtype=np.uint8)
+    g = float(np.float32(0.1234567))
+    w32, wq = orc.dequant(codes, scales, g, want_wq=True)
+    for n in range(4):
+        for k in range(64):
+            exact = Fraction(float(wq[n, k])) * Fraction(g)
+            assert Fraction(float(w32[n, k])) == Fraction(float(np.float32(float(exact)))) or \
+                abs(Fraction(float(w32[n, k])) - exact) <= abs(exact) * Fraction(1, 2 ** 24)
+
+
+# ---------------------------------------------------------------- quantiser
+
+def _grid_tensor(rng, N, K, g):
+    """A tensor whose blocks are exactly on the NVFP4 grid: returns (w, codes, scales)."""
+    nb = K // 16
+    codes = rng.integers(0, 16, (N, K))
+    codes[codes == 8] = 0  # -0 is never produced
+    # one element of every block has magnitude 6 so the block max is 6*dec(s)*g
+    pos = rng.integers(0, 16, (N, nb))
+    for n in range(N):
+        for b in range(nb):
+            codes[n, 16 * b + pos[n, b]] = 7 if rng.random() < 0.5 else 15
+    scales = rng.integers(0x08, 0x7E, (N, nb))
+    scales[0, 0] = 0x7E  # the tensor's absmax block carries 448
+    mag = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], dtype=np.float64)
+    e2m1 = np.where(codes & 8, -1.0, 1.0) * mag[codes & 7]
+    dec = np.array([float(v) for v in torch.arange(256, dtype=torch.int32).to(torch.uint8)
+                    .view(torch.float8_e4m3fn).to(torch.float64)])
+    w = e2m1 * np.repeat(dec[scales], 16, axis=1) * g
+    packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+    return w.astype(np.float32), packed, scales.astype(np.uint8)
+
+
+def test_quantize_round_trips_grid_tensors(orc):
+    rng = np.random.default_rng(7)
+    for g in (2.0 ** -8, 2.0 ** -3, 1.0):
+        w, codes, scales = _grid_tensor(rng, 8, 64, g)
+        c2, s2, g2 = orc.quantize(w)
+        assert g2 == g
+        assert np.array_equal(s2, scales)
+        assert np.array_equal(c2, codes)
+
+
+def test_quantize_recipe_invariants(orc):
+    w = synth.w_f32(64, 256, seed=3, tensor_id=0)
+    codes, scales, g = orc.quantize(w)
+    amax = float(np.max(np.abs(w)))
+    assert g == float(np.float32(amax / 2688.0))
+    w32, wq = orc.dequant(codes, scales, g, want_wq=True)
+    dec = np.array([orc.e4m3_decode(int(b)) for b in range(256)])
+    sv = np.repeat(dec[scales], 16, axis=1)
+    # the block holding the tensor's absmax has scale 448 (0x7E)
+    n0, k0 = np.unravel_index(np.argmax(np.abs(w)), w.shape)
+    assert scales[n0, k0 // 16] == 0x7E
+    # every element is within one grid step of the scaled value, sign is kept
+    err = np.abs(w.astype(np.float64) - wq * g)
+    assert np.all(err <= sv * g * 1.0 + 1e-30)
+    assert np.all((wq == 0) | (np.sign(wq) == np.sign(w)))
+    # block max maps to at most 6*(1 + 2^-4) on the E2M1 grid (E4M3 rounding bound, normal scales)
+    bmax = np.abs(w.astype(np.float64)).reshape(64, 16, 16).max(axis=2)
+    dv = dec[scales]
+    normal = dv >= 2.0 ** -6
+    assert np.all(bmax[normal] / (dv[normal] * g) <= 6.0 * (1 + 2.0 ** -4))
+
+
+def test_quantize_zero_tensor(orc):
+    codes, scales, g = orc.quantize(np.zeros((4, 32), dtype=np.float32))
+    assert g == 0.0 and not codes.any() and not scales.any()
+
+
+def test_quantize_rejects_nonfinite(orc):
+    w = np.zeros((2, 16), dtype=np.float32)
+    w[1, 3] = np.inf
+    with pytest.raises(ValueError):
+        orc.quantize(w)
+
+
+# ---------------------------------------------------------------- GEMM
+
+def test_gemm_hand_worked(orc):
+    rows = {r[0]: r[1:] for r in read_golden("gemm_worked.txt")}
+    codes = np.array([[int(b, 16) for b in rows["codes"]]], dtype=np.uint8)
+    scales = np.array([[int(rows["scale"][0], 16)]], dtype=np.uint8)
+    g = float(rows["g"][0])
+    x = np.array([[float(v) for v in rows["x0"]], [float(v) for v in rows["x1"]]], dtype=np.float32)
+    y, a = orc.gemm(synth.f32_to_bf16_bits(x), codes, scales, g)
+    assert y[:, 0].tolist() == [float(v) for v in rows["y"]]
+
+
+def _exact_y(x_bits, wq, g):
+    xf = synth.bf16_bits_to_f32(x_bits).astype(np.float64)
+    M, K = xf.shape
+    N = wq.shape[0]
+    out = []
+    for m in range(M):
+        row = []
+        for n in range(N):
+            s = sum(Fraction(float(xf[m, k])) * Fraction(float(wq[n, k])) for k in range(K))
+            row.append(s * Fraction(g))
+        out.append(row)
+    return out
+
+
+def test_gemm_brute_force_2x16x16_exact(orc):
+    for trial in range(4):
+        w = synth.w_f32(16, 16, seed=trial, tensor_id=1)
+        codes, scales, g = orc.quantize(w)
+        x = synth.x_bf16(2, 16, seed=trial, tensor_id=2)
+        y, a = orc.gemm(x, codes, scales, g)
+        _, wq = orc.dequant(codes, scales, g, want_wq=True)
+        ex = _exact_y(x, wq, g)
+        for m in range(2):
+            for n in range(16):
+                # sum of 16 exact products: within one fp64 rounding of the product with g
+                assert abs(Fraction(y[m, n]) - ex[m][n]) <= Fraction(a[m, n]) * Fraction(1, 2 ** 50)
+
+
+def test_gemm_matches_numpy_matmul(orc):
+    w = synth.w_f32(48, 512, seed=0, tensor_id=3, dist="t4")
+    codes, scales, g = orc.quantize(w)
+    x = synth.x_bf16(5, 512, seed=0, tensor_id=4)
+    y, a = orc.gemm(x, codes, scales, g)
+    _, wq = orc.dequant(codes, scales, g, want_wq=True)
+    ref = (synth.bf16_bits_to_f32(x).astype(np.float64) @ wq.T) * g
+    assert np.all(np.abs(y - ref) <= a * 1e-12)
+    assert np.all(a >= np.abs(y) * (1 - 1e-12))
+
+
+def test_gemm_identity_weight_returns_x(orc):
+    K = 64
+    codes = np.zeros((K, K // 2), dtype=np.uint8)
+    for n in range(K):
+        codes[n, n // 2] = 0x02 if n % 2 == 0 else 0x20  # code 2 = 1.0 on the diagonal
+    scales = np.full((K, K // 16), 0x38, dtype=np.uint8)
+    x = synth.x_bf16(7, K, seed=1, tensor_id=5)
+    y, _ = orc.gemm(x, codes, scales, 1.0)
+    assert np.array_equal(y, synth.bf16_bits_to_f32(x).astype(np.float64))
+
+
+def test_gemm_one_hot_weight_is_permuted_scaled_copy(orc):
+    rng = np.random.default_rng(2)
+    K = N = 128
+    perm = rng.permutation(K)
+    codes = np.zeros((N, K // 2), dtype=np.uint8)
+    for n in range(N):
+        k = perm[n]
+        codes[n, k // 2] |= (0xD if k % 2 == 0 else 0xD0)  # code 0xD = -3.0
+    scales = np.full((N, K // 16), 0x30, dtype=np.uint8)  # 0.5
+    x = synth.x_bf16(3, K, seed=2, tensor_id=6)
+    y, _ = orc.gemm(x, codes, scales, 0.25)
+    xf = synth.bf16_bits_to_f32(x).astype(np.float64)
+    assert np.array_equal(y, xf[:, perm] * (-3.0 * 0.5 * 0.25))
+
+
+def test_gemm_small_integer_exact(orc):
+    rng = np.random.default_rng(4)
+    M, N, K = 4, 32, 256
+    x = rng.integers(-4, 5, (M, K)).astype(np.float32)
+    codes = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    scales = np.full((N, K // 16), 0x38, dtype=np.uint8)
+    g = 2.0 ** -3
+    y, _ = orc.gemm(synth.f32_to_bf16_bits(x), codes, scales, g)
+    mag = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6])
+    lo, hi = codes & 15, codes >> 4
+    c = np.empty((N, K), dtype=np.int64)
+    c[:, 0::2], c[:, 1::2] = lo, hi
+    wv = np.where(c & 8, -1.0, 1.0) * mag[c & 7]
+    want = (x.astype(np.float64) @ wv.T) * g  # integers and halves: exact in fp64
+    assert np.array_equal(y, want)
+
+
+def test_gemm_row_independent_of_M(orc):
+    w = synth.w_f32(40, 1024, seed=9, tensor_id=7)
+    codes, scales, g = orc.quantize(w)
+    x = synth.x_bf16(8, 1024, seed=9, tensor_id=8)
+    y8, _ = orc.gemm(x, codes, scales, g)
+    for i in range(8):
+        y1, _ = orc.gemm(x[i:i + 1], codes, scales, g)
+        assert np.array_equal(y1[0], y8[i])
+
+
+def test_gemm_sampled_equals_full(orc):
+    w = synth.w_f32(64, 256, seed=1, tensor_id=9)
+    codes, scales, g = orc.quantize(w)
+    x = synth.x_bf16(6, 256, seed=1, tensor_id=10)
+    y, a = orc.gemm(x, codes, scales, g)
+    rng = np.random.default_rng(0)
+    mi, ni = rng.integers(0, 6, 50), rng.integers(0, 64, 50)
+    ys, as_ = orc.gemm_sampled(x, codes, scales, g, mi, ni)
+    assert np.array_equal(ys, y[mi, ni]) and np.array_equal(as_, a[mi, ni])
