@@ -1,0 +1,430 @@
+"""Benchmark of the NVFP4 verify GEMM on B200: the full 64-layer verify-pass weight stream.
+
+Workload (the spec configuration): 64 layers x {QKV 5120->7168, O 5120->5120,
+gate+up 5120->34816, down 17408->5120}, all NVFP4 (21.14 G weights, 11.89 GB of codes and
+scales), each matrix with its own X (bf16, N(0,1)) and Y. Weights are drawn on the GPU
+(N(0, 0.02); 0.02*t(4) for down) and packed by the library's quantiser; everything is
+synthetic and seeded. One step = one pass of the whole stack at every row count M = 1..32,
+one tl_nvfp4_verify_stack launch per M (the staircase). The working set (11.9 GB) is far
+larger than L2, so no flush is needed between passes.
+
+Prints ONE JSON line (rank 0). Value = algorithmic bytes of all passes / device time.
+With --gpus N (torchrun), every rank runs its own replica (the path does not shard;
+replicas only); value = all ranks' bytes / max-over-ranks time.
+
+--impl reference times the CPU oracle (the only reference this workload has) on a bounded
+sample of the same workload on the host cores.
+"""
+
+from __future__ import annotations
+
+import argparse
+import ctypes
+import glob
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "verify-GEMM µs and HBM GB/s vs rows M=1–32; % of B200 HBM peak (1 GPU)"
+LAYERS = 64
+M_SWEEP = list(range(1, 33))
+WORKLOAD = ("64-layer verify-pass weight stream: 64 x {QKV 5120->7168, O 5120->5120, gate+up 5120->34816, "
+            "down 17408->5120}, NVFP4 (E2M1 codes, E4M3 per-16 scales, FP32 tensor scale), bf16 X/Y, "
+            "one stack pass per M = 1..32")
+
+
+def stack_shapes():
+    import synth
+    out = []
+    for layer in range(LAYERS):
+        for j, (name, K, N) in enumerate(synth.LAYER_SHAPES):
+            out.append((layer, j, name, N, K, synth.LAYER_DISTS[name]))
+    return out
+
+
+def w_bytes(shapes):
+    return sum(N * K // 2 + N * K // 16 + 4 for (_, _, _, N, K, _) in shapes)
+
+
+def pass_bytes(shapes, M):
+    """Algorithmic bytes of one stack pass: every code, scale, X and Y element once."""
+    return w_bytes(shapes) + sum(2 * M * K + 2 * M * N for (_, _, _, N, K, _) in shapes)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def source_hash():
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "nvfp4_weight_gemm_b200", "csrc", "*"))):
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """dram bytes per launch from the committed ncu summary, if it was taken on this source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None, None
+    d = json.load(open(p))
+    if d.get("source_hash") != source_hash():
+        return None, None
+    return d.get("dram_bytes_per_launch"), d
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"tl_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        pw = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows), "power_w_max": max(pw) if pw else None}
+
+
+# --------------------------------------------------------------------------- CPU oracle sample
+
+def cpu_sample(rows_per_shape: int, M: int):
+    """Time the CPU oracle on `rows_per_shape` weight rows of each of the four layer shapes at M rows.
+
+    Returns (bytes, seconds, threads). The oracle is used as it stands (fp64, OpenMP over rows)."""
+    import oracle
+    import synth
+    oracle.build()
+    total_b, total_t = 0, 0.0
+    for j, (name, K, N) in enumerate(synth.LAYER_SHAPES):
+        w = synth.w_f32(rows_per_shape, K, seed=0, tensor_id=j, dist=synth.LAYER_DISTS[name])
+        codes, scales, g = oracle.quantize(w)
+        x = synth.x_bf16(M, K, seed=0, tensor_id=synth.X_ID_BASE + j)
+        t0 = time.perf_counter()
+        oracle.gemm(x, codes, scales, g)
+        total_t += time.perf_counter() - t0
+        total_b += rows_per_shape * K // 2 + rows_per_shape * K // 16 + 2 * M * K + 2 * M * rows_per_shape
+    return total_b, total_t, oracle.num_threads()
+
+
+CPU_ROWS = 192
+CPU_SAMPLE_DESC = (f"{CPU_ROWS} weight rows of each layer shape (QKV, O, gate+up, down), full K, at M = 32: "
+                   f"fp64 oracle GEMM, GB/s over the same algorithmic bytes")
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    for _ in range(args.warmup):
+        cpu_sample(CPU_ROWS // 4, 32)
+    byts, secs = 0, 0.0
+    threads = 1
+    for _ in range(args.steps):
+        b, s, threads = cpu_sample(CPU_ROWS, 32)
+        byts += b
+        secs += s
+    value = byts / secs / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample": CPU_SAMPLE_DESC},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": CPU_SAMPLE_DESC},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------- GPU arm
+
+def build_stack(dev, seed=0):
+    """Draw and pack every weight of the stack on `dev`. Returns [(codes, scales, g, N, K)]."""
+    import torch
+    import nvfp4_weight_gemm_b200 as tl
+    import synth
+    out = []
+    for (layer, j, name, N, K, dist) in stack_shapes():
+        w = synth.w_f32_torch(N, K, seed, layer * 4 + j, dev, dist)
+        codes, scales, g = tl.quantize(w)
+        del w
+        out.append((codes, scales, g, N, K))
+    torch.cuda.synchronize()
+    return out
+
+
+def main_gpu(args):
+    import torch
+    import torch.distributed as dist
+    import nvfp4_weight_gemm_b200 as tl
+    import synth
+    from nvfp4_weight_gemm_b200 import build as tlbuild
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if rank == 0:
+        tlbuild.build()
+    if world > 1:
+        dist.barrier()
+    tl.init(local)
+
+    shapes = stack_shapes()
+    stack = build_stack(dev, seed=rank)
+    Mmax = max(M_SWEEP)
+    xs = [synth.x_bf16_torch(Mmax, K, rank, synth.X_ID_BASE + i, dev) for i, (_, _, _, N, K) in enumerate(stack)]
+    ys = [torch.empty((Mmax, N), dtype=torch.bfloat16, device=dev) for (_, _, _, N, K) in stack]
+    stream = torch.cuda.Stream(device=dev)
+
+    # one plan per M: X/Y views of the first M rows (row-major prefixes are contiguous)
+    plans = {M: tl.Plan([(c, s, g, xs[i][:M], ys[i][:M]) for i, (c, s, g, N, K) in enumerate(stack)], M)
+             for M in M_SWEEP}
+
+    def run_pass(M):
+        plans[M].run(stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, args.warmup)):
+            for M in M_SWEEP:
+                run_pass(M)
+    stream.synchronize()
+    tl.check_device_error(stream)
+
+    # ---- timed region: device events around every launch, on the launching stream
+    n_launch = args.steps * len(M_SWEEP)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_launch)]
+    clk = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clk.start()
+    time.sleep(0.3)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_stop = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    i = 0
+    for _ in range(args.steps):
+        for M in M_SWEEP:
+            ev[i][0].record(stream)
+            run_pass(M)
+            ev[i][1].record(stream)
+            i += 1
+    t_stop.record(stream)
+    stream.synchronize()
+    clocks = clk.stop()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    tl.check_device_error(stream)
+    total_ms = t_start.elapsed_time(t_stop)
+    per = [e0.elapsed_time(e1) for e0, e1 in ev]
+    per_M = {M: statistics.median(per[j::len(M_SWEEP)]) for j, M in enumerate(M_SWEEP)}
+    per_M_min = {M: min(per[j::len(M_SWEEP)]) for j, M in enumerate(M_SWEEP)}
+    bytes_step = sum(pass_bytes(shapes, M) for M in M_SWEEP)
+    launch_ms_sum = sum(per)
+
+    # ---- end to end through the C ABI with host buffers (copies inside the timed region):
+    # per M, a plan whose X_i / Y_i are packed back to back in one device buffer each
+    xtot = sum(Mmax * K for (_, _, _, N, K) in stack)
+    ytot = sum(Mmax * N for (_, _, _, N, K) in stack)
+    x_host = torch.empty(xtot, dtype=torch.bfloat16).pin_memory()
+    off = 0
+    for x in xs:
+        x_host[off:off + x.numel()].copy_(x.reshape(-1).cpu())
+        off += x.numel()
+    y_host = torch.empty(ytot, dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty(xtot, dtype=torch.bfloat16, device=dev)
+    y_dev = torch.empty(ytot, dtype=torch.bfloat16, device=dev)
+    e2e_plans = {}
+    for M in M_SWEEP:
+        ents, xo, yo = [], 0, 0
+        for (c, s, g, N, K) in stack:
+            ents.append((c, s, g, x_dev[xo:xo + M * K].view(M, K), y_dev[yo:yo + M * N].view(M, N)))
+            xo += M * K
+            yo += M * N
+        e2e_plans[M] = tl.Plan(ents, M)
+    e2e_h2d = sum(2 * M * K for M in M_SWEEP for (_, _, _, N, K) in stack)
+    e2e_d2h = sum(2 * M * N for M in M_SWEEP for (_, _, _, N, K) in stack)
+
+    def e2e_step():
+        for M in M_SWEEP:
+            e2e_plans[M].run_host(x_host, y_host, stream=stream)
+
+    e2e_step()
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    e0.record(stream)
+    e2e_steps = max(1, args.steps // 2)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    stream.synchronize()
+    tl.check_device_error(stream)
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    for pl in e2e_plans.values():
+        pl.close()
+
+    # ---- M-invariance: row i at M=k against the same row computed alone (M=1)
+    inv = {}
+    for k in (8, 16, 24, 32):
+        plans[k].run(stream=stream)
+        stream.synchronize()
+        yk = [y[:k].clone() for y in ys]
+        same = total = 0
+        for i_row in range(k):
+            p1 = tl.Plan([(c, s, g, xs[i][i_row:i_row + 1], ys[i][:1]) for i, (c, s, g, N, K) in enumerate(stack)], 1)
+            p1.run(stream=stream)
+            stream.synchronize()
+            p1.close()
+            for i in range(len(stack)):
+                same += int(torch.equal(ys[i][0], yk[i][i_row]))
+                total += 1
+        inv[str(k)] = same / total
+    tl.check_device_error(stream)
+
+    # ---- reduce over ranks: max time, summed bytes
+    stats = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(stats, op=dist.ReduceOp.MAX)
+    total_ms, e2e_ms = stats.tolist()
+
+    if rank == 0:
+        peak, peak_kind = load_peaks()
+        value = world * bytes_step * args.steps / (total_ms * 1e-3) / 1e9
+        achieved = bytes_step * args.steps / (launch_ms_sum * 1e-3) / 1e9
+        traffic, _ = profiled_traffic()
+        stair = {}
+        for M in M_SWEEP:
+            gbs = pass_bytes(shapes, M) / (per_M[M] * 1e-3) / 1e9
+            stair[str(M)] = {"us": round(per_M[M] * 1e3, 1), "us_min": round(per_M_min[M] * 1e3, 1),
+                             "gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
+                             "w_only_gbs": round(w_bytes(shapes) / (per_M[M] * 1e-3) / 1e9, 1)}
+        cb, cs, cthreads = cpu_sample(CPU_ROWS, 32)
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "matrices": len(shapes), "weights": sum(N * K for (_, _, _, N, K, _) in shapes),
+                       "w_bytes": w_bytes(shapes), "M": "1..32 (one pass each per step)",
+                       "l2": "working set 11.9 GB >> 126 MB L2; no flush needed", "parallelism": f"replicas x{world}"},
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": traffic, "peak_kind": peak_kind,
+                         "kernel": "gemm_tc_kernel (one launch per stack pass)"},
+            "staircase": stair,
+            "min_frac_over_M": round(min(v["frac"] for v in stair.values()), 4),
+            "m_invariance_row_fraction": inv,
+            "cpu_baseline": {"value": round(cb / cs / 1e9, 4), "unit": "GB/s", "cores": cthreads, "kind": "oracle",
+                             "sample": CPU_SAMPLE_DESC},
+            "e2e": {"value": round(world * bytes_step / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                    "h2d_bytes_per_step": e2e_h2d, "d2h_bytes_per_step": e2e_d2h},
+            "gpu_launches": n_launch,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    for pl in plans.values():
+        pl.close()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def run_profile_case(args):
+    """Small case for ncu: one matrix (N x K), `--reps` launches of the tensor-core path at --M rows.
+
+    Inputs are drawn and packed on the device like the stack's; prints one summary line."""
+    import torch
+    import nvfp4_weight_gemm_b200 as tl
+    import synth
+    N, K = (int(v) for v in args.profile_matrix.lower().split("x"))
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    tl.init(0)
+    w = synth.w_f32_torch(N, K, 0, 0, dev)
+    codes, scales, g = tl.quantize(w)
+    del w
+    x = synth.x_bf16_torch(args.M, K, 0, synth.X_ID_BASE, dev)
+    y = torch.empty((args.M, N), dtype=torch.bfloat16, device=dev)
+    plan = tl.Plan([(codes, scales, g, x, y)], args.M)
+    for _ in range(args.reps):
+        plan.run()
+    torch.cuda.synchronize()
+    tl.check_device_error()
+    plan.close()
+    print(json.dumps({"profile_case": f"{N}x{K}", "M": args.M, "reps": args.reps}), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--profile-matrix", default=None, help="NxK: run one matrix --reps times (for ncu)")
+    ap.add_argument("--M", type=int, default=32)
+    ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    if args.profile_matrix:
+        return run_profile_case(args)
+    return main_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

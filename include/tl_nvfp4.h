@@ -1,0 +1,188 @@
+/*
+ * tl_nvfp4.h -- C ABI of libtl_nvfp4.so, the NVFP4 verify GEMM for B200 (sm_100a).
+ *
+ * The operation. One verify pass of a speculative decoder checks all rows of
+ * a draft tree (8/16/24/32 rows: 7/15/23/31 nodes plus the root) with one
+ * forward pass of the big model, and that pass is dominated by reading every
+ * weight once (TandemLLM docs v0.12.0, "What TandemLLM is", section 1.2; the
+ * StairCut research page, "What it says"). Each projection of that pass is
+ *
+ *     Y[M,N] = X[M,K] . dequant(W)[N,K]^T,      1 <= M <= 32,
+ *
+ * with W stored as NVFP4: four bits a weight and one scale per 16 weights
+ * (same page, section 1.2). At the bit level:
+ *   codes    uint8 [N][K/2]  two E2M1 codes per byte, low nibble = even k;
+ *                            E2M1 magnitudes {0, 0.5, 1, 1.5, 2, 3, 4, 6}, bit 3 = sign
+ *   scales   uint8 [N][K/16] one E4M3 ("fn": no inf, 0x7F/0xFF NaN, max 448)
+ *                            scale per 16-element K block
+ *   global_scale  float      one FP32 tensor scale that multiplies:
+ *                            w[n,k] = e2m1(code) * e4m3(scale) * global_scale
+ *   x        bf16  [M][K]    the draft-tree rows
+ *   y        bf16  [M][N]    fp32 accumulation, rounded to bf16 (nearest even) once
+ * All arrays are row-major and contiguous, in device memory unless stated.
+ *
+ * Determinism. The reduction order of every output element is fixed: the same
+ * inputs give bit-identical Y on every run (the pages' NVFP4 kernels keep a
+ * fixed reduction order; "What TandemLLM is", section 1.7). No float atomics.
+ *
+ * Ownership and execution. The caller owns every buffer and stream. Calls are
+ * asynchronous on `stream` (a cudaStream_t; NULL means the legacy default
+ * stream) and do not synchronise, unless stated. The library keeps one small
+ * per-device state (split-K workspace, error word, descriptor cache) created
+ * by tl_init() or lazily by the first call on a device; call tl_init() before
+ * capturing a stream into a CUDA graph. Entry points are thread-safe for
+ * distinct streams; calls on one stream must not be interleaved from several
+ * host threads without external ordering.
+ *
+ * Errors. Every entry point validates its arguments first: on a violation it
+ * launches nothing and returns a status; tl_last_error_message() then holds a
+ * one-line reason for the calling thread. Faults found on the device (a wait
+ * that ran out, an invalid internal state) are recorded in a device status
+ * word and reported by tl_check_device_error().
+ */
+#ifndef TL_NVFP4_H
+#define TL_NVFP4_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    TL_OK = 0,
+    TL_ERR_INVALID_VALUE = 1,   /* a size or pointer argument is out of range */
+    TL_ERR_MISALIGNED = 2,      /* a pointer is not 16-byte aligned */
+    TL_ERR_UNSUPPORTED = 3,     /* valid request this build does not serve (e.g. M > 32) */
+    TL_ERR_CUDA = 4,            /* a CUDA runtime/driver call failed */
+    TL_ERR_TIMEOUT = 5,         /* a device-side wait ran past its iteration limit */
+    TL_ERR_NOT_INITIALIZED = 6, /* no usable device / state */
+    TL_ERR_NONFINITE = 7,       /* quantiser input holds NaN or infinity */
+    TL_ERR_DEVICE_FAULT = 8     /* the device status word holds an internal error */
+} tl_status;
+
+/* Largest number of draft-tree rows one call serves. */
+#define TL_NVFP4_MAX_M 32
+/* K must be a positive multiple of this. */
+#define TL_NVFP4_K_ALIGN 256
+/* Largest number of matrices one tl_nvfp4_verify_stack() call takes. */
+#define TL_NVFP4_MAX_STACK 1024
+
+/* Create the per-device state of `device` (workspace, status word). Idempotent.
+ * Does not change the calling thread's current device. */
+tl_status tl_init(int device);
+
+/* Free every per-device state. No call may be in flight. */
+void tl_shutdown(void);
+
+/* Y = X . dequant(W)^T for one weight matrix (see the top of this file).
+ *   x      device bf16 [M][K], 16-byte aligned
+ *   M      0..32 (0 is a no-op returning TL_OK; > 32 returns TL_ERR_UNSUPPORTED)
+ *   w_codes, w_scales  device, 16-byte aligned, layouts above
+ *   global_scale       finite
+ *   y      device bf16 [M][N], 16-byte aligned; must not overlap x or W
+ *   N      >= 1;  K  > 0 and K % 256 == 0
+ * Kernel: the tensor-core path (tcgen05, A = dequantised W in tensor memory,
+ * B = X in shared memory, fp32 accumulator in tensor memory), persistent
+ * stream-K over all SMs; split-K partials are combined in fixed k order. */
+tl_status tl_nvfp4_verify_gemm(const void* x, int M, const void* w_codes, const void* w_scales,
+                               float global_scale, void* y, int N, int K, void* stream);
+
+/* The same operation on CUDA cores only (one warp per weight row, fp32 FMA; no tensor
+ * cores, no workspace, no split-K). Same arguments, rules and determinism as
+ * tl_nvfp4_verify_gemm(); an independent second GPU path for cross-checks and for the
+ * smallest M, where the tensor-core tile is mostly padding. */
+tl_status tl_nvfp4_verify_gemm_simt(const void* x, int M, const void* w_codes, const void* w_scales,
+                                    float global_scale, void* y, int N, int K, void* stream);
+
+/* One matrix of a layer stack. Every matrix has its own X and Y. */
+typedef struct {
+    const void* w_codes;   /* device uint8 [N][K/2] */
+    const void* w_scales;  /* device uint8 [N][K/16] */
+    const void* x;         /* device bf16 [M][K] */
+    void* y;               /* device bf16 [M][N] */
+    float global_scale;
+    int N;
+    int K;
+} tl_nvfp4_matrix;
+
+/* The verify GEMM of `n_mats` independent matrices (e.g. QKV, O, gate+up and
+ * down of 64 layers) in one persistent launch: all matrices' k-tiles form one
+ * work list that is split evenly over the SMs, so no SM idles at a matrix
+ * boundary. `mats` is a HOST array read during the call; each entry obeys the
+ * rules of tl_nvfp4_verify_gemm(), with the same M for all. 1 <= n_mats <=
+ * TL_NVFP4_MAX_STACK. The matrices are independent: order of completion is
+ * unspecified; each Y is deterministic. */
+tl_status tl_nvfp4_verify_stack(const tl_nvfp4_matrix* mats, int n_mats, int M, void* stream);
+
+/* End-to-end form of tl_nvfp4_verify_stack() for callers whose X and Y live
+ * in host memory: copies X from `x_host` to `x_dev`, runs the stack, copies Y
+ * from `y_dev` to `y_host`, all on `stream` (asynchronous; pinned host memory
+ * makes the copies truly asynchronous). X_i (M x K_i bf16) sits at byte
+ * offset sum_{j<i} 2*M*K_j of x_host and x_dev; Y_i (M x N_i bf16) at offset
+ * sum_{j<i} 2*M*N_j of y_host and y_dev. The x and y fields of `mats` are
+ * ignored. Offsets of each X_i/Y_i must stay 16-byte aligned (M*K_i and
+ * M*N_i even multiples of 8 elements) or TL_ERR_MISALIGNED is returned. */
+tl_status tl_nvfp4_verify_stack_host(const tl_nvfp4_matrix* mats, int n_mats, int M,
+                                     const void* x_host, void* x_dev, void* y_host, void* y_dev,
+                                     void* stream);
+
+/* Plans: the descriptors of a stack built once, launched many times.
+ *
+ * tl_nvfp4_plan_create() validates `mats` (same rules as tl_nvfp4_verify_stack),
+ * encodes the TMA descriptors of every matrix and uploads them to the device once
+ * (synchronous; must not run during stream capture). The plan keeps no pointer to
+ * `mats`; it records the device pointers inside it, which must stay valid while the
+ * plan is used. tl_nvfp4_plan_run() then only launches: a few microseconds of host
+ * work, asynchronous on `stream`, and capturable into a CUDA graph.
+ * tl_nvfp4_plan_run_host() is the end-to-end form: it requires that the plan's X_i
+ * are packed back to back in one device buffer (X_{i+1} starts right after X_i) and
+ * likewise the Y_i, then copies all X from `x_host`, runs, and copies all Y to
+ * `y_host` (pinned host memory keeps the copies asynchronous); TL_ERR_INVALID_VALUE
+ * if the plan's buffers are not packed. Destroy synchronises the device before freeing.
+ * One plan must not run on two streams at once (the runs share the split-K workspace
+ * of the device; runs on one stream are ordered). */
+typedef struct tl_nvfp4_plan_st* tl_nvfp4_plan;
+tl_status tl_nvfp4_plan_create(const tl_nvfp4_matrix* mats, int n_mats, int M, tl_nvfp4_plan* plan_out);
+tl_status tl_nvfp4_plan_run(tl_nvfp4_plan plan, void* stream);
+tl_status tl_nvfp4_plan_run_host(tl_nvfp4_plan plan, const void* x_host, void* y_host, void* stream);
+tl_status tl_nvfp4_plan_destroy(tl_nvfp4_plan plan);
+
+/* Parity hook: w_out[n][k] = fp32(e2m1 * e4m3 * global_scale), rounded once
+ * (the product e2m1 * e4m3 is exact). w_out: device float [N][K], 16-byte
+ * aligned. Same size rules as tl_nvfp4_verify_gemm(). */
+tl_status tl_nvfp4_dequant(const void* w_codes, const void* w_scales, float global_scale,
+                           float* w_out, int N, int K, void* stream);
+
+/* Round-to-nearest NVFP4 quantiser (weight-pack builder):
+ *   g = fp32(absmax(w) / (6*448)); per 16-block s = E4M3_RNE_satfinite(absmax_block / 6 / g)
+ *   in fp64; codes = E2M1_RNE(w / (e4m3(s) * g)) in fp64, ties to the even code, zero -> 0x0.
+ * w: device float [N][K] (finite); codes/scales: device outputs as above.
+ * Writes g to *global_scale_out (host). SYNCHRONISES `stream` (it reads g back).
+ * Returns TL_ERR_NONFINITE, with outputs undefined, if w holds NaN or infinity. */
+tl_status tl_nvfp4_quantize(const float* w, int N, int K, void* w_codes, void* w_scales,
+                            float* global_scale_out, void* stream);
+
+/* Synchronise `stream`, then report and clear the device status word:
+ * TL_OK, TL_ERR_TIMEOUT (a bounded wait ran out) or TL_ERR_DEVICE_FAULT. */
+tl_status tl_check_device_error(void* stream);
+
+/* Self-test of the device-side failure path: launches one thread that waits, with the
+ * library's bounded wait, on an mbarrier that nothing completes, for at most
+ * `iterations` polls; when the limit runs out it records a timeout in the device
+ * status word and returns, leaving the context usable. The next
+ * tl_check_device_error() then reports TL_ERR_TIMEOUT. Touches no caller memory. */
+tl_status tl_selftest_bounded_wait(unsigned iterations, void* stream);
+
+/* Number of SMs the persistent kernels use on `device` (after tl_init). */
+int tl_num_sms(int device);
+
+/* Static strings; never NULL. */
+const char* tl_status_string(tl_status status);
+const char* tl_last_error_message(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TL_NVFP4_H */

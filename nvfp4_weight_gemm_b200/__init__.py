@@ -1,0 +1,132 @@
+"""NVFP4 verify GEMM for B200: Y[M,N] = X[M,K] . dequant(W)[N,K]^T, M <= 32.
+
+Thin Python layer over libtl_nvfp4.so (the C ABI in include/tl_nvfp4.h). Torch tensors
+are used for device memory and streams only; every step of the computation runs in the
+library's CUDA kernels. There is no CPU path.
+"""
+
+from __future__ import annotations
+
+import ctypes
+
+from . import _lib
+from ._lib import Matrix, TlError, check
+
+__all__ = ["verify_gemm", "verify_gemm_simt", "verify_stack", "verify_stack_host", "Plan", "dequant",
+           "quantize", "check_device_error", "init", "num_sms", "Matrix", "TlError"]
+
+
+def _stream(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t) -> ctypes.c_void_p:
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def init(device: int = 0) -> None:
+    check(_lib.lib().tl_init(device))
+
+
+def num_sms(device: int = 0) -> int:
+    return _lib.lib().tl_num_sms(device)
+
+
+def _gemm(name, x, codes, scales, global_scale, y=None, stream=None):
+    import torch
+    M, K = x.shape
+    N = codes.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    check(getattr(_lib.lib(), name)(_ptr(x), M, _ptr(codes), _ptr(scales), ctypes.c_float(global_scale),
+                                    _ptr(y), N, K, _stream(stream)))
+    return y
+
+
+def verify_gemm(x, codes, scales, global_scale, y=None, stream=None):
+    """Tensor-core path. x: bf16 [M, K]; codes: uint8 [N, K/2]; scales: uint8 [N, K/16]."""
+    return _gemm("tl_nvfp4_verify_gemm", x, codes, scales, global_scale, y, stream)
+
+
+def verify_gemm_simt(x, codes, scales, global_scale, y=None, stream=None):
+    """CUDA-core path (cross-check)."""
+    return _gemm("tl_nvfp4_verify_gemm_simt", x, codes, scales, global_scale, y, stream)
+
+
+def make_matrices(entries):
+    """entries: iterable of (codes, scales, global_scale, x, y) tensors -> ctypes array of Matrix."""
+    entries = list(entries)
+    arr = (Matrix * len(entries))()
+    for i, (c, s, g, x, y) in enumerate(entries):
+        arr[i] = Matrix(c.data_ptr(), s.data_ptr(), x.data_ptr() if x is not None else None,
+                        y.data_ptr() if y is not None else None, float(g), c.shape[0], c.shape[1] * 2)
+    return arr
+
+
+def verify_stack(mats, M: int, stream=None):
+    """mats: ctypes array from make_matrices (x and y set)."""
+    check(_lib.lib().tl_nvfp4_verify_stack(mats, len(mats), M, _stream(stream)))
+
+
+def verify_stack_host(mats, M: int, x_host, x_dev, y_host, y_dev, stream=None):
+    """End-to-end stack call: X from host memory in, Y to host memory out (contiguous buffers)."""
+    check(_lib.lib().tl_nvfp4_verify_stack_host(mats, len(mats), M, _ptr(x_host), _ptr(x_dev),
+                                                _ptr(y_host), _ptr(y_dev), _stream(stream)))
+
+
+class Plan:
+    """A stack whose descriptors are built once (tl_nvfp4_plan_create); run() only launches.
+
+    Keeps the ctypes matrix table and the tensors it points to alive while the plan lives."""
+
+    def __init__(self, entries, M: int):
+        self._entries = list(entries)
+        self._mats = make_matrices(self._entries)
+        self.M = M
+        h = ctypes.c_void_p()
+        check(_lib.lib().tl_nvfp4_plan_create(self._mats, len(self._mats), M, ctypes.byref(h)))
+        self._h = h
+
+    def run(self, stream=None):
+        check(_lib.lib().tl_nvfp4_plan_run(self._h, _stream(stream)))
+
+    def run_host(self, x_host, y_host, stream=None):
+        check(_lib.lib().tl_nvfp4_plan_run_host(self._h, _ptr(x_host), _ptr(y_host), _stream(stream)))
+
+    def close(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            _lib.lib().tl_nvfp4_plan_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def dequant(codes, scales, global_scale, out=None, stream=None):
+    import torch
+    N, K = codes.shape[0], codes.shape[1] * 2
+    if out is None:
+        out = torch.empty((N, K), dtype=torch.float32, device=codes.device)
+    check(_lib.lib().tl_nvfp4_dequant(_ptr(codes), _ptr(scales), ctypes.c_float(global_scale), _ptr(out), N, K,
+                                      _stream(stream)))
+    return out
+
+
+def quantize(w, stream=None):
+    """fp32 [N, K] device tensor -> (codes uint8 [N, K/2], scales uint8 [N, K/16], g). Synchronises."""
+    import torch
+    N, K = w.shape
+    codes = torch.empty((N, K // 2), dtype=torch.uint8, device=w.device)
+    scales = torch.empty((N, K // 16), dtype=torch.uint8, device=w.device)
+    g = ctypes.c_float(0.0)
+    check(_lib.lib().tl_nvfp4_quantize(_ptr(w), N, K, _ptr(codes), _ptr(scales), ctypes.byref(g), _stream(stream)))
+    return codes, scales, g.value
+
+
+def check_device_error(stream=None) -> None:
+    check(_lib.lib().tl_check_device_error(_stream(stream)))

@@ -1,0 +1,597 @@
+// tl_nvfp4_api.cu -- the C ABI of libtl_nvfp4.so (declared in include/tl_nvfp4.h).
+//
+// Host side of the NVFP4 verify GEMM: argument validation, per-device state (split-K
+// workspace, device status word), TMA descriptor construction, the stack descriptor
+// cache, and the kernel launches. No allocation happens on the GEMM path after the
+// per-device state and a stack's descriptor table exist.
+#include "tl_nvfp4.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "gemm_simt.cuh"
+#include "gemm_tc.cuh"
+#include "kernels_aux.cuh"
+
+namespace {
+
+thread_local char g_msg[512] = "no error";
+
+tl_status fail(tl_status st, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+tl_status fail(tl_status st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof g_msg, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+#define TL_CUDA(call)                                                                       \
+    do {                                                                                    \
+        cudaError_t e_ = (call);                                                            \
+        if (e_ != cudaSuccess)                                                              \
+            return fail(TL_ERR_CUDA, "%s failed: %s", #call, cudaGetErrorString(e_));        \
+    } while (0)
+
+constexpr int kMaxDevices = 64;
+constexpr int kStackCacheSlots = 8;
+
+struct StackCacheEntry {
+    std::vector<unsigned char> key;   // host bytes of the TcMat table
+    tl::TcMat* table = nullptr;       // device copy
+    unsigned long long last_use = 0;
+};
+
+struct DevState {
+    bool ready = false;
+    int num_sms = 0;
+    int* err = nullptr;            // device status word
+    float* partials = nullptr;     // [2 * num_sms][32][128]
+    unsigned* counters = nullptr;  // [4 * num_sms]
+    unsigned* qscratch = nullptr;  // quantiser absmax + non-finite flag
+    bool smem_attr_set = false;
+    StackCacheEntry cache[kStackCacheSlots];
+    unsigned long long use_clock = 0;
+};
+
+std::mutex g_mu;
+DevState g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+tl_status load_encode_fn() {
+    if (g_encode) return TL_OK;
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+        return fail(TL_ERR_CUDA, "cuTensorMapEncodeTiled unavailable from the driver");
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    return TL_OK;
+}
+
+// Create the state of `device` (caller holds g_mu). Switches device only temporarily.
+tl_status init_locked(int device) {
+    if (device < 0 || device >= kMaxDevices) return fail(TL_ERR_INVALID_VALUE, "device %d out of range", device);
+    DevState& d = g_dev[device];
+    if (d.ready) return TL_OK;
+    int prev = 0;
+    TL_CUDA(cudaGetDevice(&prev));
+    if (prev != device) TL_CUDA(cudaSetDevice(device));
+    tl_status st = TL_OK;
+    do {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, device) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) {
+            st = fail(TL_ERR_CUDA, "cannot query device %d", device);
+            break;
+        }
+        if (major != 10 || minor != 0) {
+            st = fail(TL_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a only", device,
+                      major, minor);
+            break;
+        }
+        d.num_sms = sms;
+        const size_t pbytes = (size_t)2 * sms * 32 * tl::TC_BLOCK_N * sizeof(float);
+        if (cudaMalloc(&d.err, 64) != cudaSuccess || cudaMalloc(&d.partials, pbytes) != cudaSuccess ||
+            cudaMalloc(&d.counters, (size_t)4 * sms * sizeof(unsigned)) != cudaSuccess ||
+            cudaMalloc(&d.qscratch, 64) != cudaSuccess) {
+            st = fail(TL_ERR_CUDA, "cudaMalloc of the per-device state failed");
+            break;
+        }
+        if (cudaMemset(d.err, 0, 64) != cudaSuccess ||
+            cudaMemset(d.counters, 0, (size_t)4 * sms * sizeof(unsigned)) != cudaSuccess ||
+            cudaDeviceSynchronize() != cudaSuccess) {
+            st = fail(TL_ERR_CUDA, "initialising the per-device state failed");
+            break;
+        }
+        d.ready = true;
+    } while (0);
+    if (prev != device) cudaSetDevice(prev);
+    return st;
+}
+
+tl_status current_state(DevState** out) {
+    int dev = 0;
+    TL_CUDA(cudaGetDevice(&dev));
+    std::lock_guard<std::mutex> lk(g_mu);
+    tl_status st = init_locked(dev);
+    if (st != TL_OK) return st;
+    st = load_encode_fn();
+    if (st != TL_OK) return st;
+    *out = &g_dev[dev];
+    return TL_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+// Shared checks of one matrix (M already checked).
+tl_status check_matrix(const void* x, int M, const void* codes, const void* scales, float g, const void* y, int N,
+                       int K, bool check_xy) {
+    if (N < 1) return fail(TL_ERR_INVALID_VALUE, "N = %d must be >= 1", N);
+    if (K <= 0 || K % TL_NVFP4_K_ALIGN != 0)
+        return fail(TL_ERR_INVALID_VALUE, "K = %d must be a positive multiple of %d", K, TL_NVFP4_K_ALIGN);
+    if (!codes || !scales) return fail(TL_ERR_INVALID_VALUE, "null weight pointer");
+    if (!std::isfinite(g)) return fail(TL_ERR_INVALID_VALUE, "global_scale is not finite");
+    if (!aligned16(codes) || !aligned16(scales))
+        return fail(TL_ERR_MISALIGNED, "weight pointers must be 16-byte aligned");
+    if (check_xy) {
+        if (!x || !y) return fail(TL_ERR_INVALID_VALUE, "null x or y pointer");
+        if (!aligned16(x) || !aligned16(y)) return fail(TL_ERR_MISALIGNED, "x and y must be 16-byte aligned");
+        const size_t ybytes = (size_t)M * N * 2;
+        if (overlap(y, ybytes, x, (size_t)M * K * 2) || overlap(y, ybytes, codes, (size_t)N * K / 2) ||
+            overlap(y, ybytes, scales, (size_t)N * K / 16))
+            return fail(TL_ERR_INVALID_VALUE, "y overlaps x or the weights");
+    }
+    return TL_OK;
+}
+
+tl_status encode_2d(CUtensorMap* tm, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(tm, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(TL_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return TL_OK;
+}
+
+tl_status build_mat(tl::TcMat* m, const void* x, int M, int NX, const void* codes, const void* scales, float g,
+                    void* y, int N, int K, long long tile_begin) {
+    memset(m, 0, sizeof *m);
+    tl_status st = encode_2d(&m->tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, (uint64_t)K / 2, (uint64_t)N,
+                             (uint64_t)K / 2, tl::TC_BLOCK_K / 2, tl::TC_BLOCK_N, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != TL_OK) return st;
+    st = encode_2d(&m->tm_scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, scales, (uint64_t)K / 16, (uint64_t)N,
+                   (uint64_t)K / 16, tl::TC_BLOCK_K / 16, tl::TC_BLOCK_N, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (st != TL_OK) return st;
+    st = encode_2d(&m->tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64,
+                   (uint32_t)NX, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (st != TL_OK) return st;
+    m->y = static_cast<__nv_bfloat16*>(y);
+    m->g_out = (float)((double)g * 128.0);   // W' reaches the accumulator scaled by 2^-7
+    m->N = N;
+    m->k_tiles = K / tl::TC_BLOCK_K;
+    m->n_tiles = (N + tl::TC_BLOCK_N - 1) / tl::TC_BLOCK_N;
+    m->tile_begin = tile_begin;
+    return TL_OK;
+}
+
+template <int NX>
+tl_status launch_tc(DevState& d, tl::TcParams& p, cudaStream_t stream) {
+    using C = tl::TcCfg<NX>;
+    // the attribute is per function; set for both variants on first use (idempotent, cheap)
+    TL_CUDA(cudaFuncSetAttribute(tl::gemm_tc_kernel<NX>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
+    const long long grid = p.total_tiles < d.num_sms ? p.total_tiles : d.num_sms;
+    p.partials = d.partials;
+    p.counters = d.counters;
+    p.err = d.err;
+    tl::gemm_tc_kernel<NX><<<(unsigned)grid, tl::TC_THREADS, C::SMEM_BYTES, stream>>>(p);
+    TL_CUDA(cudaGetLastError());
+    return TL_OK;
+}
+
+tl_status launch_tc_any(DevState& d, tl::TcParams& p, cudaStream_t stream) {
+    return (p.M <= 16) ? launch_tc<16>(d, p, stream) : launch_tc<32>(d, p, stream);
+}
+
+tl_status check_M(int M) {
+    if (M < 0) return fail(TL_ERR_INVALID_VALUE, "M = %d is negative", M);
+    if (M > TL_NVFP4_MAX_M) return fail(TL_ERR_UNSUPPORTED, "M = %d > %d rows is not served", M, TL_NVFP4_MAX_M);
+    return TL_OK;
+}
+
+// Device table of a stack's TcMat array: reused while the same matrices come back.
+tl_status stack_table(DevState& d, const std::vector<tl::TcMat>& mats, cudaStream_t stream, const tl::TcMat** out) {
+    const size_t bytes = mats.size() * sizeof(tl::TcMat);
+    const unsigned char* key = reinterpret_cast<const unsigned char*>(mats.data());
+    std::lock_guard<std::mutex> lk(g_mu);
+    ++d.use_clock;
+    for (auto& e : d.cache) {
+        if (e.table && e.key.size() == bytes && memcmp(e.key.data(), key, bytes) == 0) {
+            e.last_use = d.use_clock;
+            *out = e.table;
+            return TL_OK;
+        }
+    }
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    TL_CUDA(cudaStreamIsCapturing(stream, &cs));
+    if (cs != cudaStreamCaptureStatusNone)
+        return fail(TL_ERR_UNSUPPORTED, "a new stack must be run once before it is captured into a graph");
+    StackCacheEntry* victim = &d.cache[0];
+    for (auto& e : d.cache)
+        if (!e.table || e.last_use < victim->last_use) victim = &e;
+    if (victim->table) {
+        TL_CUDA(cudaDeviceSynchronize());   // the old table may be read by a kernel in flight
+        TL_CUDA(cudaFree(victim->table));
+        victim->table = nullptr;
+    }
+    TL_CUDA(cudaMalloc(&victim->table, bytes));
+    TL_CUDA(cudaMemcpy(victim->table, key, bytes, cudaMemcpyHostToDevice));
+    victim->key.assign(key, key + bytes);
+    victim->last_use = d.use_clock;
+    *out = victim->table;
+    return TL_OK;
+}
+
+// Validate a stack and build its launch parameters (host side only, plus the
+// state lookup). `table_out` receives the TcMat array when n_mats > 1.
+tl_status build_params(const tl_nvfp4_matrix* mats, int n_mats, int M, const unsigned char* x_dev,
+                       unsigned char* y_dev, DevState** dstate, tl::TcParams* p, std::vector<tl::TcMat>* table_out) {
+    tl_status st = check_M(M);
+    if (st != TL_OK) return st;
+    if (!mats) return fail(TL_ERR_INVALID_VALUE, "mats is null");
+    if (n_mats < 1 || n_mats > TL_NVFP4_MAX_STACK)
+        return fail(TL_ERR_INVALID_VALUE, "n_mats = %d outside [1, %d]", n_mats, TL_NVFP4_MAX_STACK);
+    // validate every matrix on the host before any CUDA call
+    size_t xoff = 0, yoff = 0;
+    for (int i = 0; i < n_mats; ++i) {
+        const tl_nvfp4_matrix& m = mats[i];
+        const void* x = x_dev ? static_cast<const void*>(x_dev + xoff) : m.x;
+        const void* y = y_dev ? static_cast<const void*>(y_dev + yoff) : m.y;
+        st = check_matrix(x, M, m.w_codes, m.w_scales, m.global_scale, y, m.N, m.K, true);
+        if (st != TL_OK) {
+            char why[sizeof g_msg];
+            memcpy(why, g_msg, sizeof why);
+            return fail(st, "matrix %d: %s", i, why);
+        }
+        xoff += (size_t)2 * M * m.K;
+        yoff += (size_t)2 * M * m.N;
+    }
+    if (M == 0) return TL_OK;
+    st = current_state(dstate);
+    if (st != TL_OK) return st;
+    const int NX = M <= 16 ? 16 : 32;
+    std::vector<tl::TcMat>& tbl = *table_out;
+    tbl.assign(n_mats, tl::TcMat());
+    long long tiles = 0;
+    xoff = 0;
+    yoff = 0;
+    for (int i = 0; i < n_mats; ++i) {
+        const tl_nvfp4_matrix& m = mats[i];
+        const void* x = x_dev ? static_cast<const void*>(x_dev + xoff) : m.x;
+        void* y = y_dev ? static_cast<void*>(y_dev + yoff) : m.y;
+        st = build_mat(&tbl[i], x, M, NX, m.w_codes, m.w_scales, m.global_scale, y, m.N, m.K, tiles);
+        if (st != TL_OK) return st;
+        tiles += (long long)tbl[i].n_tiles * tbl[i].k_tiles;
+        xoff += (size_t)2 * M * m.K;
+        yoff += (size_t)2 * M * m.N;
+    }
+    memset(p, 0, sizeof *p);
+    p->n_mats = n_mats;
+    p->M = M;
+    p->total_tiles = tiles;
+    p->mats = nullptr;
+    if (n_mats == 1) p->one = tbl[0];
+    return TL_OK;
+}
+
+tl_status run_stack(const tl_nvfp4_matrix* mats, int n_mats, int M, const unsigned char* x_dev,
+                    unsigned char* y_dev, void* stream_) {
+    DevState* d = nullptr;
+    tl::TcParams p;
+    std::vector<tl::TcMat> tbl;
+    tl_status st = build_params(mats, n_mats, M, x_dev, y_dev, &d, &p, &tbl);
+    if (st != TL_OK || M == 0) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    if (n_mats > 1) {
+        st = stack_table(*d, tbl, stream, &p.mats);
+        if (st != TL_OK) return st;
+    }
+    return launch_tc_any(*d, p, stream);
+}
+
+
+}  // namespace
+
+struct tl_nvfp4_plan_st {
+    int device = 0;
+    DevState* d = nullptr;
+    tl::TcParams params;
+    tl::TcMat* table = nullptr;       // device copy when n_mats > 1
+    const void* x_base = nullptr;     // packed X_i buffer (or nullptr if not packed)
+    void* y_base = nullptr;           // packed Y_i buffer (or nullptr if not packed)
+    size_t x_bytes = 0, y_bytes = 0;
+};
+
+extern "C" {
+
+tl_status tl_nvfp4_plan_create(const tl_nvfp4_matrix* mats, int n_mats, int M, tl_nvfp4_plan* plan_out) {
+    if (!plan_out) return fail(TL_ERR_INVALID_VALUE, "plan_out is null");
+    *plan_out = nullptr;
+    if (M == 0) return fail(TL_ERR_INVALID_VALUE, "a plan needs M >= 1");
+    DevState* d = nullptr;
+    tl::TcParams p;
+    std::vector<tl::TcMat> tbl;
+    tl_status st = build_params(mats, n_mats, M, nullptr, nullptr, &d, &p, &tbl);
+    if (st != TL_OK) return st;
+    tl_nvfp4_plan plan = new tl_nvfp4_plan_st();
+    TL_CUDA(cudaGetDevice(&plan->device));
+    plan->d = d;
+    plan->params = p;
+    if (n_mats > 1) {
+        const size_t bytes = tbl.size() * sizeof(tl::TcMat);
+        if (cudaMalloc(&plan->table, bytes) != cudaSuccess ||
+            cudaMemcpy(plan->table, tbl.data(), bytes, cudaMemcpyHostToDevice) != cudaSuccess) {
+            if (plan->table) cudaFree(plan->table);
+            delete plan;
+            return fail(TL_ERR_CUDA, "uploading the plan's descriptor table failed");
+        }
+        plan->params.mats = plan->table;
+    }
+    // packed X / Y buffers (needed by the host-buffer form only)
+    bool xpk = true, ypk = true;
+    const unsigned char* xb = static_cast<const unsigned char*>(mats[0].x);
+    const unsigned char* yb = static_cast<const unsigned char*>(mats[0].y);
+    size_t xo = 0, yo = 0;
+    for (int i = 0; i < n_mats; ++i) {
+        xpk = xpk && static_cast<const unsigned char*>(mats[i].x) == xb + xo;
+        ypk = ypk && static_cast<const unsigned char*>(mats[i].y) == yb + yo;
+        xo += (size_t)2 * M * mats[i].K;
+        yo += (size_t)2 * M * mats[i].N;
+    }
+    if (xpk) { plan->x_base = xb; plan->x_bytes = xo; }
+    if (ypk) { plan->y_base = (void*)yb; plan->y_bytes = yo; }
+    *plan_out = plan;
+    return TL_OK;
+}
+
+tl_status tl_nvfp4_plan_run(tl_nvfp4_plan plan, void* stream) {
+    if (!plan) return fail(TL_ERR_INVALID_VALUE, "plan is null");
+    tl::TcParams p = plan->params;
+    return launch_tc_any(*plan->d, p, static_cast<cudaStream_t>(stream));
+}
+
+tl_status tl_nvfp4_plan_run_host(tl_nvfp4_plan plan, const void* x_host, void* y_host, void* stream) {
+    if (!plan) return fail(TL_ERR_INVALID_VALUE, "plan is null");
+    if (!x_host || !y_host) return fail(TL_ERR_INVALID_VALUE, "null host buffer");
+    if (!plan->x_base || !plan->y_base)
+        return fail(TL_ERR_INVALID_VALUE, "the plan's X and Y buffers are not packed back to back");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    TL_CUDA(cudaMemcpyAsync(const_cast<void*>(plan->x_base), x_host, plan->x_bytes, cudaMemcpyHostToDevice, s));
+    tl::TcParams p = plan->params;
+    tl_status st = launch_tc_any(*plan->d, p, s);
+    if (st != TL_OK) return st;
+    TL_CUDA(cudaMemcpyAsync(y_host, plan->y_base, plan->y_bytes, cudaMemcpyDeviceToHost, s));
+    return TL_OK;
+}
+
+tl_status tl_nvfp4_plan_destroy(tl_nvfp4_plan plan) {
+    if (!plan) return TL_OK;
+    if (plan->table) {
+        int prev = 0;
+        cudaGetDevice(&prev);
+        cudaSetDevice(plan->device);
+        cudaDeviceSynchronize();
+        cudaFree(plan->table);
+        cudaSetDevice(prev);
+    }
+    delete plan;
+    return TL_OK;
+}
+
+tl_status tl_init(int device) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    tl_status st = init_locked(device);
+    if (st != TL_OK) return st;
+    return load_encode_fn();
+}
+
+void tl_shutdown(void) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    int prev = 0;
+    cudaGetDevice(&prev);
+    for (int i = 0; i < kMaxDevices; ++i) {
+        DevState& d = g_dev[i];
+        if (!d.ready) continue;
+        cudaSetDevice(i);
+        cudaDeviceSynchronize();
+        cudaFree(d.err);
+        cudaFree(d.partials);
+        cudaFree(d.counters);
+        cudaFree(d.qscratch);
+        for (auto& e : d.cache)
+            if (e.table) cudaFree(e.table);
+        d = DevState();
+    }
+    cudaSetDevice(prev);
+}
+
+tl_status tl_nvfp4_verify_gemm(const void* x, int M, const void* w_codes, const void* w_scales, float global_scale,
+                               void* y, int N, int K, void* stream) {
+    tl_status st = check_M(M);
+    if (st != TL_OK) return st;
+    st = check_matrix(x, M, w_codes, w_scales, global_scale, y, N, K, true);
+    if (st != TL_OK) return st;
+    if (M == 0) return TL_OK;
+    tl_nvfp4_matrix m{w_codes, w_scales, x, y, global_scale, N, K};
+    return run_stack(&m, 1, M, nullptr, nullptr, stream);
+}
+
+tl_status tl_nvfp4_verify_gemm_simt(const void* x, int M, const void* w_codes, const void* w_scales,
+                                    float global_scale, void* y, int N, int K, void* stream) {
+    tl_status st = check_M(M);
+    if (st != TL_OK) return st;
+    st = check_matrix(x, M, w_codes, w_scales, global_scale, y, N, K, true);
+    if (st != TL_OK) return st;
+    if (M == 0) return TL_OK;
+    DevState* d = nullptr;
+    st = current_state(&d);
+    if (st != TL_OK) return st;
+    const unsigned grid = (unsigned)((N + tl::SIMT_WARPS - 1) / tl::SIMT_WARPS);
+    auto xs = static_cast<const __nv_bfloat16*>(x);
+    auto cs = static_cast<const uint8_t*>(w_codes);
+    auto ss = static_cast<const uint8_t*>(w_scales);
+    auto ys = static_cast<__nv_bfloat16*>(y);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (M <= 8)
+        tl::gemm_simt_kernel<8><<<grid, tl::SIMT_WARPS * 32, 0, s>>>(xs, M, cs, ss, global_scale, ys, N, K);
+    else if (M <= 16)
+        tl::gemm_simt_kernel<16><<<grid, tl::SIMT_WARPS * 32, 0, s>>>(xs, M, cs, ss, global_scale, ys, N, K);
+    else
+        tl::gemm_simt_kernel<32><<<grid, tl::SIMT_WARPS * 32, 0, s>>>(xs, M, cs, ss, global_scale, ys, N, K);
+    TL_CUDA(cudaGetLastError());
+    return TL_OK;
+}
+
+tl_status tl_nvfp4_verify_stack(const tl_nvfp4_matrix* mats, int n_mats, int M, void* stream) {
+    return run_stack(mats, n_mats, M, nullptr, nullptr, stream);
+}
+
+tl_status tl_nvfp4_verify_stack_host(const tl_nvfp4_matrix* mats, int n_mats, int M, const void* x_host,
+                                     void* x_dev, void* y_host, void* y_dev, void* stream) {
+    tl_status st = check_M(M);
+    if (st != TL_OK) return st;
+    if (!mats || n_mats < 1 || n_mats > TL_NVFP4_MAX_STACK)
+        return fail(TL_ERR_INVALID_VALUE, "mats is null or n_mats = %d outside [1, %d]", n_mats, TL_NVFP4_MAX_STACK);
+    if (!x_host || !x_dev || !y_host || !y_dev) return fail(TL_ERR_INVALID_VALUE, "null host or device buffer");
+    if (M == 0) return TL_OK;
+    size_t xb = 0, yb = 0;
+    for (int i = 0; i < n_mats; ++i) {
+        if ((((size_t)M * mats[i].K) % 8) != 0 || (((size_t)M * mats[i].N) % 8) != 0)
+            return fail(TL_ERR_MISALIGNED, "matrix %d: M*K and M*N must be multiples of 8 elements", i);
+        if (mats[i].K < 0 || mats[i].N < 0) return fail(TL_ERR_INVALID_VALUE, "matrix %d: negative size", i);
+        xb += (size_t)2 * M * mats[i].K;
+        yb += (size_t)2 * M * mats[i].N;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    TL_CUDA(cudaMemcpyAsync(x_dev, x_host, xb, cudaMemcpyHostToDevice, s));
+    st = run_stack(mats, n_mats, M, static_cast<const unsigned char*>(x_dev), static_cast<unsigned char*>(y_dev),
+                   stream);
+    if (st != TL_OK) return st;
+    TL_CUDA(cudaMemcpyAsync(y_host, y_dev, yb, cudaMemcpyDeviceToHost, s));
+    return TL_OK;
+}
+
+tl_status tl_nvfp4_dequant(const void* w_codes, const void* w_scales, float global_scale, float* w_out, int N, int K,
+                           void* stream) {
+    tl_status st = check_matrix(nullptr, 0, w_codes, w_scales, global_scale, nullptr, N, K, false);
+    if (st != TL_OK) return st;
+    if (!w_out) return fail(TL_ERR_INVALID_VALUE, "w_out is null");
+    if (!aligned16(w_out)) return fail(TL_ERR_MISALIGNED, "w_out must be 16-byte aligned");
+    DevState* d = nullptr;
+    st = current_state(&d);
+    if (st != TL_OK) return st;
+    const long long blocks = (long long)N * (K / 16);
+    tl::dequant_kernel<<<(unsigned)((blocks + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint8_t*>(w_codes), static_cast<const uint8_t*>(w_scales), global_scale, blocks, w_out);
+    TL_CUDA(cudaGetLastError());
+    return TL_OK;
+}
+
+tl_status tl_nvfp4_quantize(const float* w, int N, int K, void* w_codes, void* w_scales, float* global_scale_out,
+                            void* stream) {
+    if (N < 1) return fail(TL_ERR_INVALID_VALUE, "N = %d must be >= 1", N);
+    if (K <= 0 || K % 16 != 0) return fail(TL_ERR_INVALID_VALUE, "K = %d must be a positive multiple of 16", K);
+    if (!w || !w_codes || !w_scales || !global_scale_out) return fail(TL_ERR_INVALID_VALUE, "null pointer");
+    if (!aligned16(w) || !aligned16(w_codes) || !aligned16(w_scales))
+        return fail(TL_ERR_MISALIGNED, "w, codes and scales must be 16-byte aligned");
+    DevState* d = nullptr;
+    tl_status st = current_state(&d);
+    if (st != TL_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const long long count = (long long)N * K;
+    TL_CUDA(cudaMemsetAsync(d->qscratch, 0, 8, s));
+    tl::absmax_kernel<<<(unsigned)(4 * d->num_sms), 512, 0, s>>>(w, count, d->qscratch);
+    TL_CUDA(cudaGetLastError());
+    unsigned h[2] = {0, 0};
+    TL_CUDA(cudaMemcpyAsync(h, d->qscratch, 8, cudaMemcpyDeviceToHost, s));
+    TL_CUDA(cudaStreamSynchronize(s));
+    if (h[1]) return fail(TL_ERR_NONFINITE, "w holds NaN or infinity");
+    float amax;
+    memcpy(&amax, &h[0], 4);
+    const float g = (float)((double)amax / (6.0 * 448.0));
+    const long long blocks = count / 16;
+    tl::quantize_kernel<<<(unsigned)((blocks + 255) / 256), 256, 0, s>>>(w, blocks, g, static_cast<uint8_t*>(w_codes),
+                                                                        static_cast<uint8_t*>(w_scales));
+    TL_CUDA(cudaGetLastError());
+    TL_CUDA(cudaStreamSynchronize(s));
+    *global_scale_out = g;
+    return TL_OK;
+}
+
+tl_status tl_check_device_error(void* stream) {
+    DevState* d = nullptr;
+    tl_status st = current_state(&d);
+    if (st != TL_OK) return st;
+    TL_CUDA(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+    int code = 0;
+    TL_CUDA(cudaMemcpy(&code, d->err, sizeof code, cudaMemcpyDeviceToHost));
+    if (code == 0) return TL_OK;
+    // a kernel that gave up may have left split-K counters raised: clear them for the next launch
+    TL_CUDA(cudaMemset(d->err, 0, sizeof code));
+    TL_CUDA(cudaMemset(d->counters, 0, (size_t)4 * d->num_sms * sizeof(unsigned)));
+    TL_CUDA(cudaDeviceSynchronize());
+    if ((code & 0xF00) == 0x100)
+        return fail(TL_ERR_TIMEOUT, "a device-side wait ran past its limit (code 0x%x)", code);
+    return fail(TL_ERR_DEVICE_FAULT, "device status word 0x%x", code);
+}
+
+tl_status tl_selftest_bounded_wait(unsigned iterations, void* stream) {
+    DevState* d = nullptr;
+    tl_status st = current_state(&d);
+    if (st != TL_OK) return st;
+    tl::selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(iterations, d->err);
+    TL_CUDA(cudaGetLastError());
+    return TL_OK;
+}
+
+int tl_num_sms(int device) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (device < 0 || device >= kMaxDevices || !g_dev[device].ready) return 0;
+    return g_dev[device].num_sms;
+}
+
+const char* tl_status_string(tl_status s) {
+    switch (s) {
+        case TL_OK: return "TL_OK";
+        case TL_ERR_INVALID_VALUE: return "TL_ERR_INVALID_VALUE";
+        case TL_ERR_MISALIGNED: return "TL_ERR_MISALIGNED";
+        case TL_ERR_UNSUPPORTED: return "TL_ERR_UNSUPPORTED";
+        case TL_ERR_CUDA: return "TL_ERR_CUDA";
+        case TL_ERR_TIMEOUT: return "TL_ERR_TIMEOUT";
+        case TL_ERR_NOT_INITIALIZED: return "TL_ERR_NOT_INITIALIZED";
+        case TL_ERR_NONFINITE: return "TL_ERR_NONFINITE";
+        case TL_ERR_DEVICE_FAULT: return "TL_ERR_DEVICE_FAULT";
+    }
+    return "TL_ERR_UNKNOWN";
+}
+
+const char* tl_last_error_message(void) { return g_msg; }
+
+}  // extern "C"

@@ -1,0 +1,323 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the same seeded inputs.
+
+Bars (all written here):
+  * dequantised weights and quantiser output: bit-exact;
+  * Y: |y - y_ref| <= 1e-3 * sum_k |x_k w_k| + 2^-8 * |y_ref| per element (fp32 accumulation,
+    one bf16 rounding: the 2^-8 term covers the output rounding);
+  * cases whose exact result is representable (identity, one-hot, small integers): bit-exact
+    against bf16(y_ref);
+  * determinism: repeated runs bit-identical.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():  # collected on CPU hosts, skipped there
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import nvfp4_weight_gemm_b200 as tl  # noqa: E402
+
+DEV = torch.device("cuda:0")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _init():
+    from nvfp4_weight_gemm_b200 import build
+    build.build()
+    oracle.build()
+    tl.init(0)
+    yield
+    tl.check_device_error()
+
+
+# ------------------------------------------------------------------ helpers
+
+def dev_u8(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+
+
+def dev_bf16(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(DEV).view(torch.bfloat16)
+
+
+def host_f64(y):
+    return y.float().cpu().numpy().astype(np.float64)
+
+
+def bf16_round(a):
+    """bf16(a) for fp64 values that are exact in fp32 (no double rounding then)."""
+    return torch.from_numpy(np.asarray(a, dtype=np.float64)).float().to(torch.bfloat16).double().numpy()
+
+
+def assert_within_tol(y, y_ref, a_ref, what=""):
+    tol = 1e-3 * a_ref + 2.0 ** -8 * np.abs(y_ref)
+    err = np.abs(y - y_ref)
+    bad = err > tol
+    assert not bad.any(), (f"{what}: {bad.sum()} of {bad.size} outside tolerance; worst excess "
+                           f"{np.max(err - tol):.3e} at {np.unravel_index(np.argmax(err - tol), err.shape)}")
+
+
+def make_weight(N, K, seed, tid, dist="normal"):
+    w = synth.w_f32(N, K, seed=seed, tensor_id=tid, dist=dist)
+    codes, scales, g = oracle.quantize(w)
+    return w, codes, scales, g
+
+
+def run_both_paths(x_bits, codes, scales, g):
+    x = dev_bf16(x_bits)
+    c, s = dev_u8(codes), dev_u8(scales)
+    y_tc = tl.verify_gemm(x, c, s, g)
+    y_simt = tl.verify_gemm_simt(x, c, s, g)
+    torch.cuda.synchronize()
+    tl.check_device_error()
+    return host_f64(y_tc), host_f64(y_simt)
+
+
+# ------------------------------------------------------------------ format kernels
+
+def test_dequant_bit_exact_tiny():
+    _, codes, scales, g = make_weight(256, 512, 0, 0)
+    w_ref = oracle.dequant(codes, scales, g)
+    w_gpu = tl.dequant(dev_u8(codes), dev_u8(scales), g).cpu().numpy()
+    assert np.array_equal(w_gpu.view(np.uint32), w_ref.view(np.uint32))
+
+
+def test_dequant_bit_exact_all_bytes():
+    rng = np.random.default_rng(3)
+    N, K = 64, 4096
+    codes = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    scales = np.tile(np.arange(256, dtype=np.uint8), N * (K // 16) // 256).reshape(N, K // 16)
+    for g in (1.0, float(np.float32(0.0123)), float(np.float32(3.7e-39))):
+        w_ref = oracle.dequant(codes, scales, g)
+        w_gpu = tl.dequant(dev_u8(codes), dev_u8(scales), g).cpu().numpy()
+        same = (w_gpu.view(np.uint32) == w_ref.view(np.uint32)) | (np.isnan(w_gpu) & np.isnan(w_ref))
+        assert same.all(), g
+
+
+@pytest.mark.parametrize("N,K,dist", [(256, 512, "normal"), (677, 2304, "normal"), (640, 4096, "t4"),
+                                      (5120, 5120, "normal")])
+def test_quantize_bit_exact(N, K, dist):
+    w = synth.w_f32(N, K, seed=1, tensor_id=N + K, dist=dist)
+    codes, scales, g = oracle.quantize(w)
+    c2, s2, g2 = tl.quantize(torch.from_numpy(w).to(DEV))
+    assert g2 == g
+    assert np.array_equal(s2.cpu().numpy(), scales)
+    assert np.array_equal(c2.cpu().numpy(), codes)
+
+
+def test_quantize_special_tensors():
+    c, s, g = tl.quantize(torch.zeros((16, 256), device=DEV))
+    assert g == 0.0 and not c.any() and not s.any()
+    w = torch.ones((16, 256), device=DEV)
+    w[3, 17] = float("nan")
+    with pytest.raises(tl.TlError):
+        tl.quantize(w)
+
+
+# ------------------------------------------------------------------ GEMM parity
+
+def test_tiny_config_both_paths():
+    _, codes, scales, g = make_weight(256, 512, 0, 0)
+    x = synth.x_bf16(8, 512, seed=0)
+    y_ref, a_ref = oracle.gemm(x, codes, scales, g)
+    y_tc, y_simt = run_both_paths(x, codes, scales, g)
+    assert_within_tol(y_tc, y_ref, a_ref, "tensor-core")
+    assert_within_tol(y_simt, y_ref, a_ref, "simt")
+
+
+@pytest.mark.parametrize("M", [1, 2, 7, 8, 15, 16, 17, 24, 31, 32])
+def test_ragged_split_k_all_row_counts(M):
+    # 6 n-tiles (last one 37 rows), 9 k-tiles: every n-tile is split over several CTAs
+    _, codes, scales, g = make_weight(677, 2304, 2, 1)
+    x = synth.x_bf16(M, 2304, seed=2, tensor_id=synth.X_ID_BASE + M)
+    y_ref, a_ref = oracle.gemm(x, codes, scales, g)
+    y_tc, y_simt = run_both_paths(x, codes, scales, g)
+    assert_within_tol(y_tc, y_ref, a_ref, f"tensor-core M={M}")
+    assert_within_tol(y_simt, y_ref, a_ref, f"simt M={M}")
+
+
+@pytest.mark.parametrize("M", [1, 8, 16, 24, 32])
+def test_attention_projection_full(M):
+    _, codes, scales, g = make_weight(5120, 5120, 0, 2)
+    x = synth.x_bf16(M, 5120, seed=0, tensor_id=synth.X_ID_BASE + 2)
+    y_ref, a_ref = oracle.gemm(x, codes, scales, g)
+    y = host_f64(tl.verify_gemm(dev_bf16(x), dev_u8(codes), dev_u8(scales), g))
+    tl.check_device_error()
+    assert_within_tol(y, y_ref, a_ref, f"attn M={M}")
+
+
+def _sampled_check(N, K, dist, Ms, tid):
+    _, codes, scales, g = make_weight(N, K, 0, tid, dist)
+    c, s = dev_u8(codes), dev_u8(scales)
+    rng = np.random.default_rng(tid)
+    for M in Ms:
+        x = synth.x_bf16(M, K, seed=0, tensor_id=synth.X_ID_BASE + tid)
+        y = host_f64(tl.verify_gemm(dev_bf16(x), c, s, g))
+        tl.check_device_error()
+        mi = rng.integers(0, M, 4096)
+        ni = np.concatenate([rng.integers(0, N, 4000), np.arange(N - 96, N)])
+        y_ref, a_ref = oracle.gemm_sampled(x, codes, scales, g, mi, ni)
+        assert_within_tol(y[mi, ni], y_ref, a_ref, f"{N}x{K} M={M}")
+        assert np.isfinite(y).all()
+
+
+def test_mlp_gate_up_sampled():
+    _sampled_check(34816, 5120, "normal", [1, 13, 32], 10)
+
+
+def test_mlp_down_heavy_tail_sampled():
+    _sampled_check(5120, 17408, "t4", [1, 19, 32], 11)
+
+
+# ------------------------------------------------------------------ exact special cases
+
+def test_identity_weight_returns_x_exactly():
+    K = 512
+    codes = np.zeros((K, K // 2), dtype=np.uint8)
+    for n in range(K):
+        codes[n, n // 2] = 0x02 if n % 2 == 0 else 0x20
+    scales = np.full((K, K // 16), 0x38, dtype=np.uint8)
+    for M in (3, 32):
+        x = synth.x_bf16(M, K, seed=5, tensor_id=M)
+        y_tc, y_simt = run_both_paths(x, codes, scales, 1.0)
+        xf = synth.bf16_bits_to_f32(x).astype(np.float64)
+        assert np.array_equal(y_tc, xf) and np.array_equal(y_simt, xf)
+
+
+def test_one_hot_weight_exact():
+    rng = np.random.default_rng(8)
+    K = N = 1024
+    perm = rng.permutation(K)
+    codes = np.zeros((N, K // 2), dtype=np.uint8)
+    for n in range(N):
+        k = perm[n]
+        codes[n, k // 2] |= (0xD if k % 2 == 0 else 0xD0)   # -3.0
+    scales = np.full((N, K // 16), 0x30, dtype=np.uint8)    # 0.5
+    x = synth.x_bf16(20, K, seed=6)
+    y_ref, _ = oracle.gemm(x, codes, scales, 0.25)
+    y_tc, y_simt = run_both_paths(x, codes, scales, 0.25)
+    want = bf16_round(y_ref)
+    assert np.array_equal(y_tc, want) and np.array_equal(y_simt, want)
+
+
+def test_small_integer_exact():
+    rng = np.random.default_rng(9)
+    M, N, K = 32, 384, 1024
+    x = synth.f32_to_bf16_bits(rng.integers(-4, 5, (M, K)).astype(np.float32))
+    codes = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    scales = np.full((N, K // 16), 0x38, dtype=np.uint8)
+    g = 2.0 ** -3
+    y_ref, _ = oracle.gemm(x, codes, scales, g)
+    y_tc, y_simt = run_both_paths(x, codes, scales, g)
+    want = bf16_round(y_ref)
+    assert np.array_equal(y_tc, want) and np.array_equal(y_simt, want)
+
+
+def test_subnormal_scales_and_zero_blocks():
+    # scales across the whole E4M3 range, including subnormals and zero, with random codes
+    rng = np.random.default_rng(12)
+    M, N, K = 9, 256, 2048
+    codes = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    scales = rng.integers(0, 0x7F, (N, K // 16), dtype=np.uint8)
+    scales[:, ::7] = rng.integers(0, 8, scales[:, ::7].shape)
+    x = synth.x_bf16(M, K, seed=12)
+    y_ref, a_ref = oracle.gemm(x, codes, scales, 0.5)
+    y_tc, y_simt = run_both_paths(x, codes, scales, 0.5)
+    assert_within_tol(y_tc, y_ref, a_ref, "tensor-core")
+    assert_within_tol(y_simt, y_ref, a_ref, "simt")
+
+
+# ------------------------------------------------------------------ determinism, stack, host path
+
+def test_repeat_runs_bit_identical():
+    _, codes, scales, g = make_weight(677, 2304, 2, 1)
+    x = dev_bf16(synth.x_bf16(32, 2304, seed=4))
+    c, s = dev_u8(codes), dev_u8(scales)
+    first = tl.verify_gemm(x, c, s, g).clone()
+    for _ in range(5):
+        assert torch.equal(tl.verify_gemm(x, c, s, g), first)
+    tl.check_device_error()
+
+
+def _small_stack(M, n_layers=3):
+    shapes = [(384, 1024), (256, 1024), (1280, 1024), (256, 2560)]
+    ents, refs = [], []
+    for layer in range(n_layers):
+        for j, (N, K) in enumerate(shapes):
+            tid = 100 + 4 * layer + j
+            _, codes, scales, g = make_weight(N, K, 3, tid, "t4" if j == 3 else "normal")
+            x = synth.x_bf16(M, K, seed=3, tensor_id=synth.X_ID_BASE + tid)
+            y_ref, a_ref = oracle.gemm(x, codes, scales, g)
+            ents.append((dev_u8(codes), dev_u8(scales), g, dev_bf16(x),
+                         torch.empty((M, N), dtype=torch.bfloat16, device=DEV)))
+            refs.append((y_ref, a_ref, x))
+    return ents, refs
+
+
+@pytest.mark.parametrize("M", [8, 24])
+def test_stack_matches_oracle_and_single_calls(M):
+    ents, refs = _small_stack(M)
+    mats = tl.make_matrices(ents)
+    tl.verify_stack(mats, M)
+    torch.cuda.synchronize()
+    tl.check_device_error()
+    for (c, s, g, x, y), (y_ref, a_ref, _) in zip(ents, refs):
+        assert_within_tol(host_f64(y), y_ref, a_ref, "stack")
+    # the cached descriptor table is reused on the second call: same results
+    ys = [e[4].clone() for e in ents]
+    tl.verify_stack(mats, M)
+    for e, y0 in zip(ents, ys):
+        assert torch.equal(e[4], y0)
+
+
+def test_stack_host_buffers_end_to_end():
+    M = 16
+    ents, refs = _small_stack(M, n_layers=2)
+    xs = torch.cat([e[3].reshape(-1) for e in ents]).cpu().pin_memory()
+    ytot = sum(e[4].numel() for e in ents)
+    x_dev = torch.empty_like(xs, device=DEV)
+    y_dev = torch.empty(ytot, dtype=torch.bfloat16, device=DEV)
+    y_host = torch.empty(ytot, dtype=torch.bfloat16).pin_memory()
+    mats = tl.make_matrices([(c, s, g, None, None) for c, s, g, _, _ in ents])
+    tl.verify_stack_host(mats, M, xs, x_dev, y_host, y_dev)
+    torch.cuda.synchronize()
+    tl.check_device_error()
+    off = 0
+    for (c, s, g, x, y), (y_ref, a_ref, _) in zip(ents, refs):
+        n = y.numel()
+        got = y_host[off:off + n].view(y.shape).float().numpy().astype(np.float64)
+        assert_within_tol(got, y_ref, a_ref, "stack host")
+        off += n
+
+
+# ------------------------------------------------------------------ failure path
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    from nvfp4_weight_gemm_b200 import _lib
+    tl.check_device_error()
+    _lib.check(_lib.lib().tl_selftest_bounded_wait(1000, None))
+    with pytest.raises(tl.TlError) as ei:
+        tl.check_device_error()
+    assert ei.value.status == 5
+    tl.check_device_error()  # cleared
+    _, codes, scales, g = make_weight(256, 512, 0, 0)
+    x = synth.x_bf16(8, 512, seed=0)
+    y_ref, a_ref = oracle.gemm(x, codes, scales, g)
+    y_tc, _ = run_both_paths(x, codes, scales, g)
+    assert_within_tol(y_tc, y_ref, a_ref, "after timeout")
+
+
+def test_zero_rows_is_a_no_op():
+    y = torch.full((1, 256), 7.0, dtype=torch.bfloat16, device=DEV)
+    from nvfp4_weight_gemm_b200 import _lib
+    import ctypes
+    st = _lib.lib().tl_nvfp4_verify_gemm(ctypes.c_void_p(y.data_ptr()), 0, ctypes.c_void_p(y.data_ptr() + 4096),
+                                         ctypes.c_void_p(y.data_ptr() + 8192), ctypes.c_float(1.0),
+                                         ctypes.c_void_p(y.data_ptr()), 256, 512, None)
+    assert st == 0 and bool((y == 7.0).all())
