@@ -17,6 +17,8 @@
 //     and stores it into tensor memory, the A operand. Warp 1 issues tcgen05.mma with
 //     A from tensor memory, B = X tile (bf16, shared memory, 128-byte swizzle) and the
 //     fp32 accumulator in tensor memory (M_mma = 128 weight rows, N_mma = 16 or 32 X rows).
+//     The dequantisers form two groups of four warps that take alternate tiles, so one
+//     group's tensor-memory stores overlap the other group's decode.
 //     Warps 12..15 read the accumulator and write Y (or a partial).
 //   * Dequantisation without a table. For code c = s e1 e0 m, the bf16 bit pattern
 //     (e1 e0 m) << 6 | s << 15 is exactly e2m1(c) * 2^-126 (code 1 lands on a bf16
@@ -38,12 +40,22 @@
 
 namespace tl {
 
+// Independent accumulators per output tile: consecutive k-steps of a tile go to
+// different accumulators (k-step i -> accumulator i % TC_NACC) so that successive MMAs
+// do not wait on each other; the epilogue adds them in a fixed order.
+#ifndef TL_TC_NACC
+#define TL_TC_NACC 2
+#endif
+
 constexpr int TC_BLOCK_N = 128;        // weight rows per tile (MMA M)
 constexpr int TC_BLOCK_K = 256;        // k per tile / pipeline stage
-constexpr int TC_NUM_A = 3;            // tensor-memory A buffers (128 columns each)
+constexpr int TC_NACC = TL_TC_NACC;
+constexpr int TC_NUM_A = TC_NACC >= 4 ? 2 : 3;   // tensor-memory A buffers (128 columns each)
 constexpr int TC_THREADS = 512;
 constexpr int TC_TMEM_COLS = 512;
 constexpr int TC_ACC_COL0 = 128 * TC_NUM_A;   // accumulators after the A buffers
+constexpr int TC_ACC_COLS = 32 * TC_NACC;     // one accumulator buffer: TC_NACC x 32 fp32 columns
+static_assert(TC_ACC_COL0 + 2 * TC_ACC_COLS <= TC_TMEM_COLS, "tensor memory budget");
 
 enum : int {
     TL_DEV_ERR_TIMEOUT_PRODUCER = 0x101,
@@ -183,7 +195,7 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
     uint64_t* full = bars;                          // [STAGES] TMA bytes landed
     uint64_t* empty = full + C::STAGES;             // [STAGES] stage consumed (MMA commit)
-    uint64_t* aready = empty + C::STAGES;           // [NUM_A] A buffer written (8 warps)
+    uint64_t* aready = empty + C::STAGES;           // [NUM_A] A buffer written (4 warps of a group)
     uint64_t* afree = aready + TC_NUM_A;            // [NUM_A] A buffer read by MMA (commit)
     uint64_t* accfull = afree + TC_NUM_A;           // [2] accumulator complete (commit)
     uint64_t* accempty = accfull + 2;               // [2] accumulator read (4 warps)
@@ -200,7 +212,7 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-        for (int i = 0; i < TC_NUM_A; ++i) { mbar_init(&aready[i], 8); mbar_init(&afree[i], 1); }
+        for (int i = 0; i < TC_NUM_A; ++i) { mbar_init(&aready[i], 4); mbar_init(&afree[i], 1); }
         for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], 4); }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -268,7 +280,7 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem + (uint32_t)(TC_ACC_COL0 + 32 * acc);
+                const uint32_t d_tmem = tmem + (uint32_t)(TC_ACC_COL0 + TC_ACC_COLS * acc);
                 for (int kt = sg.k0; kt < sg.k1; ++kt) {
                     if (*abort_flag || !mbar_wait(&full[s], ph, TL_WAIT_LIMIT) ||
                         !mbar_wait(&aready[a], aph, TL_WAIT_LIMIT)) {
@@ -282,7 +294,8 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
 #pragma unroll
                     for (int i = 0; i < TC_BLOCK_K / 16; ++i) {
                         const uint64_t bdesc = smem_desc_k_sw128(xs + (i >> 2) * C::X_SUB + (i & 3) * 32);
-                        mma_ts_f16(d_tmem, a_tmem + 8u * i, bdesc, C::IDESC, (kt > sg.k0 || i > 0) ? 1u : 0u);
+                        mma_ts_f16(d_tmem + 32u * (uint32_t)(i % TC_NACC), a_tmem + 8u * i, bdesc, C::IDESC,
+                                   (kt > sg.k0 || i >= TC_NACC) ? 1u : 0u);
                     }
                     mma_commit(&empty[s]);
                     mma_commit(&afree[a]);
@@ -299,17 +312,24 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
         }
     } else if (warp >= 4 && warp < 12) {
         // ------------------------------------------------------------ dequantisers
-        const int h = (warp - 4) >> 2;           // which 128-k half of the tile
+        // Two groups of four warps take alternate tiles (group g: tiles c with c % 2 == g),
+        // so one group's tensor-memory store latency overlaps the other group's decode.
+        // Thread r of a group owns weight row r of the tile and decodes all 256 k of it.
+        const int grp = (warp - 4) >> 2;
         const int q = warp & 3;                  // tensor-memory lane quarter
         const int r = 32 * q + lane;             // weight row within the tile
         const uint32_t t_lane = tmem + ((uint32_t)(32 * q) << 16);
-        int s = 0, a = 0;
-        uint32_t ph = 0, aph = 0;
+        long long c = 0;                          // tile counter of this CTA
         TcSegIter it(mats, p.n_mats, t_begin, t_end);
         TcSeg sg;
         bool ok = true;
         while (ok && it.next(sg)) {
-            for (int kt = sg.k0; kt < sg.k1; ++kt) {
+            for (int kt = sg.k0; kt < sg.k1; ++kt, ++c) {
+                if ((int)(c & 1) != grp) continue;
+                const int s = (int)(c % C::STAGES);
+                const uint32_t ph = (uint32_t)((c / C::STAGES) & 1);
+                const int a = (int)(c % TC_NUM_A);
+                const uint32_t aph = (uint32_t)((c / TC_NUM_A) & 1);
                 if (*abort_flag || !mbar_wait(&full[s], ph, TL_WAIT_LIMIT) ||
                     !mbar_wait(&afree[a], aph ^ 1u, TL_WAIT_LIMIT)) {
                     tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_DEQUANT);
@@ -318,32 +338,33 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
                 }
                 tc_fence_after();
                 const uint8_t* st = smem + s * C::STAGE_BYTES;
-                uint4 c[4];
+                const uint4 sc = *reinterpret_cast<const uint4*>(st + C::CODES_BYTES + C::X_BYTES + r * 16);
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    const int j = 4 * h + jj;
-                    c[jj] = *reinterpret_cast<const uint4*>(st + r * 128 + ((j ^ (r & 7)) << 4));
-                }
-                const uint2 sc = *reinterpret_cast<const uint2*>(st + C::CODES_BYTES + C::X_BYTES + r * 16 + 8 * h);
-                uint32_t S[8];
-                scales8_to_bf16x2(sc, S);
-                uint32_t out[64];
+                for (int h = 0; h < 2; ++h) {   // two 128-k halves: 64 code bytes, 8 scales each
+                    uint4 cw[4];
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    decode8(c[jj].x, S[2 * jj], &out[16 * jj + 0]);
-                    decode8(c[jj].y, S[2 * jj], &out[16 * jj + 4]);
-                    decode8(c[jj].z, S[2 * jj + 1], &out[16 * jj + 8]);
-                    decode8(c[jj].w, S[2 * jj + 1], &out[16 * jj + 12]);
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const int j = 4 * h + jj;
+                        cw[jj] = *reinterpret_cast<const uint4*>(st + r * 128 + ((j ^ (r & 7)) << 4));
+                    }
+                    uint32_t S[8];
+                    scales8_to_bf16x2(h == 0 ? make_uint2(sc.x, sc.y) : make_uint2(sc.z, sc.w), S);
+                    uint32_t out[64];
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        decode8(cw[jj].x, S[2 * jj], &out[16 * jj + 0]);
+                        decode8(cw[jj].y, S[2 * jj], &out[16 * jj + 4]);
+                        decode8(cw[jj].z, S[2 * jj + 1], &out[16 * jj + 8]);
+                        decode8(cw[jj].w, S[2 * jj + 1], &out[16 * jj + 12]);
+                    }
+                    const uint32_t col = (uint32_t)(128 * a + 64 * h);
+                    tmem_st32(t_lane + col, *reinterpret_cast<const uint32_t(*)[32]>(&out[0]));
+                    tmem_st32(t_lane + col + 32, *reinterpret_cast<const uint32_t(*)[32]>(&out[32]));
                 }
-                const uint32_t col = (uint32_t)(128 * a + 64 * h);
-                tmem_st32(t_lane + col, *reinterpret_cast<const uint32_t(*)[32]>(&out[0]));
-                tmem_st32(t_lane + col + 32, *reinterpret_cast<const uint32_t(*)[32]>(&out[32]));
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&aready[a]);
-                if (++s == C::STAGES) { s = 0; ph ^= 1u; }
-                if (++a == TC_NUM_A) { a = 0; aph ^= 1u; }
             }
         }
     } else if (warp >= 12) {
@@ -363,14 +384,17 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
             }
             tc_fence_after();
             float v[NX];
-            {
+#pragma unroll
+            for (int i = 0; i < NX; ++i) v[i] = 0.0f;
+#pragma unroll
+            for (int j = 0; j < TC_NACC; ++j) {   // fixed order: accumulator 0, 1, ...
                 uint32_t raw[16];
 #pragma unroll
                 for (int c0 = 0; c0 < NX; c0 += 16) {
-                    tmem_ld16(t_lane + (uint32_t)(TC_ACC_COL0 + 32 * acc + c0), raw);
+                    tmem_ld16(t_lane + (uint32_t)(TC_ACC_COL0 + TC_ACC_COLS * acc + 32 * j + c0), raw);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) v[c0 + i] = __uint_as_float(raw[i]);
+                    for (int i = 0; i < 16; ++i) v[c0 + i] += __uint_as_float(raw[i]);
                 }
             }
             tc_fence_before();
