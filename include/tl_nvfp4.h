@@ -95,6 +95,30 @@ tl_status tl_nvfp4_verify_gemm(const void* x, int M, const void* w_codes, const 
 tl_status tl_nvfp4_verify_gemm_simt(const void* x, int M, const void* w_codes, const void* w_scales,
                                     float global_scale, void* y, int N, int K, void* stream);
 
+/* tl_nvfp4_verify_gemm() for callers that cannot allocate device memory. The paper has
+ * no counterpart to this entry point; it exists for deployment.
+ *
+ * Who needs it: a serving engine that gives all free HBM to its KV-cache pool at start-up
+ * leaves nothing for a library's first-call workspace, and some host runtimes route all
+ * device memory through their own pool and do not let a library call cudaMalloc. This
+ * call allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ *
+ * Same arguments, rules, kernel and results as tl_nvfp4_verify_gemm(). Its split-K
+ * scratch is one static device array inside this library, 5 MiB (partials for up to
+ * 160 CTAs, their counters, a status word), which every GPU that loads the library holds
+ * until the process exits. Limits: M <= 32 (larger M returns TL_ERR_UNSUPPORTED with a
+ * message); the grid is capped at 160 CTAs.
+ *
+ * The first call on a device does a one-time set-up with that device current (it looks up
+ * the array's device address and the SM count); make that first call before capturing a
+ * stream into a graph. Every call shares the one array and each launch clears its counters
+ * first, so calls whose kernels overlap on the GPU (different streams, or several host
+ * threads without ordering) race and give undefined results: keep them on one stream.
+ * A device-side wait that runs out is recorded only in the array's own status word, not
+ * reported by tl_check_device_error(). */
+tl_status tl_nvfp4_verify_gemm_noalloc(const void* x, int M, const void* w_codes, const void* w_scales,
+                                       float global_scale, void* y, int N, int K, void* stream);
+
 /* One matrix of a layer stack. Every matrix has its own X and Y. */
 typedef struct {
     const void* w_codes;   /* device uint8 [N][K/2] */

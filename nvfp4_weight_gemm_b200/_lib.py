@@ -22,7 +22,7 @@ STATUS = {
 
 # Every symbol include/tl_nvfp4.h declares.
 EXPORTS = (
-    "tl_init", "tl_shutdown", "tl_nvfp4_verify_gemm", "tl_nvfp4_verify_gemm_simt",
+    "tl_init", "tl_shutdown", "tl_nvfp4_verify_gemm", "tl_nvfp4_verify_gemm_simt", "tl_nvfp4_verify_gemm_noalloc",
     "tl_nvfp4_verify_stack", "tl_nvfp4_verify_stack_host", "tl_nvfp4_plan_create",
     "tl_nvfp4_plan_run", "tl_nvfp4_plan_run_host", "tl_nvfp4_plan_destroy", "tl_nvfp4_dequant",
     "tl_nvfp4_quantize", "tl_check_device_error", "tl_selftest_bounded_wait", "tl_num_sms", "tl_status_string",
@@ -60,6 +60,7 @@ def lib() -> ctypes.CDLL:
             "tl_shutdown": [],
             "tl_nvfp4_verify_gemm": [vp, i, vp, vp, f, vp, i, i, vp],
             "tl_nvfp4_verify_gemm_simt": [vp, i, vp, vp, f, vp, i, i, vp],
+            "tl_nvfp4_verify_gemm_noalloc": [vp, i, vp, vp, f, vp, i, i, vp],
             "tl_nvfp4_verify_stack": [ctypes.POINTER(Matrix), i, i, vp],
             "tl_nvfp4_verify_stack_host": [ctypes.POINTER(Matrix), i, i, vp, vp, vp, vp, vp],
             "tl_nvfp4_plan_create": [ctypes.POINTER(Matrix), i, i, ctypes.POINTER(vp)],

@@ -317,7 +317,106 @@ tl_status run_stack(const tl_nvfp4_matrix* mats, int n_mats, int M, const unsign
 }
 
 
+// ---------------------------------------------------------------------------
+// An entry point that allocates nothing.
+//
+// Some callers cannot let a library allocate device memory at call time: a serving
+// engine that hands all free HBM to its KV-cache pool at start-up has nothing left
+// for a first-call workspace, and some host runtimes route every device allocation
+// through their own pool and forbid libraries from calling cudaMalloc. For them,
+// tl_nvfp4_verify_gemm_noalloc() runs the same tensor-core kernel with its split-K
+// scratch in the static array below, which the CUDA module reserves when it loads.
+
+// Room for the split-K partials of up to kNoAllocMaxCtas CTAs (two 32 x 128 fp32 tiles
+// each, 5 MiB in all), their counters (must be zero when a launch starts) and a status word.
+constexpr int kNoAllocMaxCtas = 160;
+struct NoAllocScratch {
+    float partials[2 * kNoAllocMaxCtas * 32 * tl::TC_BLOCK_N];
+    unsigned counters[4 * kNoAllocMaxCtas];
+    int err[16];
+};
+
+// Every GPU that loads this library holds this array until the process exits. In host code
+// its name is only a stand-in: the device address comes from cudaGetSymbolAddress below.
+static __device__ __align__(256) NoAllocScratch g_noalloc_scratch;
+
+struct NoAllocDevice {
+    bool ready = false;
+    int num_sms = 0;
+    NoAllocScratch* scratch = nullptr;   // device address of g_noalloc_scratch on this device
+};
+NoAllocDevice g_noalloc[kMaxDevices];
+
+// Once per device, with that device current: resolve the scratch address and the SM count.
+tl_status noalloc_setup(int device, NoAllocDevice** out) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    NoAllocDevice& nd = g_noalloc[device];
+    if (!nd.ready) {
+        int major = 0, minor = 0, sms = 0;
+        TL_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device));
+        TL_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, device));
+        TL_CUDA(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device));
+        if (major != 10 || minor != 0)
+            return fail(TL_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a only", device,
+                        major, minor);
+        void* ptr = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (e != cudaSuccess || ptr == nullptr)
+            return fail(TL_ERR_CUDA, "cudaGetSymbolAddress of the static scratch failed: %s", cudaGetErrorString(e));
+        tl_status st = load_encode_fn();
+        if (st != TL_OK) return st;
+        TL_CUDA(cudaFuncSetAttribute(tl::gemm_tc_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     tl::TcCfg<16>::SMEM_BYTES));
+        TL_CUDA(cudaFuncSetAttribute(tl::gemm_tc_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     tl::TcCfg<32>::SMEM_BYTES));
+        nd.num_sms = sms;
+        nd.scratch = static_cast<NoAllocScratch*>(ptr);
+        nd.ready = true;
+    }
+    *out = &nd;
+    return TL_OK;
+}
+
 }  // namespace
+
+extern "C" tl_status tl_nvfp4_verify_gemm_noalloc(const void* x, int M, const void* w_codes, const void* w_scales,
+                                                  float global_scale, void* y, int N, int K, void* stream) {
+    tl_status st = check_M(M);
+    if (st != TL_OK) return st;
+    st = check_matrix(x, M, w_codes, w_scales, global_scale, y, N, K, true);
+    if (st != TL_OK) return st;
+    if (M == 0) return TL_OK;
+    int dev = 0;
+    TL_CUDA(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) return fail(TL_ERR_INVALID_VALUE, "device %d out of range", dev);
+    NoAllocDevice* nd = nullptr;
+    st = noalloc_setup(dev, &nd);
+    if (st != TL_OK) return st;
+    const int NX = M <= 16 ? 16 : 32;
+    tl::TcParams p;
+    memset(&p, 0, sizeof p);
+    st = build_mat(&p.one, x, M, NX, w_codes, w_scales, global_scale, y, N, K, 0);
+    if (st != TL_OK) return st;
+    p.mats = nullptr;
+    p.n_mats = 1;
+    p.M = M;
+    p.total_tiles = (long long)p.one.n_tiles * p.one.k_tiles;
+    p.partials = nd->scratch->partials;
+    p.counters = nd->scratch->counters;
+    p.err = nd->scratch->err;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // the counters must start at zero; a launch that gave up could have left them raised
+    TL_CUDA(cudaMemsetAsync(p.counters, 0, sizeof(nd->scratch->counters), s));
+    long long grid = p.total_tiles;
+    if (grid > nd->num_sms) grid = nd->num_sms;
+    if (grid > kNoAllocMaxCtas) grid = kNoAllocMaxCtas;
+    if (NX == 16)
+        tl::gemm_tc_kernel<16><<<(unsigned)grid, tl::TC_THREADS, tl::TcCfg<16>::SMEM_BYTES, s>>>(p);
+    else
+        tl::gemm_tc_kernel<32><<<(unsigned)grid, tl::TC_THREADS, tl::TcCfg<32>::SMEM_BYTES, s>>>(p);
+    TL_CUDA(cudaGetLastError());
+    return TL_OK;
+}
 
 struct tl_nvfp4_plan_st {
     int device = 0;
