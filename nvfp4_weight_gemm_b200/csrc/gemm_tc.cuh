@@ -18,7 +18,9 @@
 //     A from tensor memory, B = X tile (bf16, shared memory, 128-byte swizzle) and the
 //     fp32 accumulator in tensor memory (M_mma = 128 weight rows, N_mma = 16 or 32 X rows).
 //     The dequantisers form two groups of four warps that take alternate tiles, so one
-//     group's tensor-memory stores overlap the other group's decode.
+//     group's tensor-memory stores overlap the other group's decode. A single thread keeps
+//     only about one tcgen05.mma in flight per ~90 cycles at these small N, so warps 1..3
+//     each issue a third of every tile's 16 k-steps into their own accumulator.
 //     Warps 12..15 read the accumulator and write Y (or a partial).
 //   * Dequantisation without a table. For code c = s e1 e0 m, the bf16 bit pattern
 //     (e1 e0 m) << 6 | s << 15 is exactly e2m1(c) * 2^-126 (code 1 lands on a bf16
@@ -40,22 +42,15 @@
 
 namespace tl {
 
-// Independent accumulators per output tile: consecutive k-steps of a tile go to
-// different accumulators (k-step i -> accumulator i % TC_NACC) so that successive MMAs
-// do not wait on each other; the epilogue adds them in a fixed order.
-#ifndef TL_TC_NACC
-#define TL_TC_NACC 2
-#endif
-
 constexpr int TC_BLOCK_N = 128;        // weight rows per tile (MMA M)
 constexpr int TC_BLOCK_K = 256;        // k per tile / pipeline stage
-constexpr int TC_NACC = TL_TC_NACC;
-constexpr int TC_NUM_A = TC_NACC >= 4 ? 2 : 3;   // tensor-memory A buffers (128 columns each)
 constexpr int TC_THREADS = 512;
 constexpr int TC_TMEM_COLS = 512;
-constexpr int TC_ACC_COL0 = 128 * TC_NUM_A;   // accumulators after the A buffers
-constexpr int TC_ACC_COLS = 32 * TC_NACC;     // one accumulator buffer: TC_NACC x 32 fp32 columns
-static_assert(TC_ACC_COL0 + 2 * TC_ACC_COLS <= TC_TMEM_COLS, "tensor memory budget");
+// MMA issuers. One thread can only keep about one tcgen05.mma in flight per ~90 cycles,
+// whatever N is, so three issuer warps (1..3) share each tile's 16 k-steps (6 / 5 / 5);
+// issuer j accumulates into its own accumulator j and the epilogue adds them in order.
+constexpr int TC_NISSUE = 3;
+__host__ __device__ constexpr int tc_ks_begin(int j) { return j == 0 ? 0 : (j == 1 ? 6 : (j == 2 ? 11 : 16)); }
 
 enum : int {
     TL_DEV_ERR_TIMEOUT_PRODUCER = 0x101,
@@ -99,6 +94,12 @@ struct TcCfg {
     static constexpr int STAGES = (NX == 32) ? 6 : 8;
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 512 /*barriers*/;
     static constexpr uint32_t IDESC = idesc_f16(1u, 128u, (uint32_t)NX);
+    // tensor memory: A buffers (128 columns each), then two accumulator buffers of
+    // TC_NISSUE accumulators of NX fp32 columns each
+    static constexpr int NUM_A = (NX == 16) ? 3 : 2;
+    static constexpr int ACC_COL0 = 128 * NUM_A;
+    static constexpr int ACC_BUF_COLS = TC_NISSUE * NX;
+    static_assert(ACC_COL0 + 2 * ACC_BUF_COLS <= TC_TMEM_COLS, "tensor memory budget");
 };
 
 struct TcSeg {
@@ -161,7 +162,26 @@ __device__ __forceinline__ uint32_t hmul2_bf16(uint32_t a, uint32_t b) {
 }
 
 // Eight scale bytes -> eight bf16x2 words, both halves e4m3(s) * 2^119 (exact).
+// Fast path for finite, positive, normal scales (every scale the quantiser writes except
+// all-zero blocks): bf16 bits of s * 2^119 are ((s & 0x7F) << 4) + (239 << 7). Anything
+// else (zero or subnormal scale, sign bit, NaN) takes the exact float route.
 __device__ __forceinline__ void scales8_to_bf16x2(uint2 sc, uint32_t (&S)[8]) {
+    const uint32_t e0 = sc.x & 0x78787878u, e1 = sc.y & 0x78787878u;
+    const uint32_t zero_exp = ((e0 - 0x01010101u) & ~e0) | ((e1 - 0x01010101u) & ~e1);   // a byte had e == 0
+    const uint32_t nan_or_neg = ((sc.x | sc.y) & 0x80808080u) |
+                                (((sc.x & 0x7F7F7F7Fu) + 0x01010101u) & 0x80808080u) |
+                                (((sc.y & 0x7F7F7F7Fu) + 0x01010101u) & 0x80808080u);   // bit 7 set or byte 0x7F
+    if (((zero_exp & 0x80808080u) | nan_or_neg) == 0u) {
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            // [b_lo, 0, b_hi, 0] -> bf16 of each scale * 2^119 in its own half
+            const uint32_t w = prmt(p < 2 ? sc.x : sc.y, 0u, (p & 1) ? 0x4342u : 0x4140u);
+            const uint32_t b = (w << 4) + 0x77807780u;
+            S[2 * p] = prmt(b, 0u, 0x1010u);
+            S[2 * p + 1] = prmt(b, 0u, 0x3232u);
+        }
+        return;
+    }
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
         const uint32_t two = ((p < 2 ? sc.x : sc.y) >> (16 * (p & 1))) & 0xFFFFu;
@@ -186,6 +206,55 @@ __device__ __forceinline__ void decode8(uint32_t q, uint32_t S, uint32_t* out) {
     }
 }
 
+// MMA issuer J (warp 1 + J, lane 0): k-steps [tc_ks_begin(J), tc_ks_begin(J + 1)) of every
+// tile into accumulator J.
+template <int NX, int J>
+__device__ __forceinline__ void tc_mma_issuer(const TcParams& p, const TcMat* mats, long long t_begin, long long t_end,
+                                              uint8_t* smem, uint32_t tmem, uint64_t* full, uint64_t* empty,
+                                              uint64_t* aready, uint64_t* afree, uint64_t* accfull,
+                                              uint64_t* accempty, uint64_t* drain, volatile int* abort_flag) {
+    using C = TcCfg<NX>;
+    constexpr int I0 = tc_ks_begin(J), I1 = tc_ks_begin(J + 1);
+    int s = 0, a = 0, acc = 0;
+    uint32_t ph = 0, aph = 0, accph = 0;
+    TcSegIter it(mats, p.n_mats, t_begin, t_end);
+    TcSeg sg;
+    bool ok = true;
+    while (ok && it.next(sg)) {
+        if (*abort_flag || !mbar_wait(&accempty[acc], accph ^ 1u, TL_WAIT_LIMIT)) {
+            tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_MMA);
+            break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(C::ACC_COL0 + C::ACC_BUF_COLS * acc + NX * J);
+        for (int kt = sg.k0; kt < sg.k1; ++kt) {
+            if (*abort_flag || !mbar_wait(&full[s], ph, TL_WAIT_LIMIT) ||
+                !mbar_wait(&aready[a], aph, TL_WAIT_LIMIT)) {
+                tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_MMA);
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t xs = smem_u32(smem + s * C::STAGE_BYTES + C::CODES_BYTES);
+            const uint32_t a_tmem = tmem + (uint32_t)(128 * a);
+#pragma unroll
+            for (int i = I0; i < I1; ++i) {
+                const uint64_t bdesc = smem_desc_k_sw128(xs + (i >> 2) * C::X_SUB + (i & 3) * 32);
+                mma_ts_f16(d_tmem, a_tmem + 8u * i, bdesc, C::IDESC, (kt > sg.k0 || i > I0) ? 1u : 0u);
+            }
+            mma_commit(&empty[s]);
+            mma_commit(&afree[a]);
+            if (++s == C::STAGES) { s = 0; ph ^= 1u; }
+            if (++a == C::NUM_A) { a = 0; aph ^= 1u; }
+        }
+        if (!ok) break;
+        mma_commit(&accfull[acc]);
+        if (++acc == 2) { acc = 0; accph ^= 1u; }
+    }
+    // no MMA of this issuer may still run when tensor memory is released
+    mma_commit(drain);
+}
+
 template <int NX>
 __global__ void __launch_bounds__(TC_THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ TcParams p) {
@@ -194,12 +263,12 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
     uint64_t* full = bars;                          // [STAGES] TMA bytes landed
-    uint64_t* empty = full + C::STAGES;             // [STAGES] stage consumed (MMA commit)
+    uint64_t* empty = full + C::STAGES;             // [STAGES] stage consumed (one commit per issuer)
     uint64_t* aready = empty + C::STAGES;           // [NUM_A] A buffer written (4 warps of a group)
-    uint64_t* afree = aready + TC_NUM_A;            // [NUM_A] A buffer read by MMA (commit)
-    uint64_t* accfull = afree + TC_NUM_A;           // [2] accumulator complete (commit)
-    uint64_t* accempty = accfull + 2;               // [2] accumulator read (4 warps)
-    uint64_t* drain = accempty + 2;                 // [1] final MMA drain
+    uint64_t* afree = aready + C::NUM_A;            // [NUM_A] A buffer read (one commit per issuer)
+    uint64_t* accfull = afree + C::NUM_A;           // [2] accumulators complete (one commit per issuer)
+    uint64_t* accempty = accfull + 2;               // [2] accumulators read (4 epilogue warps)
+    uint64_t* drain = accempty + 2;                 // [1] every MMA finished (one commit per issuer)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -211,10 +280,10 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
     const long long t_end = tc_range_start(blockIdx.x + 1, p.total_tiles, ctas);
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < C::STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-        for (int i = 0; i < TC_NUM_A; ++i) { mbar_init(&aready[i], 4); mbar_init(&afree[i], 1); }
-        for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], 4); }
-        mbar_init(drain, 1);
+        for (int i = 0; i < C::STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], TC_NISSUE); }
+        for (int i = 0; i < C::NUM_A; ++i) { mbar_init(&aready[i], 4); mbar_init(&afree[i], TC_NISSUE); }
+        for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], TC_NISSUE); mbar_init(&accempty[i], 4); }
+        mbar_init(drain, TC_NISSUE);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -266,59 +335,30 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
                     if (!mbar_wait(&full[i], (last_ph >> i) & 1u, TL_WAIT_LIMIT))
                         tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_DRAIN);
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp >= 1 && warp <= TC_NISSUE) {
+        // ------------------------------------------------------------ MMA issuers
         if (lane == 0) {
-            int s = 0, a = 0, acc = 0;
-            uint32_t ph = 0, aph = 0, accph = 0;
-            TcSegIter it(mats, p.n_mats, t_begin, t_end);
-            TcSeg sg;
-            bool ok = true;
-            while (ok && it.next(sg)) {
-                if (*abort_flag || !mbar_wait(&accempty[acc], accph ^ 1u, TL_WAIT_LIMIT)) {
-                    tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_MMA);
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t d_tmem = tmem + (uint32_t)(TC_ACC_COL0 + TC_ACC_COLS * acc);
-                for (int kt = sg.k0; kt < sg.k1; ++kt) {
-                    if (*abort_flag || !mbar_wait(&full[s], ph, TL_WAIT_LIMIT) ||
-                        !mbar_wait(&aready[a], aph, TL_WAIT_LIMIT)) {
-                        tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_MMA);
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t xs = smem_u32(smem + s * C::STAGE_BYTES + C::CODES_BYTES);
-                    const uint32_t a_tmem = tmem + (uint32_t)(128 * a);
-#pragma unroll
-                    for (int i = 0; i < TC_BLOCK_K / 16; ++i) {
-                        const uint64_t bdesc = smem_desc_k_sw128(xs + (i >> 2) * C::X_SUB + (i & 3) * 32);
-                        mma_ts_f16(d_tmem + 32u * (uint32_t)(i % TC_NACC), a_tmem + 8u * i, bdesc, C::IDESC,
-                                   (kt > sg.k0 || i >= TC_NACC) ? 1u : 0u);
-                    }
-                    mma_commit(&empty[s]);
-                    mma_commit(&afree[a]);
-                    if (++s == C::STAGES) { s = 0; ph ^= 1u; }
-                    if (++a == TC_NUM_A) { a = 0; aph ^= 1u; }
-                }
-                if (!ok) break;
-                mma_commit(&accfull[acc]);
-                if (++acc == 2) { acc = 0; accph ^= 1u; }
-            }
-            // no MMA may still run when tensor memory is released
-            mma_commit(drain);
-            if (!mbar_wait(drain, 0, TL_WAIT_LIMIT)) tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_DRAIN);
+            if (warp == 1)
+                tc_mma_issuer<NX, 0>(p, mats, t_begin, t_end, smem, tmem, full, empty, aready, afree, accfull, accempty, drain, abort_flag);
+            else if (warp == 2)
+                tc_mma_issuer<NX, 1>(p, mats, t_begin, t_end, smem, tmem, full, empty, aready, afree, accfull, accempty, drain, abort_flag);
+            else
+                tc_mma_issuer<NX, 2>(p, mats, t_begin, t_end, smem, tmem, full, empty, aready, afree, accfull, accempty, drain, abort_flag);
+            if (warp == 1 && !mbar_wait(drain, 0, TL_WAIT_LIMIT)) tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_DRAIN);
         }
     } else if (warp >= 4 && warp < 12) {
         // ------------------------------------------------------------ dequantisers
         // Two groups of four warps take alternate tiles (group g: tiles c with c % 2 == g),
-        // so one group's tensor-memory store latency overlaps the other group's decode.
-        // Thread r of a group owns weight row r of the tile and decodes all 256 k of it.
+        // so one group's tensor-memory stores overlap the other group's decode.
+        // Thread r of a group owns weight row r of the tile and decodes all 256 k of it;
+        // the first half is decoded before waiting for the A buffer to be free.
         const int grp = (warp - 4) >> 2;
         const int q = warp & 3;                  // tensor-memory lane quarter
         const int r = 32 * q + lane;             // weight row within the tile
         const uint32_t t_lane = tmem + ((uint32_t)(32 * q) << 16);
+        int code_off[8];                         // 16-byte chunk j of row r in the 128-byte swizzle
+#pragma unroll
+        for (int j = 0; j < 8; ++j) code_off[j] = r * 128 + ((j ^ (r & 7)) << 4);
         long long c = 0;                          // tile counter of this CTA
         TcSegIter it(mats, p.n_mats, t_begin, t_end);
         TcSeg sg;
@@ -328,25 +368,21 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
                 if ((int)(c & 1) != grp) continue;
                 const int s = (int)(c % C::STAGES);
                 const uint32_t ph = (uint32_t)((c / C::STAGES) & 1);
-                const int a = (int)(c % TC_NUM_A);
-                const uint32_t aph = (uint32_t)((c / TC_NUM_A) & 1);
-                if (*abort_flag || !mbar_wait(&full[s], ph, TL_WAIT_LIMIT) ||
-                    !mbar_wait(&afree[a], aph ^ 1u, TL_WAIT_LIMIT)) {
+                const int a = (int)(c % C::NUM_A);
+                const uint32_t aph = (uint32_t)((c / C::NUM_A) & 1);
+                if (*abort_flag || !mbar_wait(&full[s], ph, TL_WAIT_LIMIT)) {
                     tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_DEQUANT);
                     ok = false;
                     break;
                 }
-                tc_fence_after();
                 const uint8_t* st = smem + s * C::STAGE_BYTES;
                 const uint4 sc = *reinterpret_cast<const uint4*>(st + C::CODES_BYTES + C::X_BYTES + r * 16);
+                const uint32_t col = (uint32_t)(128 * a);
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {   // two 128-k halves: 64 code bytes, 8 scales each
                     uint4 cw[4];
 #pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        const int j = 4 * h + jj;
-                        cw[jj] = *reinterpret_cast<const uint4*>(st + r * 128 + ((j ^ (r & 7)) << 4));
-                    }
+                    for (int jj = 0; jj < 4; ++jj) cw[jj] = *reinterpret_cast<const uint4*>(st + code_off[4 * h + jj]);
                     uint32_t S[8];
                     scales8_to_bf16x2(h == 0 ? make_uint2(sc.x, sc.y) : make_uint2(sc.z, sc.w), S);
                     uint32_t out[64];
@@ -357,10 +393,18 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
                         decode8(cw[jj].z, S[2 * jj + 1], &out[16 * jj + 8]);
                         decode8(cw[jj].w, S[2 * jj + 1], &out[16 * jj + 12]);
                     }
-                    const uint32_t col = (uint32_t)(128 * a + 64 * h);
-                    tmem_st32(t_lane + col, *reinterpret_cast<const uint32_t(*)[32]>(&out[0]));
-                    tmem_st32(t_lane + col + 32, *reinterpret_cast<const uint32_t(*)[32]>(&out[32]));
+                    if (h == 0) {   // the A buffer must have been read by the MMAs of tile c - NUM_A
+                        if (*abort_flag || !mbar_wait(&afree[a], aph ^ 1u, TL_WAIT_LIMIT)) {
+                            tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_DEQUANT);
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                    }
+                    tmem_st32(t_lane + col + 64 * h, *reinterpret_cast<const uint32_t(*)[32]>(&out[0]));
+                    tmem_st32(t_lane + col + 64 * h + 32, *reinterpret_cast<const uint32_t(*)[32]>(&out[32]));
                 }
+                if (!ok) break;
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
@@ -387,11 +431,11 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
 #pragma unroll
             for (int i = 0; i < NX; ++i) v[i] = 0.0f;
 #pragma unroll
-            for (int j = 0; j < TC_NACC; ++j) {   // fixed order: accumulator 0, 1, ...
+            for (int j = 0; j < TC_NISSUE; ++j) {   // fixed order: accumulator 0, 1, 2
                 uint32_t raw[16];
 #pragma unroll
                 for (int c0 = 0; c0 < NX; c0 += 16) {
-                    tmem_ld16(t_lane + (uint32_t)(TC_ACC_COL0 + TC_ACC_COLS * acc + 32 * j + c0), raw);
+                    tmem_ld16(t_lane + (uint32_t)(C::ACC_COL0 + C::ACC_BUF_COLS * acc + NX * j + c0), raw);
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 16; ++i) v[c0 + i] += __uint_as_float(raw[i]);
