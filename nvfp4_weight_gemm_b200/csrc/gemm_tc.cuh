@@ -11,17 +11,17 @@
 //     whose share starts or ends inside an n-tile writes an fp32 partial; the last of an
 //     n-tile's contributors (an atomic counter, no waiting) adds the partials in k order,
 //     so every output has one fixed reduction order.
-//   * Roles, 16 warps. Warp 0 issues TMA loads of codes, scales and the X tile into a
-//     ring of shared-memory stages. Warps 4..11 dequantise: thread r owns weight row r,
-//     reads its codes/scales from shared memory, forms W' = e2m1 * e4m3 in bf16 (exact)
-//     and stores it into tensor memory, the A operand. Warp 1 issues tcgen05.mma with
+//   * Roles, 24 warps. Warp 0 issues TMA loads of codes, scales and the X tile into a
+//     ring of shared-memory stages. Warps 4..19 dequantise: a thread owns one weight row and
+//     a 128-k half of a tile, reads its codes/scales from shared memory, forms
+//     W' = e2m1 * e4m3 in bf16 (exact) and stores it into tensor memory, the A operand. Warp 1 issues tcgen05.mma with
 //     A from tensor memory, B = X tile (bf16, shared memory, 128-byte swizzle) and the
 //     fp32 accumulator in tensor memory (M_mma = 128 weight rows, N_mma = 16 or 32 X rows).
-//     The dequantisers form two groups of four warps that take alternate tiles, so one
-//     group's tensor-memory stores overlap the other group's decode. A single thread keeps
+//     The dequantisers form two sets of eight warps that take alternate tiles, so four
+//     dequant warps share each scheduler and one set's waits overlap the other's decode. A single thread keeps
 //     only about one tcgen05.mma in flight per ~90 cycles at these small N, so warps 1..3
 //     each issue a third of every tile's 16 k-steps into their own accumulator.
-//     Warps 12..15 read the accumulator and write Y (or a partial).
+//     Warps 20..23 read the accumulators and write Y (or a partial).
 //   * Dequantisation without a table. For code c = s e1 e0 m, the bf16 bit pattern
 //     (e1 e0 m) << 6 | s << 15 is exactly e2m1(c) * 2^-126 (code 1 lands on a bf16
 //     subnormal). One bf16 multiply by e4m3(s) * 2^119 gives W' * 2^-7, exact (at most six
@@ -44,7 +44,7 @@ namespace tl {
 
 constexpr int TC_BLOCK_N = 128;        // weight rows per tile (MMA M)
 constexpr int TC_BLOCK_K = 256;        // k per tile / pipeline stage
-constexpr int TC_THREADS = 512;
+constexpr int TC_THREADS = 768;     // 24 warps: producer, 3 MMA issuers, 16 dequantisers, 4 epilogue
 constexpr int TC_TMEM_COLS = 512;
 // MMA issuers. One thread can only keep about one tcgen05.mma in flight per ~90 cycles,
 // whatever N is, so three issuer warps (1..3) share each tile's 16 k-steps (6 / 5 / 5);
@@ -264,7 +264,7 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
     uint64_t* full = bars;                          // [STAGES] TMA bytes landed
     uint64_t* empty = full + C::STAGES;             // [STAGES] stage consumed (one commit per issuer)
-    uint64_t* aready = empty + C::STAGES;           // [NUM_A] A buffer written (4 warps of a group)
+    uint64_t* aready = empty + C::STAGES;           // [NUM_A] A buffer written (8 warps of a tile set)
     uint64_t* afree = aready + C::NUM_A;            // [NUM_A] A buffer read (one commit per issuer)
     uint64_t* accfull = afree + C::NUM_A;           // [2] accumulators complete (one commit per issuer)
     uint64_t* accempty = accfull + 2;               // [2] accumulators read (4 epilogue warps)
@@ -281,7 +281,7 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], TC_NISSUE); }
-        for (int i = 0; i < C::NUM_A; ++i) { mbar_init(&aready[i], 4); mbar_init(&afree[i], TC_NISSUE); }
+        for (int i = 0; i < C::NUM_A; ++i) { mbar_init(&aready[i], 8); mbar_init(&afree[i], TC_NISSUE); }
         for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], TC_NISSUE); mbar_init(&accempty[i], 4); }
         mbar_init(drain, TC_NISSUE);
         *abort_flag = 0;
@@ -346,72 +346,77 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
                 tc_mma_issuer<NX, 2>(p, mats, t_begin, t_end, smem, tmem, full, empty, aready, afree, accfull, accempty, drain, abort_flag);
             if (warp == 1 && !mbar_wait(drain, 0, TL_WAIT_LIMIT)) tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_DRAIN);
         }
-    } else if (warp >= 4 && warp < 12) {
+    } else if (warp >= 4 && warp < 20) {
         // ------------------------------------------------------------ dequantisers
-        // Two groups of four warps take alternate tiles (group g: tiles c with c % 2 == g),
-        // so one group's tensor-memory stores overlap the other group's decode.
-        // Thread r of a group owns weight row r of the tile and decodes all 256 k of it;
-        // the first half is decoded before waiting for the A buffer to be free.
-        const int grp = (warp - 4) >> 2;
+        // 16 warps = 2 tile sets x 2 k-halves x 4 lane quarters. Set t takes the tiles with
+        // parity t, so two tiles are decoded at once; within a tile, the warp of k-half h and
+        // lane quarter q decodes rows 32q..32q+31, k in [128h, 128h + 128), in two chunks of
+        // 64 k, and stores them into tensor-memory columns [64h, 64h + 64) of the A buffer.
+        const int dq = warp - 4;
+        const int set = dq >> 3;
+        const int kh = (dq >> 2) & 1;
         const int q = warp & 3;                  // tensor-memory lane quarter
         const int r = 32 * q + lane;             // weight row within the tile
         const uint32_t t_lane = tmem + ((uint32_t)(32 * q) << 16);
-        int code_off[8];                         // 16-byte chunk j of row r in the 128-byte swizzle
-#pragma unroll
-        for (int j = 0; j < 8; ++j) code_off[j] = r * 128 + ((j ^ (r & 7)) << 4);
-        long long c = 0;                          // tile counter of this CTA
+        const int row_off = r * 128, row_sw = r & 7;   // chunk j of row r sits at row_off + ((j ^ row_sw) << 4)
+        int s = 0, a = 0, par = 0;
+        uint32_t ph = 0, aph = 0;
         TcSegIter it(mats, p.n_mats, t_begin, t_end);
         TcSeg sg;
         bool ok = true;
         while (ok && it.next(sg)) {
-            for (int kt = sg.k0; kt < sg.k1; ++kt, ++c) {
-                if ((int)(c & 1) != grp) continue;
-                const int s = (int)(c % C::STAGES);
-                const uint32_t ph = (uint32_t)((c / C::STAGES) & 1);
-                const int a = (int)(c % C::NUM_A);
-                const uint32_t aph = (uint32_t)((c / C::NUM_A) & 1);
-                if (*abort_flag || !mbar_wait(&full[s], ph, TL_WAIT_LIMIT)) {
+            for (int kt = sg.k0; kt < sg.k1; ++kt) {
+                const int ts = s, ta = a;
+                const uint32_t tph = ph, taph = aph;
+                const bool mine = (par == set);
+                if (++s == C::STAGES) { s = 0; ph ^= 1u; }
+                if (++a == C::NUM_A) { a = 0; aph ^= 1u; }
+                par ^= 1;
+                if (!mine) continue;
+                if (*abort_flag || !mbar_wait(&full[ts], tph, TL_WAIT_LIMIT)) {
                     tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_DEQUANT);
                     ok = false;
                     break;
                 }
-                const uint8_t* st = smem + s * C::STAGE_BYTES;
-                const uint4 sc = *reinterpret_cast<const uint4*>(st + C::CODES_BYTES + C::X_BYTES + r * 16);
-                const uint32_t col = (uint32_t)(128 * a);
+                const uint8_t* st = smem + ts * C::STAGE_BYTES;
+                const uint2 sc = *reinterpret_cast<const uint2*>(st + C::CODES_BYTES + C::X_BYTES + r * 16 + 8 * kh);
+                uint32_t S[8];
+                scales8_to_bf16x2(sc, S);
+                const uint32_t col = (uint32_t)(128 * ta + 64 * kh);
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {   // two 128-k halves: 64 code bytes, 8 scales each
-                    uint4 cw[4];
+                for (int hc = 0; hc < 2; ++hc) {   // two chunks of 64 k: 32 code bytes, 4 scales
+                    uint4 cw[2];
 #pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) cw[jj] = *reinterpret_cast<const uint4*>(st + code_off[4 * h + jj]);
-                    uint32_t S[8];
-                    scales8_to_bf16x2(h == 0 ? make_uint2(sc.x, sc.y) : make_uint2(sc.z, sc.w), S);
-                    uint32_t out[64];
+                    for (int jj = 0; jj < 2; ++jj)
+                        cw[jj] = *reinterpret_cast<const uint4*>(st + row_off + (((4 * kh + 2 * hc + jj) ^ row_sw) << 4));
+                    uint32_t out[32];
 #pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        decode8(cw[jj].x, S[2 * jj], &out[16 * jj + 0]);
-                        decode8(cw[jj].y, S[2 * jj], &out[16 * jj + 4]);
-                        decode8(cw[jj].z, S[2 * jj + 1], &out[16 * jj + 8]);
-                        decode8(cw[jj].w, S[2 * jj + 1], &out[16 * jj + 12]);
+                    for (int jj = 0; jj < 2; ++jj) {
+                        const uint4 w = cw[jj];
+                        const int b = 4 * hc + 2 * jj;
+                        decode8(w.x, S[b], &out[16 * jj + 0]);
+                        decode8(w.y, S[b], &out[16 * jj + 4]);
+                        decode8(w.z, S[b + 1], &out[16 * jj + 8]);
+                        decode8(w.w, S[b + 1], &out[16 * jj + 12]);
                     }
-                    if (h == 0) {   // the A buffer must have been read by the MMAs of tile c - NUM_A
-                        if (*abort_flag || !mbar_wait(&afree[a], aph ^ 1u, TL_WAIT_LIMIT)) {
+                    if (hc == 0) {   // the A buffer must have been read by the MMAs of tile c - NUM_A
+                        if (*abort_flag || !mbar_wait(&afree[ta], taph ^ 1u, TL_WAIT_LIMIT)) {
                             tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_DEQUANT);
                             ok = false;
                             break;
                         }
                         tc_fence_after();
                     }
-                    tmem_st32(t_lane + col + 64 * h, *reinterpret_cast<const uint32_t(*)[32]>(&out[0]));
-                    tmem_st32(t_lane + col + 64 * h + 32, *reinterpret_cast<const uint32_t(*)[32]>(&out[32]));
+                    tmem_st32(t_lane + col + 32 * hc, out);
                 }
                 if (!ok) break;
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&aready[a]);
+                if (lane == 0) mbar_arrive(&aready[ta]);
             }
         }
-    } else if (warp >= 12) {
+    } else if (warp >= 20) {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;
         const int r = 32 * q + lane;
@@ -427,47 +432,51 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
                 break;
             }
             tc_fence_after();
-            float v[NX];
+            const TcMat& m = mats[sg.mat];
+            const int N = m.N;
+            const int n = sg.ntile * TC_BLOCK_N + r;
+            const bool whole = (sg.k0 == 0 && sg.k1 == m.k_tiles);
+            const long long ta = m.tile_begin + (long long)sg.ntile * m.k_tiles;
+            const int my_slot = 2 * (int)blockIdx.x + (sg.t0 == t_begin ? 0 : 1);
+            float* mine = p.partials + (size_t)my_slot * (32 * TC_BLOCK_N);
+            // 16 columns (X rows) at a time: add the issuers' accumulators in fixed order,
+            // then write Y (whole n-tile) or this CTA's partial (split n-tile)
 #pragma unroll
-            for (int i = 0; i < NX; ++i) v[i] = 0.0f;
+            for (int c0 = 0; c0 < NX; c0 += 16) {
+                float v[16];
 #pragma unroll
-            for (int j = 0; j < TC_NISSUE; ++j) {   // fixed order: accumulator 0, 1, 2
-                uint32_t raw[16];
+                for (int i = 0; i < 16; ++i) v[i] = 0.0f;
 #pragma unroll
-                for (int c0 = 0; c0 < NX; c0 += 16) {
+                for (int j = 0; j < TC_NISSUE; ++j) {
+                    uint32_t raw[16];
                     tmem_ld16(t_lane + (uint32_t)(C::ACC_COL0 + C::ACC_BUF_COLS * acc + NX * j + c0), raw);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) v[c0 + i] += __uint_as_float(raw[i]);
+                    for (int i = 0; i < 16; ++i) v[i] += __uint_as_float(raw[i]);
+                }
+                if (whole) {
+                    if (n < N) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            if (c0 + i < M) m.y[(long long)(c0 + i) * N + n] = __float2bfloat16_rn(v[i] * m.g_out);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        if (c0 + i < M) mine[(c0 + i) * TC_BLOCK_N + r] = v[i];
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&accempty[acc]);
             if (++acc == 2) { acc = 0; accph ^= 1u; }
+            if (whole) continue;
 
-            const TcMat& m = mats[sg.mat];
-            const int N = m.N;
-            const int n = sg.ntile * TC_BLOCK_N + r;
-            if (sg.k0 == 0 && sg.k1 == m.k_tiles) {
-                if (n < N) {
-#pragma unroll
-                    for (int i = 0; i < NX; ++i)
-                        if (i < M) m.y[(long long)i * N + n] = __float2bfloat16_rn(v[i] * m.g_out);
-                }
-                continue;
-            }
-            // split n-tile: publish this warp's 32 rows of the partial; the last of the
-            // n-tile's contributors for these rows adds all partials in k (CTA) order
-            const long long ta = m.tile_begin + (long long)sg.ntile * m.k_tiles;
+            // split n-tile: the last of the n-tile's contributors for these 32 rows adds all
+            // partials in k (CTA) order
             const long long tb = ta + m.k_tiles;
             const int f = tc_cta_of(ta, p.total_tiles, ctas);
             const int l = tc_cta_of(tb - 1, p.total_tiles, ctas);
-            const int my_slot = 2 * (int)blockIdx.x + (sg.t0 == t_begin ? 0 : 1);
-            float* mine = p.partials + (size_t)my_slot * (32 * TC_BLOCK_N);
-#pragma unroll
-            for (int i = 0; i < NX; ++i)
-                if (i < M) mine[i * TC_BLOCK_N + r] = v[i];
             __threadfence();
             __syncwarp();
             unsigned old = 0;
@@ -475,21 +484,24 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
             old = __shfl_sync(0xFFFFFFFFu, old, 0);
             if (old == (unsigned)(l - f)) {
                 __threadfence();
-                float sum[NX];
 #pragma unroll
-                for (int i = 0; i < NX; ++i) sum[i] = 0.0f;
-                for (int c = f; c <= l; ++c) {
-                    const long long cs = tc_range_start(c, p.total_tiles, ctas);
-                    const int slot = 2 * c + ((ta > cs ? ta : cs) == cs ? 0 : 1);
-                    const float* part = p.partials + (size_t)slot * (32 * TC_BLOCK_N);
+                for (int c0 = 0; c0 < NX; c0 += 16) {
+                    float v[16];
 #pragma unroll
-                    for (int i = 0; i < NX; ++i)
-                        if (i < M) sum[i] += (c == (int)blockIdx.x) ? v[i] : __ldcg(&part[i * TC_BLOCK_N + r]);
-                }
-                if (n < N) {
+                    for (int i = 0; i < 16; ++i) v[i] = 0.0f;
+                    for (int c = f; c <= l; ++c) {
+                        const long long cs = tc_range_start(c, p.total_tiles, ctas);
+                        const int slot = 2 * c + ((ta > cs ? ta : cs) == cs ? 0 : 1);
+                        const float* part = p.partials + (size_t)slot * (32 * TC_BLOCK_N);
 #pragma unroll
-                    for (int i = 0; i < NX; ++i)
-                        if (i < M) m.y[(long long)i * N + n] = __float2bfloat16_rn(sum[i] * m.g_out);
+                        for (int i = 0; i < 16; ++i)
+                            if (c0 + i < M) v[i] += __ldcg(&part[(c0 + i) * TC_BLOCK_N + r]);
+                    }
+                    if (n < N) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            if (c0 + i < M) m.y[(long long)(c0 + i) * N + n] = __float2bfloat16_rn(v[i] * m.g_out);
+                    }
                 }
                 if (lane == 0) p.counters[4 * f + q] = 0u;   // ready for the next launch
             }
