@@ -12,7 +12,7 @@
 //     n-tile's contributors (an atomic counter, no waiting) adds the partials in k order,
 //     so every output has one fixed reduction order.
 //   * Roles, 24 warps. Warp 0 issues TMA loads of codes, scales and the X tile into a
-//     ring of shared-memory stages. Warps 4..19 dequantise: a thread owns one weight row and
+//     ring of shared-memory stages (three lanes, one rank-3 load each, per stage). Warps 4..19 dequantise: a thread owns one weight row and
 //     a 128-k half of a tile, reads its codes/scales from shared memory, forms
 //     W' = e2m1 * e4m3 in bf16 (exact) and stores it into tensor memory, the A operand. Warp 1 issues tcgen05.mma with
 //     A from tensor memory, B = X tile (bf16, shared memory, 128-byte swizzle) and the
@@ -62,9 +62,10 @@ enum : int {
 
 // One matrix of a launch: tensor maps of its codes, scales and X, and its work-list offset.
 struct alignas(64) TcMat {
-    CUtensorMap tm_codes;   // uint8 [N][K/2], box 128 B x 128 rows, 128-byte swizzle
-    CUtensorMap tm_scales;  // uint8 [N][K/16], box 16 B x 128 rows
-    CUtensorMap tm_x;       // bf16 [M][K], box 64 x NX rows, 128-byte swizzle (rows >= M read 0)
+    CUtensorMap tm_codes;   // uint8 {K/2, N, 1}, box 128 B x 128 rows x 1, 128-byte swizzle
+    CUtensorMap tm_scales;  // uint8 {K/16, N, 1}, box 16 B x 128 rows x 1
+    CUtensorMap tm_x;       // bf16 X as 3-D {64, M, K/64}, box {64, NX, 4}: the four 64-k slices of a
+                            // tile, 128-byte swizzle (rows >= M read 0)
     __nv_bfloat16* y;
     float g_out;            // epilogue multiplier: global_scale * 2^7
     int N;
@@ -94,12 +95,15 @@ struct TcCfg {
     static constexpr int STAGES = (NX == 32) ? 6 : 8;
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 512 /*barriers*/;
     static constexpr uint32_t IDESC = idesc_f16(1u, 128u, (uint32_t)NX);
-    // tensor memory: A buffers (128 columns each), then two accumulator buffers of
-    // TC_NISSUE accumulators of NX fp32 columns each
-    static constexpr int NUM_A = (NX == 16) ? 3 : 2;
+    // tensor memory: three A buffers (128 columns each) so a tile set never waits for the
+    // MMAs of its own previous tile, then ACC_BUFS accumulator buffers of TC_NISSUE
+    // accumulators of NX fp32 columns each (one buffer at NX = 32: the MMAs then wait for
+    // the epilogue once per n-tile segment, which is cheaper than a third-short A ring)
+    static constexpr int NUM_A = 3;
+    static constexpr int ACC_BUFS = (NX == 16) ? 2 : 1;
     static constexpr int ACC_COL0 = 128 * NUM_A;
     static constexpr int ACC_BUF_COLS = TC_NISSUE * NX;
-    static_assert(ACC_COL0 + 2 * ACC_BUF_COLS <= TC_TMEM_COLS, "tensor memory budget");
+    static_assert(ACC_COL0 + ACC_BUFS * ACC_BUF_COLS <= TC_TMEM_COLS, "tensor memory budget");
 };
 
 struct TcSeg {
@@ -249,7 +253,7 @@ __device__ __forceinline__ void tc_mma_issuer(const TcParams& p, const TcMat* ma
         }
         if (!ok) break;
         mma_commit(&accfull[acc]);
-        if (++acc == 2) { acc = 0; accph ^= 1u; }
+        if (++acc == C::ACC_BUFS) { acc = 0; accph ^= 1u; }
     }
     // no MMA of this issuer may still run when tensor memory is released
     mma_commit(drain);
@@ -266,8 +270,8 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
     uint64_t* empty = full + C::STAGES;             // [STAGES] stage consumed (one commit per issuer)
     uint64_t* aready = empty + C::STAGES;           // [NUM_A] A buffer written (8 warps of a tile set)
     uint64_t* afree = aready + C::NUM_A;            // [NUM_A] A buffer read (one commit per issuer)
-    uint64_t* accfull = afree + C::NUM_A;           // [2] accumulators complete (one commit per issuer)
-    uint64_t* accempty = accfull + 2;               // [2] accumulators read (4 epilogue warps)
+    uint64_t* accfull = afree + C::NUM_A;           // [ACC_BUFS] accumulators complete (one commit per issuer)
+    uint64_t* accempty = accfull + 2;               // [ACC_BUFS] accumulators read (4 epilogue warps)
     uint64_t* drain = accempty + 2;                 // [1] every MMA finished (one commit per issuer)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -282,7 +286,7 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], TC_NISSUE); }
         for (int i = 0; i < C::NUM_A; ++i) { mbar_init(&aready[i], 8); mbar_init(&afree[i], TC_NISSUE); }
-        for (int i = 0; i < 2; ++i) { mbar_init(&accfull[i], TC_NISSUE); mbar_init(&accempty[i], 4); }
+        for (int i = 0; i < C::ACC_BUFS; ++i) { mbar_init(&accfull[i], TC_NISSUE); mbar_init(&accempty[i], 4); }
         mbar_init(drain, TC_NISSUE);
         *abort_flag = 0;
         fence_barrier_init();
@@ -298,38 +302,45 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            const uint64_t pol_w = policy_evict_first();
-            const uint64_t pol_x = policy_evict_last();
-            int s = 0;
-            uint32_t ph = 0;
-            uint32_t issued = 0;   // bit s: stage s was issued at least once
-            uint32_t last_ph = 0;  // bit s: parity of its latest use
-            TcSegIter it(mats, p.n_mats, t_begin, t_end);
-            TcSeg sg;
-            bool ok = true;
-            while (ok && it.next(sg)) {
-                const TcMat& m = mats[sg.mat];
-                for (int kt = sg.k0; kt < sg.k1; ++kt) {
-                    if (*abort_flag || !mbar_wait(&empty[s], ph ^ 1u, TL_WAIT_LIMIT)) {
-                        tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_PRODUCER);
-                        ok = false;
-                        break;
-                    }
-                    uint8_t* st = smem + s * C::STAGE_BYTES;
-                    mbar_arrive_expect_tx(&full[s], (uint32_t)C::STAGE_BYTES);
-                    tma_load_2d(st, &m.tm_codes, &full[s], kt * (TC_BLOCK_K / 2), sg.ntile * TC_BLOCK_N, pol_w);
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        tma_load_2d(st + C::CODES_BYTES + j * C::X_SUB, &m.tm_x, &full[s], kt * TC_BLOCK_K + 64 * j, 0, pol_x);
-                    tma_load_2d(st + C::CODES_BYTES + C::X_BYTES, &m.tm_scales, &full[s], kt * (TC_BLOCK_K / 16),
-                                sg.ntile * TC_BLOCK_N, pol_w);
-                    issued |= 1u << s;
-                    last_ph = (last_ph & ~(1u << s)) | (ph << s);
-                    if (++s == C::STAGES) { s = 0; ph ^= 1u; }
+        // The whole warp runs the loop and every lane waits for the stage itself; lane 0 posts
+        // the stage's byte count, then lanes 0, 1, 2 copy codes, X and scales with one
+        // converged 3-D load (all three maps are rank 3).
+        const uint64_t pol = (lane == 1) ? policy_evict_last() : policy_evict_first();
+        const uint32_t dst_off = (lane == 0) ? 0u : (lane == 1) ? (uint32_t)C::CODES_BYTES
+                                                                : (uint32_t)(C::CODES_BYTES + C::X_BYTES);
+        const uint32_t smem0 = smem_u32(smem);
+        int s = 0;
+        uint32_t ph = 0;
+        uint32_t issued = 0;   // bit s: stage s was issued at least once
+        uint32_t last_ph = 0;  // bit s: parity of its latest use
+        TcSegIter it(mats, p.n_mats, t_begin, t_end);
+        TcSeg sg;
+        bool ok = true;
+        while (ok && it.next(sg)) {
+            const TcMat& m = mats[sg.mat];
+            const void* tmap = (lane == 0) ? (const void*)&m.tm_codes
+                             : (lane == 1) ? (const void*)&m.tm_x : (const void*)&m.tm_scales;
+            const int c1 = (lane == 1) ? 0 : sg.ntile * TC_BLOCK_N;
+            for (int kt = sg.k0; kt < sg.k1; ++kt) {
+                const bool got = !*abort_flag && mbar_wait(&empty[s], ph ^ 1u, TL_WAIT_LIMIT);
+                if (!__all_sync(0xFFFFFFFFu, got)) {
+                    if (lane == 0) tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_PRODUCER);
+                    ok = false;
+                    break;
                 }
+                if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)C::STAGE_BYTES);
+                __syncwarp();
+                const int c0 = (lane == 0) ? kt * (TC_BLOCK_K / 2) : (lane == 1) ? 0 : kt * (TC_BLOCK_K / 16);
+                const int c2 = (lane == 1) ? kt * 4 : 0;
+                if (lane < 3)
+                    tma_load_3d_s(smem0 + (uint32_t)(s * C::STAGE_BYTES) + dst_off, tmap, &full[s], c0, c1, c2, pol);
+                issued |= 1u << s;
+                last_ph = (last_ph & ~(1u << s)) | (ph << s);
+                if (++s == C::STAGES) { s = 0; ph ^= 1u; }
             }
-            // every issued copy must land before the CTA can leave
+        }
+        // every issued copy must land before the CTA can leave
+        if (lane == 0) {
             for (int i = 0; i < C::STAGES; ++i)
                 if ((issued >> i) & 1u)
                     if (!mbar_wait(&full[i], (last_ph >> i) & 1u, TL_WAIT_LIMIT))
@@ -469,7 +480,7 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&accempty[acc]);
-            if (++acc == 2) { acc = 0; accph ^= 1u; }
+            if (++acc == C::ACC_BUFS) { acc = 0; accph ^= 1u; }
             if (whole) continue;
 
             // split n-tile: the last of the n-tile's contributors for these 32 rows adds all

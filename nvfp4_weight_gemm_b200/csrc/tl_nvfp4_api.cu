@@ -159,29 +159,36 @@ tl_status check_matrix(const void* x, int M, const void* codes, const void* scal
     return TL_OK;
 }
 
-tl_status encode_2d(CUtensorMap* tm, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
-                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
-    cuuint64_t dims[2] = {inner, outer};
-    cuuint64_t strides[1] = {row_bytes};
-    cuuint32_t box[2] = {box_inner, box_outer};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = g_encode(tm, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return fail(TL_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+// Rank-3 tiled tensor map (dims innermost first; strides in bytes for dims 1 and 2).
+tl_status encode_3d(CUtensorMap* tm, CUtensorMapDataType dt, const void* base, const cuuint64_t (&dims)[3],
+                    const cuuint64_t (&strides)[2], const cuuint32_t (&box)[3], CUtensorMapSwizzle sw,
+                    const char* what) {
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(tm, dt, 3, const_cast<void*>(base), const_cast<cuuint64_t*>(dims),
+                          const_cast<cuuint64_t*>(strides), const_cast<cuuint32_t*>(box), estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(TL_ERR_CUDA, "cuTensorMapEncodeTiled (%s) failed (%d)", what, (int)r);
     return TL_OK;
 }
 
 tl_status build_mat(tl::TcMat* m, const void* x, int M, int NX, const void* codes, const void* scales, float g,
                     void* y, int N, int K, long long tile_begin) {
     memset(m, 0, sizeof *m);
-    tl_status st = encode_2d(&m->tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, (uint64_t)K / 2, (uint64_t)N,
-                             (uint64_t)K / 2, tl::TC_BLOCK_K / 2, tl::TC_BLOCK_N, CU_TENSOR_MAP_SWIZZLE_128B);
+    // All three maps are rank 3 so that one converged load instruction can issue them.
+    // Codes and scales: {bytes per row, N rows, 1}; a tile box is 128 rows of one k-tile.
+    const cuuint64_t n = (cuuint64_t)N, k = (cuuint64_t)K;
+    tl_status st = encode_3d(&m->tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, {k / 2, n, 1}, {k / 2, n * (k / 2)},
+                             {tl::TC_BLOCK_K / 2, tl::TC_BLOCK_N, 1}, CU_TENSOR_MAP_SWIZZLE_128B, "codes");
     if (st != TL_OK) return st;
-    st = encode_2d(&m->tm_scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, scales, (uint64_t)K / 16, (uint64_t)N,
-                   (uint64_t)K / 16, tl::TC_BLOCK_K / 16, tl::TC_BLOCK_N, CU_TENSOR_MAP_SWIZZLE_NONE);
+    st = encode_3d(&m->tm_scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, scales, {k / 16, n, 1}, {k / 16, n * (k / 16)},
+                   {tl::TC_BLOCK_K / 16, tl::TC_BLOCK_N, 1}, CU_TENSOR_MAP_SWIZZLE_NONE, "scales");
     if (st != TL_OK) return st;
-    st = encode_2d(&m->tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64,
-                   (uint32_t)NX, CU_TENSOR_MAP_SWIZZLE_128B);
+    // X viewed as {64 elements, M rows, K/64 slices}: one box {64, NX, 4} lands the four 64-k
+    // slices of a tile one after another in shared memory, each NX rows x 128 B, swizzled;
+    // rows >= M read zero.
+    st = encode_3d(&m->tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, {64, (cuuint64_t)M, k / 64}, {k * 2, 128},
+                   {64, (cuuint32_t)NX, 4}, CU_TENSOR_MAP_SWIZZLE_128B, "X");
     if (st != TL_OK) return st;
     m->y = static_cast<__nv_bfloat16*>(y);
     m->g_out = (float)((double)g * 128.0);   // W' reaches the accumulator scaled by 2^-7
