@@ -11,12 +11,15 @@
 //     whose share starts or ends inside an n-tile writes an fp32 partial; the last of an
 //     n-tile's contributors (an atomic counter, no waiting) adds the partials in k order,
 //     so every output has one fixed reduction order.
-//   * Roles, 24 warps. Warp 0 issues TMA loads of codes, scales and the X tile into a
-//     ring of shared-memory stages (three lanes, one rank-3 load each, per stage). Warps 4..19 dequantise: a thread owns one weight row and
-//     a 128-k half of a tile, reads its codes/scales from shared memory, forms
-//     W' = e2m1 * e4m3 in bf16 (exact) and stores it into tensor memory, the A operand. Warp 1 issues tcgen05.mma with
-//     A from tensor memory, B = X tile (bf16, shared memory, 128-byte swizzle) and the
-//     fp32 accumulator in tensor memory (M_mma = 128 weight rows, N_mma = 16 or 32 X rows).
+//   * Roles, 25 warps. Warp 0 streams codes and scales (TMA) into a ring of weight stages;
+//     a stage is handed back as soon as the dequantisers hold its bytes in registers, so
+//     nearly the whole ring is in flight from HBM. Warp 24 loads the X tile of each k-tile
+//     into a separate, shorter ring (an L2 hit) that the MMAs release. Warps 4..19
+//     dequantise: a thread owns one weight row and a 128-k half of a tile, reads its
+//     codes/scales from shared memory, forms W' = e2m1 * e4m3 in bf16 (exact) and stores it
+//     into tensor memory, the A operand. Warps 1..3 issue tcgen05.mma with A from tensor
+//     memory, B = X tile (bf16, shared memory, 128-byte swizzle) and the fp32 accumulator in
+//     tensor memory (M_mma = 128 weight rows, N_mma = 16 or 32 X rows).
 //     The dequantisers form two sets of eight warps that take alternate tiles, so four
 //     dequant warps share each scheduler and one set's waits overlap the other's decode. A single thread keeps
 //     only about one tcgen05.mma in flight per ~90 cycles at these small N, so warps 1..3
@@ -44,13 +47,15 @@ namespace tl {
 
 constexpr int TC_BLOCK_N = 128;        // weight rows per tile (MMA M)
 constexpr int TC_BLOCK_K = 256;        // k per tile / pipeline stage
-constexpr int TC_THREADS = 768;     // 24 warps: producer, 3 MMA issuers, 16 dequantisers, 4 epilogue
+constexpr int TC_THREADS = 832;     // 26 warps: weight producer, 4 MMA issuers, 16 dequantisers, 4 epilogue, X producer
+constexpr int TC_XWARP = 24;
 constexpr int TC_TMEM_COLS = 512;
 // MMA issuers. One thread can only keep about one tcgen05.mma in flight per ~90 cycles,
-// whatever N is, so three issuer warps (1..3) share each tile's 16 k-steps (6 / 5 / 5);
-// issuer j accumulates into its own accumulator j and the epilogue adds them in order.
-constexpr int TC_NISSUE = 3;
-__host__ __device__ constexpr int tc_ks_begin(int j) { return j == 0 ? 0 : (j == 1 ? 6 : (j == 2 ? 11 : 16)); }
+// whatever N is, so four issuer warps (1, 2, 3 and 25) share each tile's 16 k-steps, four
+// each; issuer j accumulates into its own accumulator j and the epilogue adds them in order.
+constexpr int TC_NISSUE = 4;
+__host__ __device__ constexpr int tc_ks_begin(int j) { return 4 * j; }
+__host__ __device__ constexpr int tc_issuer_of_warp(int w) { return (w >= 1 && w <= 3) ? w - 1 : (w == 25 ? 3 : -1); }
 
 enum : int {
     TL_DEV_ERR_TIMEOUT_PRODUCER = 0x101,
@@ -91,15 +96,19 @@ struct TcCfg {
     static constexpr int X_SUB = NX * 128;                              // one 64-k slice of X
     static constexpr int X_BYTES = 4 * X_SUB;
     static constexpr int SCALES_BYTES = TC_BLOCK_N * (TC_BLOCK_K / 16); // 2048
-    static constexpr int STAGE_BYTES = CODES_BYTES + X_BYTES + SCALES_BYTES;
-    static constexpr int STAGES = (NX == 32) ? 6 : 8;
-    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 512 /*barriers*/;
+    // Two rings. Weight stages (codes + scales, read once from HBM) are released as soon as
+    // the dequantisers have loaded them, so almost the whole weight ring is in flight; X
+    // stages (an L2 hit) are released by the MMAs.
+    static constexpr int W_STAGE_BYTES = CODES_BYTES + SCALES_BYTES;   // 18432
+    static constexpr int W_STAGES = (NX == 32) ? 9 : 11;
+    static constexpr int X_RING = W_STAGES * W_STAGE_BYTES;            // offset of the X ring
+    static constexpr int NUM_A = 3;                                    // tile slots: A buffer + X stage
+    static constexpr int SMEM_BYTES = X_RING + NUM_A * X_BYTES + 1024 /*align*/ + 512 /*barriers*/;
     static constexpr uint32_t IDESC = idesc_f16(1u, 128u, (uint32_t)NX);
     // tensor memory: three A buffers (128 columns each) so a tile set never waits for the
     // MMAs of its own previous tile, then ACC_BUFS accumulator buffers of TC_NISSUE
     // accumulators of NX fp32 columns each (one buffer at NX = 32: the MMAs then wait for
     // the epilogue once per n-tile segment, which is cheaper than a third-short A ring)
-    static constexpr int NUM_A = 3;
     static constexpr int ACC_BUFS = (NX == 16) ? 2 : 1;
     static constexpr int ACC_COL0 = 128 * NUM_A;
     static constexpr int ACC_BUF_COLS = TC_NISSUE * NX;
@@ -153,6 +162,15 @@ __device__ __forceinline__ void tc_fail(int* err, volatile int* abort_flag, int 
     *abort_flag = 1;
 }
 
+// Bounded wait that also gives up when another role has aborted the CTA.
+__device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    for (uint32_t i = 0; i < TL_WAIT_LIMIT; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+    }
+    return false;
+}
+
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     uint32_t d;
     asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
@@ -197,6 +215,32 @@ __device__ __forceinline__ void scales8_to_bf16x2(uint2 sc, uint32_t (&S)[8]) {
     }
 }
 
+// Four scale bytes -> four bf16x2 words, both halves e4m3(s) * 2^119 (exact); the same
+// fast path and exact fallback as the eight-byte form.
+__device__ __forceinline__ void scales4_to_bf16x2(uint32_t sc, uint32_t (&S)[4]) {
+    const uint32_t e = sc & 0x78787878u;
+    const uint32_t zero_exp = (e - 0x01010101u) & ~e;   // a byte had e == 0
+    const uint32_t nan_or_neg = (sc & 0x80808080u) | (((sc & 0x7F7F7F7Fu) + 0x01010101u) & 0x80808080u);
+    if (((zero_exp & 0x80808080u) | nan_or_neg) == 0u) {
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            const uint32_t w = prmt(sc, 0u, p ? 0x4342u : 0x4140u);
+            const uint32_t b = (w << 4) + 0x77807780u;
+            S[2 * p] = prmt(b, 0u, 0x1010u);
+            S[2 * p + 1] = prmt(b, 0u, 0x3232u);
+        }
+        return;
+    }
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+        const __half2 h = e4m3x2_to_half2((sc >> (16 * p)) & 0xFFFFu);
+        const float f0 = __low2float(h) * 0x1p119f;
+        const float f1 = __high2float(h) * 0x1p119f;
+        S[2 * p] = prmt(__float_as_uint(f0), 0u, 0x3232u);
+        S[2 * p + 1] = prmt(__float_as_uint(f1), 0u, 0x3232u);
+    }
+}
+
 // Four code bytes (eight weights, k order) -> four bf16x2 words W' * 2^-7 in k order.
 __device__ __forceinline__ void decode8(uint32_t q, uint32_t S, uint32_t* out) {
     const uint32_t L = q & 0x0F0F0F0Fu;          // even-k nibbles, one per byte
@@ -210,53 +254,63 @@ __device__ __forceinline__ void decode8(uint32_t q, uint32_t S, uint32_t* out) {
     }
 }
 
-// MMA issuer J (warp 1 + J, lane 0): k-steps [tc_ks_begin(J), tc_ks_begin(J + 1)) of every
-// tile into accumulator J.
+// MMA issuer J (a whole warp, converged; one elected lane issues): k-steps
+// [tc_ks_begin(J), tc_ks_begin(J + 1)) of every tile into accumulator J. A tile slot (A buffer +
+// X stage) is ready when the 8 warps of its tile set have arrived and its X bytes have landed;
+// the slot is handed back by one commit per issuer.
 template <int NX, int J>
 __device__ __forceinline__ void tc_mma_issuer(const TcParams& p, const TcMat* mats, long long t_begin, long long t_end,
-                                              uint8_t* smem, uint32_t tmem, uint64_t* full, uint64_t* empty,
-                                              uint64_t* aready, uint64_t* afree, uint64_t* accfull,
-                                              uint64_t* accempty, uint64_t* drain, volatile int* abort_flag) {
+                                              uint8_t* smem, uint32_t tmem, uint64_t* ready, uint64_t* tfree,
+                                              uint64_t* accfull, uint64_t* accempty, uint64_t* drain,
+                                              volatile int* abort_flag) {
     using C = TcCfg<NX>;
     constexpr int I0 = tc_ks_begin(J), I1 = tc_ks_begin(J + 1);
-    int s = 0, a = 0, acc = 0;
-    uint32_t ph = 0, aph = 0, accph = 0;
+    const bool leader = elect_one();   // issues every MMA and commit of this issuer
+    int a = 0, acc = 0;
+    uint32_t aph = 0, accph = 0;
+    // descriptor of slot 0's X stage; the start-address field (bits 0..13, address >> 4)
+    // advances by plain addition, which never carries out of the field for shared addresses
+    const uint64_t bdesc_base = smem_desc_k_sw128(smem_u32(smem + C::X_RING));
     TcSegIter it(mats, p.n_mats, t_begin, t_end);
     TcSeg sg;
     bool ok = true;
     while (ok && it.next(sg)) {
-        if (*abort_flag || !mbar_wait(&accempty[acc], accph ^ 1u, TL_WAIT_LIMIT)) {
-            tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_MMA);
+        if (!__all_sync(0xFFFFFFFFu, tc_wait(&accempty[acc], accph ^ 1u, abort_flag))) {
+            if (leader) tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_MMA);
             break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)(C::ACC_COL0 + C::ACC_BUF_COLS * acc + NX * J);
+        uint32_t first = 1;   // the first MMA of a segment overwrites the accumulator
         for (int kt = sg.k0; kt < sg.k1; ++kt) {
-            if (*abort_flag || !mbar_wait(&full[s], ph, TL_WAIT_LIMIT) ||
-                !mbar_wait(&aready[a], aph, TL_WAIT_LIMIT)) {
-                tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_MMA);
+            if (!__all_sync(0xFFFFFFFFu, tc_wait(&ready[a], aph, abort_flag))) {
+                if (leader) tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_MMA);
                 ok = false;
                 break;
             }
             tc_fence_after();
-            const uint32_t xs = smem_u32(smem + s * C::STAGE_BYTES + C::CODES_BYTES);
-            const uint32_t a_tmem = tmem + (uint32_t)(128 * a);
+            const uint64_t bdesc0 = bdesc_base + (uint64_t)((a * C::X_BYTES) >> 4);
+            const uint32_t a_tmem = tmem + (uint32_t)(128 * a + 8 * I0);
+            if (leader) {
 #pragma unroll
-            for (int i = I0; i < I1; ++i) {
-                const uint64_t bdesc = smem_desc_k_sw128(xs + (i >> 2) * C::X_SUB + (i & 3) * 32);
-                mma_ts_f16(d_tmem, a_tmem + 8u * i, bdesc, C::IDESC, (kt > sg.k0 || i > I0) ? 1u : 0u);
+                for (int i = I0; i < I1; ++i)
+                    mma_ts_f16(d_tmem, a_tmem + 8u * (i - I0),
+                               bdesc0 + (uint64_t)((((i >> 2) * C::X_SUB + (i & 3) * 32)) >> 4), C::IDESC,
+                               (i == I0) ? (first ^ 1u) : 1u);
+                mma_commit(&tfree[a]);
             }
-            mma_commit(&empty[s]);
-            mma_commit(&afree[a]);
-            if (++s == C::STAGES) { s = 0; ph ^= 1u; }
+            __syncwarp();
+            first = 0;
             if (++a == C::NUM_A) { a = 0; aph ^= 1u; }
         }
         if (!ok) break;
-        mma_commit(&accfull[acc]);
+        if (leader) mma_commit(&accfull[acc]);
+        __syncwarp();
         if (++acc == C::ACC_BUFS) { acc = 0; accph ^= 1u; }
     }
     // no MMA of this issuer may still run when tensor memory is released
-    mma_commit(drain);
+    if (leader) mma_commit(drain);
+    __syncwarp();
 }
 
 template <int NX>
@@ -265,12 +319,12 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
     using C = TcCfg<NX>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
-    uint64_t* full = bars;                          // [STAGES] TMA bytes landed
-    uint64_t* empty = full + C::STAGES;             // [STAGES] stage consumed (one commit per issuer)
-    uint64_t* aready = empty + C::STAGES;           // [NUM_A] A buffer written (8 warps of a tile set)
-    uint64_t* afree = aready + C::NUM_A;            // [NUM_A] A buffer read (one commit per issuer)
-    uint64_t* accfull = afree + C::NUM_A;           // [ACC_BUFS] accumulators complete (one commit per issuer)
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::X_RING + C::NUM_A * C::X_BYTES);
+    uint64_t* wfull = bars;                         // [W_STAGES] codes + scales landed
+    uint64_t* wempty = wfull + C::W_STAGES;         // [W_STAGES] loaded by the 8 warps of a tile set
+    uint64_t* ready = wempty + C::W_STAGES;         // [NUM_A] tile slot filled: 8 warps of a tile set + X bytes
+    uint64_t* tfree = ready + C::NUM_A;             // [NUM_A] tile slot read by the MMAs (one commit per issuer)
+    uint64_t* accfull = tfree + C::NUM_A;           // [ACC_BUFS] accumulators complete (one commit per issuer)
     uint64_t* accempty = accfull + 2;               // [ACC_BUFS] accumulators read (4 epilogue warps)
     uint64_t* drain = accempty + 2;                 // [1] every MMA finished (one commit per issuer)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -284,8 +338,8 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
     const long long t_end = tc_range_start(blockIdx.x + 1, p.total_tiles, ctas);
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < C::STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], TC_NISSUE); }
-        for (int i = 0; i < C::NUM_A; ++i) { mbar_init(&aready[i], 8); mbar_init(&afree[i], TC_NISSUE); }
+        for (int i = 0; i < C::W_STAGES; ++i) { mbar_init(&wfull[i], 1); mbar_init(&wempty[i], 8); }
+        for (int i = 0; i < C::NUM_A; ++i) { mbar_init(&ready[i], 9); mbar_init(&tfree[i], TC_NISSUE); }
         for (int i = 0; i < C::ACC_BUFS; ++i) { mbar_init(&accfull[i], TC_NISSUE); mbar_init(&accempty[i], 4); }
         mbar_init(drain, TC_NISSUE);
         *abort_flag = 0;
@@ -301,13 +355,12 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer
+        // ------------------------------------------------------------ weight producer
         // The whole warp runs the loop and every lane waits for the stage itself; lane 0 posts
-        // the stage's byte count, then lanes 0, 1, 2 copy codes, X and scales with one
-        // converged 3-D load (all three maps are rank 3).
-        const uint64_t pol = (lane == 1) ? policy_evict_last() : policy_evict_first();
-        const uint32_t dst_off = (lane == 0) ? 0u : (lane == 1) ? (uint32_t)C::CODES_BYTES
-                                                                : (uint32_t)(C::CODES_BYTES + C::X_BYTES);
+        // the stage's byte count, then lanes 0 and 1 copy codes and scales with one converged
+        // 3-D load.
+        const uint64_t pol = policy_evict_first();
+        const uint32_t dst_off = (lane == 0) ? 0u : (uint32_t)C::CODES_BYTES;
         const uint32_t smem0 = smem_u32(smem);
         int s = 0;
         uint32_t ph = 0;
@@ -318,51 +371,95 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
         bool ok = true;
         while (ok && it.next(sg)) {
             const TcMat& m = mats[sg.mat];
-            const void* tmap = (lane == 0) ? (const void*)&m.tm_codes
-                             : (lane == 1) ? (const void*)&m.tm_x : (const void*)&m.tm_scales;
-            const int c1 = (lane == 1) ? 0 : sg.ntile * TC_BLOCK_N;
+            const void* tmap = (lane == 0) ? (const void*)&m.tm_codes : (const void*)&m.tm_scales;
+            const int c1 = sg.ntile * TC_BLOCK_N;
             for (int kt = sg.k0; kt < sg.k1; ++kt) {
-                const bool got = !*abort_flag && mbar_wait(&empty[s], ph ^ 1u, TL_WAIT_LIMIT);
+                const bool got = !*abort_flag && mbar_wait(&wempty[s], ph ^ 1u, TL_WAIT_LIMIT);
                 if (!__all_sync(0xFFFFFFFFu, got)) {
                     if (lane == 0) tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_PRODUCER);
                     ok = false;
                     break;
                 }
-                if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)C::STAGE_BYTES);
+                if (lane == 0) mbar_arrive_expect_tx(&wfull[s], (uint32_t)C::W_STAGE_BYTES);
                 __syncwarp();
-                const int c0 = (lane == 0) ? kt * (TC_BLOCK_K / 2) : (lane == 1) ? 0 : kt * (TC_BLOCK_K / 16);
-                const int c2 = (lane == 1) ? kt * 4 : 0;
-                if (lane < 3)
-                    tma_load_3d_s(smem0 + (uint32_t)(s * C::STAGE_BYTES) + dst_off, tmap, &full[s], c0, c1, c2, pol);
+                const int c0 = (lane == 0) ? kt * (TC_BLOCK_K / 2) : kt * (TC_BLOCK_K / 16);
+                if (lane < 2)
+                    tma_load_3d_s(smem0 + (uint32_t)(s * C::W_STAGE_BYTES) + dst_off, tmap, &wfull[s], c0, c1, 0, pol);
                 issued |= 1u << s;
                 last_ph = (last_ph & ~(1u << s)) | (ph << s);
-                if (++s == C::STAGES) { s = 0; ph ^= 1u; }
+                if (++s == C::W_STAGES) { s = 0; ph ^= 1u; }
             }
         }
         // every issued copy must land before the CTA can leave
         if (lane == 0) {
-            for (int i = 0; i < C::STAGES; ++i)
+            for (int i = 0; i < C::W_STAGES; ++i)
                 if ((issued >> i) & 1u)
-                    if (!mbar_wait(&full[i], (last_ph >> i) & 1u, TL_WAIT_LIMIT))
+                    if (!mbar_wait(&wfull[i], (last_ph >> i) & 1u, TL_WAIT_LIMIT))
                         tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_DRAIN);
         }
-    } else if (warp >= 1 && warp <= TC_NISSUE) {
-        // ------------------------------------------------------------ MMA issuers
-        if (lane == 0) {
-            if (warp == 1)
-                tc_mma_issuer<NX, 0>(p, mats, t_begin, t_end, smem, tmem, full, empty, aready, afree, accfull, accempty, drain, abort_flag);
-            else if (warp == 2)
-                tc_mma_issuer<NX, 1>(p, mats, t_begin, t_end, smem, tmem, full, empty, aready, afree, accfull, accempty, drain, abort_flag);
-            else
-                tc_mma_issuer<NX, 2>(p, mats, t_begin, t_end, smem, tmem, full, empty, aready, afree, accfull, accempty, drain, abort_flag);
-            if (warp == 1 && !mbar_wait(drain, 0, TL_WAIT_LIMIT)) tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_DRAIN);
+    } else if (warp == TC_XWARP) {
+        // ------------------------------------------------------------ X producer
+        // The X tile of tile n goes into the X stage of tile slot n % NUM_A; its arrival is
+        // the ninth arrival (plus the bytes) on the slot's ready barrier. The warp runs the
+        // loop converged; one elected lane issues.
+        const bool leader = elect_one();
+        const uint64_t pol = policy_evict_last();
+        int a = 0;
+        uint32_t aph = 0;
+        uint32_t issued = 0, last_ph = 0;
+        TcSegIter it(mats, p.n_mats, t_begin, t_end);
+        TcSeg sg;
+        bool ok = true;
+        while (ok && it.next(sg)) {
+            const TcMat& m = mats[sg.mat];
+            for (int kt = sg.k0; kt < sg.k1; ++kt) {
+                if (!__all_sync(0xFFFFFFFFu, tc_wait(&tfree[a], aph ^ 1u, abort_flag))) {
+                    if (leader) tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_PRODUCER);
+                    ok = false;
+                    break;
+                }
+                if (leader) {
+                    mbar_arrive_expect_tx(&ready[a], (uint32_t)C::X_BYTES);
+                    tma_load_3d_s(smem_u32(smem + C::X_RING + a * C::X_BYTES), &m.tm_x, &ready[a], 0, 0, kt * 4, pol);
+                }
+                __syncwarp();
+                issued |= 1u << a;
+                last_ph = (last_ph & ~(1u << a)) | (aph << a);
+                if (++a == C::NUM_A) { a = 0; aph ^= 1u; }
+            }
         }
+        // the slot of every issued copy completes before the CTA leaves (at once on the
+        // normal path, where the MMAs consumed it; bounded on an error path)
+        if (leader) {
+            for (int i = 0; i < C::NUM_A; ++i)
+                if ((issued >> i) & 1u)
+                    if (!mbar_wait(&ready[i], (last_ph >> i) & 1u, TL_WAIT_LIMIT))
+                        tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_DRAIN);
+        }
+    } else if (tc_issuer_of_warp(warp) >= 0) {
+        // ------------------------------------------------------------ MMA issuers
+        const int j = tc_issuer_of_warp(warp);
+        if (j == 0)
+            tc_mma_issuer<NX, 0>(p, mats, t_begin, t_end, smem, tmem, ready, tfree, accfull, accempty, drain, abort_flag);
+        else if (j == 1)
+            tc_mma_issuer<NX, 1>(p, mats, t_begin, t_end, smem, tmem, ready, tfree, accfull, accempty, drain, abort_flag);
+        else if (j == 2)
+            tc_mma_issuer<NX, 2>(p, mats, t_begin, t_end, smem, tmem, ready, tfree, accfull, accempty, drain, abort_flag);
+        else
+            tc_mma_issuer<NX, 3>(p, mats, t_begin, t_end, smem, tmem, ready, tfree, accfull, accempty, drain, abort_flag);
+        if (warp == 1 && !__all_sync(0xFFFFFFFFu, mbar_wait(drain, 0, TL_WAIT_LIMIT)) && lane == 0)
+            tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_DRAIN);
     } else if (warp >= 4 && warp < 20) {
         // ------------------------------------------------------------ dequantisers
         // 16 warps = 2 tile sets x 2 k-halves x 4 lane quarters. Set t takes the tiles with
-        // parity t, so two tiles are decoded at once; within a tile, the warp of k-half h and
-        // lane quarter q decodes rows 32q..32q+31, k in [128h, 128h + 128), in two chunks of
-        // 64 k, and stores them into tensor-memory columns [64h, 64h + 64) of the A buffer.
+        // parity t, so one set's barrier and load latencies overlap the other set's decode.
+        // Within a tile the warp of k-half h and lane quarter q decodes rows 32q..32q+31,
+        // k in [128h, 128h + 128) (64 code bytes and 8 scales per thread) in two chunks of
+        // 64 k, stored into
+        // tensor-memory columns [64h, 64h + 64) of the tile's slot. Barrier tests for the next
+        // tile and for this tile's slot are issued before the decode; a tile's stores are
+        // completed (and its slot marked ready) after the next tile's first chunk is decoded.
+        // Wait outcomes are warp-uniform.
         const int dq = warp - 4;
         const int set = dq >> 3;
         const int kh = (dq >> 2) & 1;
@@ -370,64 +467,106 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
         const int r = 32 * q + lane;             // weight row within the tile
         const uint32_t t_lane = tmem + ((uint32_t)(32 * q) << 16);
         const int row_off = r * 128, row_sw = r & 7;   // chunk j of row r sits at row_off + ((j ^ row_sw) << 4)
-        int s = 0, a = 0, par = 0;
+        const uint32_t sc_off = (uint32_t)(C::CODES_BYTES + r * 16 + 8 * kh);
+        uint32_t cw_off[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) cw_off[j] = (uint32_t)(row_off + (((4 * kh + j) ^ row_sw) << 4));
+        const long long ntiles = t_end - t_begin;
+        // this set's tiles are n = set, set + 2, ...: stage n % W_STAGES, slot n % NUM_A
+        int s = set, a = set;
         uint32_t ph = 0, aph = 0;
-        TcSegIter it(mats, p.n_mats, t_begin, t_end);
-        TcSeg sg;
+        auto advance2 = [](int& idx, uint32_t& phase, int ring) {
+            idx += 2;
+            if (idx >= ring) { idx -= ring; phase ^= 1u; }
+        };
+        // registers hold the scales and first-chunk codes of the current tile; the second
+        // chunk's codes are read after the first chunk is stored, then the stage goes back
+        uint2 sc = make_uint2(0, 0);
+        uint4 cw0 = make_uint4(0, 0, 0, 0), cw1 = cw0;
+        const uint8_t* st_cur = smem;
         bool ok = true;
-        while (ok && it.next(sg)) {
-            for (int kt = sg.k0; kt < sg.k1; ++kt) {
-                const int ts = s, ta = a;
-                const uint32_t tph = ph, taph = aph;
-                const bool mine = (par == set);
-                if (++s == C::STAGES) { s = 0; ph ^= 1u; }
-                if (++a == C::NUM_A) { a = 0; aph ^= 1u; }
-                par ^= 1;
-                if (!mine) continue;
-                if (*abort_flag || !mbar_wait(&full[ts], tph, TL_WAIT_LIMIT)) {
-                    tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_DEQUANT);
-                    ok = false;
-                    break;
-                }
-                const uint8_t* st = smem + ts * C::STAGE_BYTES;
-                const uint2 sc = *reinterpret_cast<const uint2*>(st + C::CODES_BYTES + C::X_BYTES + r * 16 + 8 * kh);
-                uint32_t S[8];
-                scales8_to_bf16x2(sc, S);
-                const uint32_t col = (uint32_t)(128 * ta + 64 * kh);
-#pragma unroll
-                for (int hc = 0; hc < 2; ++hc) {   // two chunks of 64 k: 32 code bytes, 4 scales
-                    uint4 cw[2];
-#pragma unroll
-                    for (int jj = 0; jj < 2; ++jj)
-                        cw[jj] = *reinterpret_cast<const uint4*>(st + row_off + (((4 * kh + 2 * hc + jj) ^ row_sw) << 4));
-                    uint32_t out[32];
-#pragma unroll
-                    for (int jj = 0; jj < 2; ++jj) {
-                        const uint4 w = cw[jj];
-                        const int b = 4 * hc + 2 * jj;
-                        decode8(w.x, S[b], &out[16 * jj + 0]);
-                        decode8(w.y, S[b], &out[16 * jj + 4]);
-                        decode8(w.z, S[b + 1], &out[16 * jj + 8]);
-                        decode8(w.w, S[b + 1], &out[16 * jj + 12]);
-                    }
-                    if (hc == 0) {   // the A buffer must have been read by the MMAs of tile c - NUM_A
-                        if (*abort_flag || !mbar_wait(&afree[ta], taph ^ 1u, TL_WAIT_LIMIT)) {
-                            tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_DEQUANT);
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                    }
-                    tmem_st32(t_lane + col + 32 * hc, out);
-                }
-                if (!ok) break;
+        if (set < ntiles) {
+            ok = __all_sync(0xFFFFFFFFu, tc_wait(&wfull[s], ph, abort_flag));
+            if (ok) {
+                st_cur = smem + s * C::W_STAGE_BYTES;
+                sc = *reinterpret_cast<const uint2*>(st_cur + sc_off);
+                cw0 = *reinterpret_cast<const uint4*>(st_cur + cw_off[0]);
+                cw1 = *reinterpret_cast<const uint4*>(st_cur + cw_off[1]);
+            } else if (lane == 0) {
+                tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_DEQUANT);
+            }
+        }
+        int s_cur = s;
+        advance2(s, ph, C::W_STAGES);
+        int a_prev = -1;
+        for (long long n = set; ok && n < ntiles; n += 2) {
+            const bool has_next = n + 2 < ntiles;
+            const bool next_ready = __all_sync(0xFFFFFFFFu, has_next ? mbar_test(&wfull[s], ph) : true);
+            // the slot must have been read by the MMAs of tile n - NUM_A
+            const bool a_ready = __all_sync(0xFFFFFFFFu, mbar_test(&tfree[a], aph ^ 1u));
+            uint32_t S[4];
+            scales4_to_bf16x2(sc.x, S);
+            uint32_t out[32];
+            decode8(cw0.x, S[0], &out[0]);
+            decode8(cw0.y, S[0], &out[4]);
+            decode8(cw0.z, S[1], &out[8]);
+            decode8(cw0.w, S[1], &out[12]);
+            decode8(cw1.x, S[2], &out[16]);
+            decode8(cw1.y, S[2], &out[20]);
+            decode8(cw1.z, S[3], &out[24]);
+            decode8(cw1.w, S[3], &out[28]);
+            if (a_prev >= 0) {   // the previous tile's stores: complete them, hand its slot to the MMAs
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&aready[ta]);
+                if (lane == 0) mbar_arrive(&ready[a_prev]);
+                a_prev = -1;
+            }
+            if (!a_ready && !__all_sync(0xFFFFFFFFu, tc_wait(&tfree[a], aph ^ 1u, abort_flag))) {
+                if (lane == 0) tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_DEQUANT);
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t col = t_lane + (uint32_t)(128 * a + 64 * kh);
+            tmem_st32(col, out);
+            cw0 = *reinterpret_cast<const uint4*>(st_cur + cw_off[2]);
+            cw1 = *reinterpret_cast<const uint4*>(st_cur + cw_off[3]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&wempty[s_cur]);   // every byte of the stage this warp needs is in registers
+            scales4_to_bf16x2(sc.y, S);
+            decode8(cw0.x, S[0], &out[0]);
+            decode8(cw0.y, S[0], &out[4]);
+            decode8(cw0.z, S[1], &out[8]);
+            decode8(cw0.w, S[1], &out[12]);
+            decode8(cw1.x, S[2], &out[16]);
+            decode8(cw1.y, S[2], &out[20]);
+            decode8(cw1.z, S[3], &out[24]);
+            decode8(cw1.w, S[3], &out[28]);
+            tmem_st32(col + 32u, out);
+            a_prev = a;
+            advance2(a, aph, C::NUM_A);
+            if (has_next) {
+                if (!next_ready && !__all_sync(0xFFFFFFFFu, tc_wait(&wfull[s], ph, abort_flag))) {
+                    if (lane == 0) tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_DEQUANT);
+                    ok = false;
+                    break;
+                }
+                st_cur = smem + s * C::W_STAGE_BYTES;
+                s_cur = s;
+                sc = *reinterpret_cast<const uint2*>(st_cur + sc_off);
+                cw0 = *reinterpret_cast<const uint4*>(st_cur + cw_off[0]);
+                cw1 = *reinterpret_cast<const uint4*>(st_cur + cw_off[1]);
+                advance2(s, ph, C::W_STAGES);
             }
         }
-    } else if (warp >= 20) {
+        tmem_wait_st();   // no store of this warp may be in flight when tensor memory is released
+        if (ok && a_prev >= 0) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ready[a_prev]);
+        }
+    } else if (warp >= 20 && warp < 24) {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;
         const int r = 32 * q + lane;
