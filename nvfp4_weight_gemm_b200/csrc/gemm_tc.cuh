@@ -87,6 +87,7 @@ struct TcParams {
     float* partials;        // [2 * gridDim.x][32][128] fp32
     unsigned* counters;     // [4 * gridDim.x], zero between launches
     int* err;               // device status word
+    uint32_t spread_mul;    // 0x1040, passed at run time so the decode multiply stays one IMAD
     TcMat one;
 };
 
@@ -242,14 +243,17 @@ __device__ __forceinline__ void scales4_to_bf16x2(uint32_t sc, uint32_t (&S)[4])
 }
 
 // Four code bytes (eight weights, k order) -> four bf16x2 words W' * 2^-7 in k order.
-__device__ __forceinline__ void decode8(uint32_t q, uint32_t S, uint32_t* out) {
+// `spread` is 0x1040 (x * 2^6 + x * 2^12); it arrives as a kernel argument so that the
+// compiler keeps the multiply as one IMAD (FMA pipe) instead of shifts on the integer pipe,
+// which the prmt/lop3 steps already keep busy.
+__device__ __forceinline__ void decode8(uint32_t q, uint32_t S, uint32_t spread, uint32_t* out) {
     const uint32_t L = q & 0x0F0F0F0Fu;          // even-k nibbles, one per byte
     const uint32_t H = (q >> 4) & 0x0F0F0F0Fu;   // odd-k nibbles
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         // [L.byte i, 0, H.byte i, 0]; selector 8 replicates the (zero) sign of L.byte 0
         const uint32_t t = prmt(L, H, (uint32_t)i | 0x80u | ((uint32_t)(4 + i) << 8) | 0x8000u);
-        const uint32_t w = (t * 0x1040u) & 0x81C081C0u;   // e1e0m -> bits 6..8, sign -> bit 15
+        const uint32_t w = (t * spread) & 0x81C081C0u;   // e1e0m -> bits 6..8, sign -> bit 15
         out[i] = hmul2_bf16(w, S);
     }
 }
@@ -374,7 +378,7 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
             const void* tmap = (lane == 0) ? (const void*)&m.tm_codes : (const void*)&m.tm_scales;
             const int c1 = sg.ntile * TC_BLOCK_N;
             for (int kt = sg.k0; kt < sg.k1; ++kt) {
-                const bool got = !*abort_flag && mbar_wait(&wempty[s], ph ^ 1u, TL_WAIT_LIMIT);
+                const bool got = tc_wait(&wempty[s], ph ^ 1u, abort_flag);
                 if (!__all_sync(0xFFFFFFFFu, got)) {
                     if (lane == 0) tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_PRODUCER);
                     ok = false;
@@ -457,8 +461,7 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
         // k in [128h, 128h + 128) (64 code bytes and 8 scales per thread) in two chunks of
         // 64 k, stored into
         // tensor-memory columns [64h, 64h + 64) of the tile's slot. Barrier tests for the next
-        // tile and for this tile's slot are issued before the decode; a tile's stores are
-        // completed (and its slot marked ready) after the next tile's first chunk is decoded.
+        // tile and for this tile's slot are issued before the decode.
         // Wait outcomes are warp-uniform.
         const int dq = warp - 4;
         const int set = dq >> 3;
@@ -472,6 +475,7 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) cw_off[j] = (uint32_t)(row_off + (((4 * kh + j) ^ row_sw) << 4));
         const long long ntiles = t_end - t_begin;
+        const uint32_t spread = p.spread_mul;
         // this set's tiles are n = set, set + 2, ...: stage n % W_STAGES, slot n % NUM_A
         int s = set, a = set;
         uint32_t ph = 0, aph = 0;
@@ -498,7 +502,6 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
         }
         int s_cur = s;
         advance2(s, ph, C::W_STAGES);
-        int a_prev = -1;
         for (long long n = set; ok && n < ntiles; n += 2) {
             const bool has_next = n + 2 < ntiles;
             const bool next_ready = __all_sync(0xFFFFFFFFu, has_next ? mbar_test(&wfull[s], ph) : true);
@@ -507,21 +510,17 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
             uint32_t S[4];
             scales4_to_bf16x2(sc.x, S);
             uint32_t out[32];
-            decode8(cw0.x, S[0], &out[0]);
-            decode8(cw0.y, S[0], &out[4]);
-            decode8(cw0.z, S[1], &out[8]);
-            decode8(cw0.w, S[1], &out[12]);
-            decode8(cw1.x, S[2], &out[16]);
-            decode8(cw1.y, S[2], &out[20]);
-            decode8(cw1.z, S[3], &out[24]);
-            decode8(cw1.w, S[3], &out[28]);
-            if (a_prev >= 0) {   // the previous tile's stores: complete them, hand its slot to the MMAs
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&ready[a_prev]);
-                a_prev = -1;
-            }
+            decode8(cw0.x, S[0], spread, &out[0]);
+            decode8(cw0.y, S[0], spread, &out[4]);
+            decode8(cw0.z, S[1], spread, &out[8]);
+            decode8(cw0.w, S[1], spread, &out[12]);
+            decode8(cw1.x, S[2], spread, &out[16]);
+            decode8(cw1.y, S[2], spread, &out[20]);
+            decode8(cw1.z, S[3], spread, &out[24]);
+            decode8(cw1.w, S[3], spread, &out[28]);
+            // second chunk's codes: in flight while the first chunk is stored
+            cw0 = *reinterpret_cast<const uint4*>(st_cur + cw_off[2]);
+            cw1 = *reinterpret_cast<const uint4*>(st_cur + cw_off[3]);
             if (!a_ready && !__all_sync(0xFFFFFFFFu, tc_wait(&tfree[a], aph ^ 1u, abort_flag))) {
                 if (lane == 0) tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_DEQUANT);
                 ok = false;
@@ -530,22 +529,19 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
             tc_fence_after();
             const uint32_t col = t_lane + (uint32_t)(128 * a + 64 * kh);
             tmem_st32(col, out);
-            cw0 = *reinterpret_cast<const uint4*>(st_cur + cw_off[2]);
-            cw1 = *reinterpret_cast<const uint4*>(st_cur + cw_off[3]);
             __syncwarp();
             if (lane == 0) mbar_arrive(&wempty[s_cur]);   // every byte of the stage this warp needs is in registers
             scales4_to_bf16x2(sc.y, S);
-            decode8(cw0.x, S[0], &out[0]);
-            decode8(cw0.y, S[0], &out[4]);
-            decode8(cw0.z, S[1], &out[8]);
-            decode8(cw0.w, S[1], &out[12]);
-            decode8(cw1.x, S[2], &out[16]);
-            decode8(cw1.y, S[2], &out[20]);
-            decode8(cw1.z, S[3], &out[24]);
-            decode8(cw1.w, S[3], &out[28]);
+            decode8(cw0.x, S[0], spread, &out[0]);
+            decode8(cw0.y, S[0], spread, &out[4]);
+            decode8(cw0.z, S[1], spread, &out[8]);
+            decode8(cw0.w, S[1], spread, &out[12]);
+            decode8(cw1.x, S[2], spread, &out[16]);
+            decode8(cw1.y, S[2], spread, &out[20]);
+            decode8(cw1.z, S[3], spread, &out[24]);
+            decode8(cw1.w, S[3], spread, &out[28]);
             tmem_st32(col + 32u, out);
-            a_prev = a;
-            advance2(a, aph, C::NUM_A);
+            // the next tile's scales and first-chunk codes: in flight while the stores complete
             if (has_next) {
                 if (!next_ready && !__all_sync(0xFFFFFFFFu, tc_wait(&wfull[s], ph, abort_flag))) {
                     if (lane == 0) tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_DEQUANT);
@@ -559,13 +555,13 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
                 cw1 = *reinterpret_cast<const uint4*>(st_cur + cw_off[1]);
                 advance2(s, ph, C::W_STAGES);
             }
-        }
-        tmem_wait_st();   // no store of this warp may be in flight when tensor memory is released
-        if (ok && a_prev >= 0) {
+            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&ready[a_prev]);
+            if (lane == 0) mbar_arrive(&ready[a]);   // the slot goes to the MMAs
+            advance2(a, aph, C::NUM_A);
         }
+        tmem_wait_st();   // no store of this warp may be in flight when tensor memory is released
     } else if (warp >= 20 && warp < 24) {
         // ------------------------------------------------------------ epilogue
         const int q = warp & 3;
@@ -577,7 +573,7 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
         TcSegIter it(mats, p.n_mats, t_begin, t_end);
         TcSeg sg;
         while (it.next(sg)) {
-            if (*abort_flag || !mbar_wait(&accfull[acc], accph, TL_WAIT_LIMIT)) {
+            if (!tc_wait(&accfull[acc], accph, abort_flag)) {
                 tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_EPILOGUE);
                 break;
             }
@@ -589,37 +585,37 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
             const long long ta = m.tile_begin + (long long)sg.ntile * m.k_tiles;
             const int my_slot = 2 * (int)blockIdx.x + (sg.t0 == t_begin ? 0 : 1);
             float* mine = p.partials + (size_t)my_slot * (32 * TC_BLOCK_N);
-            // 16 columns (X rows) at a time: add the issuers' accumulators in fixed order,
-            // then write Y (whole n-tile) or this CTA's partial (split n-tile)
+            // add the issuers' accumulators in fixed order into registers, hand the
+            // accumulators back to the MMAs, then write Y (whole n-tile) or this CTA's partial
+            float v[NX];
 #pragma unroll
-            for (int c0 = 0; c0 < NX; c0 += 16) {
-                float v[16];
+            for (int i = 0; i < NX; ++i) v[i] = 0.0f;
 #pragma unroll
-                for (int i = 0; i < 16; ++i) v[i] = 0.0f;
+            for (int j = 0; j < TC_NISSUE; ++j) {
 #pragma unroll
-                for (int j = 0; j < TC_NISSUE; ++j) {
+                for (int c0 = 0; c0 < NX; c0 += 16) {
                     uint32_t raw[16];
                     tmem_ld16(t_lane + (uint32_t)(C::ACC_COL0 + C::ACC_BUF_COLS * acc + NX * j + c0), raw);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) v[i] += __uint_as_float(raw[i]);
-                }
-                if (whole) {
-                    if (n < N) {
-#pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            if (c0 + i < M) m.y[(long long)(c0 + i) * N + n] = __float2bfloat16_rn(v[i] * m.g_out);
-                    }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        if (c0 + i < M) mine[(c0 + i) * TC_BLOCK_N + r] = v[i];
+                    for (int i = 0; i < 16; ++i) v[c0 + i] += __uint_as_float(raw[i]);
                 }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&accempty[acc]);
             if (++acc == C::ACC_BUFS) { acc = 0; accph ^= 1u; }
+            if (whole) {
+                if (n < N) {
+#pragma unroll
+                    for (int i = 0; i < NX; ++i)
+                        if (i < M) m.y[(long long)i * N + n] = __float2bfloat16_rn(v[i] * m.g_out);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < NX; ++i)
+                    if (i < M) mine[i * TC_BLOCK_N + r] = v[i];
+            }
             if (whole) continue;
 
             // split n-tile: the last of the n-tile's contributors for these 32 rows adds all

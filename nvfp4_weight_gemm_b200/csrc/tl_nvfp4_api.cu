@@ -208,6 +208,7 @@ tl_status launch_tc(DevState& d, tl::TcParams& p, cudaStream_t stream) {
     p.partials = d.partials;
     p.counters = d.counters;
     p.err = d.err;
+    p.spread_mul = 0x1040u;
     tl::gemm_tc_kernel<NX><<<(unsigned)grid, tl::TC_THREADS, C::SMEM_BYTES, stream>>>(p);
     TL_CUDA(cudaGetLastError());
     return TL_OK;
@@ -411,6 +412,7 @@ extern "C" tl_status tl_nvfp4_verify_gemm_noalloc(const void* x, int M, const vo
     p.partials = nd->scratch->partials;
     p.counters = nd->scratch->counters;
     p.err = nd->scratch->err;
+    p.spread_mul = 0x1040u;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     // the counters must start at zero; a launch that gave up could have left them raised
     TL_CUDA(cudaMemsetAsync(p.counters, 0, sizeof(nd->scratch->counters), s));
