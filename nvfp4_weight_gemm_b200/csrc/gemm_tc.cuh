@@ -88,6 +88,7 @@ struct TcParams {
     unsigned* counters;     // [4 * gridDim.x], zero between launches
     int* err;               // device status word
     uint32_t spread_mul;    // 0x1040, passed at run time so the decode multiply stays one IMAD
+    uint32_t scale_mul;     // 0x00100010 (byte << 4 into both bf16 halves), likewise
     TcMat one;
 };
 
@@ -184,54 +185,30 @@ __device__ __forceinline__ uint32_t hmul2_bf16(uint32_t a, uint32_t b) {
     return d;
 }
 
-// Eight scale bytes -> eight bf16x2 words, both halves e4m3(s) * 2^119 (exact).
-// Fast path for finite, positive, normal scales (every scale the quantiser writes except
-// all-zero blocks): bf16 bits of s * 2^119 are ((s & 0x7F) << 4) + (239 << 7). Anything
-// else (zero or subnormal scale, sign bit, NaN) takes the exact float route.
-__device__ __forceinline__ void scales8_to_bf16x2(uint2 sc, uint32_t (&S)[8]) {
+// Scale bytes -> bf16x2 words, both halves e4m3(s) * 2^119 (exact).
+//
+// Fast path, for finite, positive, normal scales (every scale the quantiser writes except
+// all-zero blocks): the bf16 bits of s * 2^119 are (s << 4) + (239 << 7), which one IMAD forms
+// in both halves at once from the byte (s << 4 | s << 20) + 0x77807780. A tile's eight bytes are
+// checked once; anything else (zero or subnormal scale, sign bit, NaN) takes the exact float
+// route for the whole tile.
+__device__ __forceinline__ bool scales_fast_ok(uint2 sc) {
     const uint32_t e0 = sc.x & 0x78787878u, e1 = sc.y & 0x78787878u;
     const uint32_t zero_exp = ((e0 - 0x01010101u) & ~e0) | ((e1 - 0x01010101u) & ~e1);   // a byte had e == 0
     const uint32_t nan_or_neg = ((sc.x | sc.y) & 0x80808080u) |
                                 (((sc.x & 0x7F7F7F7Fu) + 0x01010101u) & 0x80808080u) |
                                 (((sc.y & 0x7F7F7F7Fu) + 0x01010101u) & 0x80808080u);   // bit 7 set or byte 0x7F
-    if (((zero_exp & 0x80808080u) | nan_or_neg) == 0u) {
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            // [b_lo, 0, b_hi, 0] -> bf16 of each scale * 2^119 in its own half
-            const uint32_t w = prmt(p < 2 ? sc.x : sc.y, 0u, (p & 1) ? 0x4342u : 0x4140u);
-            const uint32_t b = (w << 4) + 0x77807780u;
-            S[2 * p] = prmt(b, 0u, 0x1010u);
-            S[2 * p + 1] = prmt(b, 0u, 0x3232u);
-        }
-        return;
-    }
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-        const uint32_t two = ((p < 2 ? sc.x : sc.y) >> (16 * (p & 1))) & 0xFFFFu;
-        const __half2 h = e4m3x2_to_half2(two);
-        const float f0 = __low2float(h) * 0x1p119f;
-        const float f1 = __high2float(h) * 0x1p119f;
-        S[2 * p] = prmt(__float_as_uint(f0), 0u, 0x3232u);
-        S[2 * p + 1] = prmt(__float_as_uint(f1), 0u, 0x3232u);
-    }
+    return ((zero_exp & 0x80808080u) | nan_or_neg) == 0u;
 }
 
-// Four scale bytes -> four bf16x2 words, both halves e4m3(s) * 2^119 (exact); the same
-// fast path and exact fallback as the eight-byte form.
-__device__ __forceinline__ void scales4_to_bf16x2(uint32_t sc, uint32_t (&S)[4]) {
-    const uint32_t e = sc & 0x78787878u;
-    const uint32_t zero_exp = (e - 0x01010101u) & ~e;   // a byte had e == 0
-    const uint32_t nan_or_neg = (sc & 0x80808080u) | (((sc & 0x7F7F7F7Fu) + 0x01010101u) & 0x80808080u);
-    if (((zero_exp & 0x80808080u) | nan_or_neg) == 0u) {
+// Four scale bytes of `sc` (fast path only; see scales_fast_ok).
+__device__ __forceinline__ void scales4_fast(uint32_t sc, uint32_t mul, uint32_t (&S)[4]) {
 #pragma unroll
-        for (int p = 0; p < 2; ++p) {
-            const uint32_t w = prmt(sc, 0u, p ? 0x4342u : 0x4140u);
-            const uint32_t b = (w << 4) + 0x77807780u;
-            S[2 * p] = prmt(b, 0u, 0x1010u);
-            S[2 * p + 1] = prmt(b, 0u, 0x3232u);
-        }
-        return;
-    }
+    for (int p = 0; p < 4; ++p) S[p] = prmt(sc, 0u, 0x4440u | (uint32_t)p) * mul + 0x77807780u;
+}
+
+// Four scale bytes of `sc`, exactly, for any byte value.
+__device__ __forceinline__ void scales4_exact(uint32_t sc, uint32_t (&S)[4]) {
 #pragma unroll
     for (int p = 0; p < 2; ++p) {
         const __half2 h = e4m3x2_to_half2((sc >> (16 * p)) & 0xFFFFu);
@@ -476,6 +453,7 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
         for (int j = 0; j < 4; ++j) cw_off[j] = (uint32_t)(row_off + (((4 * kh + j) ^ row_sw) << 4));
         const long long ntiles = t_end - t_begin;
         const uint32_t spread = p.spread_mul;
+        const uint32_t smul = p.scale_mul;
         // this set's tiles are n = set, set + 2, ...: stage n % W_STAGES, slot n % NUM_A
         int s = set, a = set;
         uint32_t ph = 0, aph = 0;
@@ -507,8 +485,9 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
             const bool next_ready = __all_sync(0xFFFFFFFFu, has_next ? mbar_test(&wfull[s], ph) : true);
             // the slot must have been read by the MMAs of tile n - NUM_A
             const bool a_ready = __all_sync(0xFFFFFFFFu, mbar_test(&tfree[a], aph ^ 1u));
+            const bool fast = scales_fast_ok(sc);
             uint32_t S[4];
-            scales4_to_bf16x2(sc.x, S);
+            if (fast) scales4_fast(sc.x, smul, S); else scales4_exact(sc.x, S);
             uint32_t out[32];
             decode8(cw0.x, S[0], spread, &out[0]);
             decode8(cw0.y, S[0], spread, &out[4]);
@@ -531,7 +510,7 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
             tmem_st32(col, out);
             __syncwarp();
             if (lane == 0) mbar_arrive(&wempty[s_cur]);   // every byte of the stage this warp needs is in registers
-            scales4_to_bf16x2(sc.y, S);
+            if (fast) scales4_fast(sc.y, smul, S); else scales4_exact(sc.y, S);
             decode8(cw0.x, S[0], spread, &out[0]);
             decode8(cw0.y, S[0], spread, &out[4]);
             decode8(cw0.z, S[1], spread, &out[8]);

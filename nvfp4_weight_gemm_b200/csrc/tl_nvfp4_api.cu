@@ -209,6 +209,7 @@ tl_status launch_tc(DevState& d, tl::TcParams& p, cudaStream_t stream) {
     p.counters = d.counters;
     p.err = d.err;
     p.spread_mul = 0x1040u;
+    p.scale_mul = 0x00100010u;
     tl::gemm_tc_kernel<NX><<<(unsigned)grid, tl::TC_THREADS, C::SMEM_BYTES, stream>>>(p);
     TL_CUDA(cudaGetLastError());
     return TL_OK;
@@ -413,6 +414,7 @@ extern "C" tl_status tl_nvfp4_verify_gemm_noalloc(const void* x, int M, const vo
     p.counters = nd->scratch->counters;
     p.err = nd->scratch->err;
     p.spread_mul = 0x1040u;
+    p.scale_mul = 0x00100010u;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     // the counters must start at zero; a launch that gave up could have left them raised
     TL_CUDA(cudaMemsetAsync(p.counters, 0, sizeof(nd->scratch->counters), s));
