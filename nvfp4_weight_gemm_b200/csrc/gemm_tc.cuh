@@ -451,7 +451,7 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
         uint32_t cw_off[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) cw_off[j] = (uint32_t)(row_off + (((4 * kh + j) ^ row_sw) << 4));
-        const long long ntiles = t_end - t_begin;
+        const int ntiles = (int)(t_end - t_begin);   // a CTA's share is far below 2^31 tiles
         const uint32_t spread = p.spread_mul;
         const uint32_t smul = p.scale_mul;
         // this set's tiles are n = set, set + 2, ...: stage n % W_STAGES, slot n % NUM_A
@@ -480,11 +480,12 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
         }
         int s_cur = s;
         advance2(s, ph, C::W_STAGES);
-        for (long long n = set; ok && n < ntiles; n += 2) {
+        for (int n = set; ok && n < ntiles; n += 2) {
             const bool has_next = n + 2 < ntiles;
-            const bool next_ready = __all_sync(0xFFFFFFFFu, has_next ? mbar_test(&wfull[s], ph) : true);
-            // the slot must have been read by the MMAs of tile n - NUM_A
-            const bool a_ready = __all_sync(0xFFFFFFFFu, mbar_test(&tfree[a], aph ^ 1u));
+            // the next tile's stage, and this tile's slot (read by the MMAs of tile n - NUM_A):
+            // one vote when both are ready, the usual case; each is waited for on its own otherwise
+            const bool both_ready = __all_sync(0xFFFFFFFFu, (!has_next || mbar_test(&wfull[s], ph)) &&
+                                                             mbar_test(&tfree[a], aph ^ 1u));
             const bool fast = scales_fast_ok(sc);
             uint32_t S[4];
             if (fast) scales4_fast(sc.x, smul, S); else scales4_exact(sc.x, S);
@@ -500,7 +501,7 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
             // second chunk's codes: in flight while the first chunk is stored
             cw0 = *reinterpret_cast<const uint4*>(st_cur + cw_off[2]);
             cw1 = *reinterpret_cast<const uint4*>(st_cur + cw_off[3]);
-            if (!a_ready && !__all_sync(0xFFFFFFFFu, tc_wait(&tfree[a], aph ^ 1u, abort_flag))) {
+            if (!both_ready && !__all_sync(0xFFFFFFFFu, tc_wait(&tfree[a], aph ^ 1u, abort_flag))) {
                 if (lane == 0) tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_DEQUANT);
                 ok = false;
                 break;
@@ -522,7 +523,7 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
             tmem_st32(col + 32u, out);
             // the next tile's scales and first-chunk codes: in flight while the stores complete
             if (has_next) {
-                if (!next_ready && !__all_sync(0xFFFFFFFFu, tc_wait(&wfull[s], ph, abort_flag))) {
+                if (!both_ready && !__all_sync(0xFFFFFFFFu, tc_wait(&wfull[s], ph, abort_flag))) {
                     if (lane == 0) tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_DEQUANT);
                     ok = false;
                     break;
