@@ -40,6 +40,12 @@ WORKLOAD = ("64-layer verify-pass weight stream: 64 x {QKV 5120->7168, O 5120->5
             "one stack pass per M = 1..32")
 
 
+# tensor-core paths of the library (tl_set_gemm_path) and what one stack pass launches on each
+PATHS = {"block-scaled": 0, "bf16-exact": 1}
+KERNELS = {"block-scaled": "x_split_kernel + gemm_bs_kernel (two launches per stack pass, timed together)",
+           "bf16-exact": "gemm_tc_kernel (one launch per stack pass)"}
+
+
 def stack_shapes():
     import synth
     out = []
@@ -219,6 +225,8 @@ def main_gpu(args):
     if world > 1:
         dist.barrier()
     tl.init(local)
+    tl.set_gemm_path(PATHS[args.path])
+    launches_per_pass = 2 if args.path == "block-scaled" else 1
 
     shapes = stack_shapes()
     stack = build_stack(dev, seed=rank)
@@ -359,12 +367,12 @@ def main_gpu(args):
             "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "matrices": len(shapes), "weights": sum(N * K for (_, _, _, N, K, _) in shapes),
+            "config": {"workload": WORKLOAD, "path": args.path, "matrices": len(shapes), "weights": sum(N * K for (_, _, _, N, K, _) in shapes),
                        "w_bytes": w_bytes(shapes), "M": "1..32 (one pass each per step)",
                        "l2": "working set 11.9 GB >> 126 MB L2; no flush needed", "parallelism": f"replicas x{world}"},
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": traffic, "peak_kind": peak_kind,
-                         "kernel": "gemm_tc_kernel (one launch per stack pass)"},
+                         "kernel": KERNELS[args.path]},
             "staircase": stair,
             "min_frac_over_M": round(min(v["frac"] for v in stair.values()), 4),
             "m_invariance_row_fraction": inv,
@@ -372,7 +380,7 @@ def main_gpu(args):
                              "sample": CPU_SAMPLE_DESC},
             "e2e": {"value": round(world * bytes_step / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
                     "h2d_bytes_per_step": e2e_h2d, "d2h_bytes_per_step": e2e_d2h},
-            "gpu_launches": n_launch,
+            "gpu_launches": n_launch * launches_per_pass,
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
@@ -395,6 +403,7 @@ def run_profile_case(args):
     dev = torch.device("cuda:0")
     torch.cuda.set_device(dev)
     tl.init(0)
+    tl.set_gemm_path(PATHS[args.path])
     w = synth.w_f32_torch(N, K, 0, 0, dev)
     codes, scales, g = tl.quantize(w)
     del w
@@ -406,7 +415,7 @@ def run_profile_case(args):
     torch.cuda.synchronize()
     tl.check_device_error()
     plan.close()
-    print(json.dumps({"profile_case": f"{N}x{K}", "M": args.M, "reps": args.reps}), flush=True)
+    print(json.dumps({"profile_case": f"{N}x{K}", "M": args.M, "reps": args.reps, "path": args.path}), flush=True)
     return 0
 
 
@@ -419,6 +428,8 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--path", default="block-scaled", choices=sorted(PATHS),
+                    help="tensor-core path: block-scaled (default) or bf16-exact")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -68,6 +68,40 @@ typedef enum {
 /* Largest number of matrices one tl_nvfp4_verify_stack() call takes. */
 #define TL_NVFP4_MAX_STACK 1024
 
+/* Tensor-core paths of tl_nvfp4_verify_gemm(), tl_nvfp4_verify_stack(),
+ * tl_nvfp4_verify_stack_host() and of plans (a plan keeps the path that was selected
+ * when it was created). tl_nvfp4_verify_gemm_noalloc() always takes TL_PATH_BF16_EXACT.
+ *
+ * TL_PATH_BLOCK_SCALED (the default). Before the GEMM, a small kernel writes each row of
+ * X as a power of two times a sum of four NVFP4-shaped pieces (E2M1 codes with one E4M3
+ * scale per 16 k; each piece codes what the pieces before it left over). The GEMM then
+ * feeds the weights' codes and scales and those pieces straight into the FP4
+ * block-scaled tensor-core MMA, which decodes on the fly: no CUDA-core work per weight.
+ * Accuracy: each X element is represented to within (1.125/6)^4 (about 1.24e-3) of the
+ * largest |x| of its 16-element block, plus a floor about 2^-20 below the row's largest
+ * |x|. Spread over a dense row of W, as in real weights, that keeps Y within
+ * |y - y_ref| <= 1e-3 * sum_k |x w| + 2^-8 |y_ref| of the exact product (the pages'
+ * workload shapes and distributions are tested). A row of W with very few nonzero
+ * weights (an identity or one-hot matrix) can exceed that bound on an X element that is
+ * much smaller than its block's largest: use TL_PATH_BF16_EXACT for such weights. Reduction
+ * order is fixed, so runs are bit-identical, and a row's result does not depend on M. A
+ * row of X holding a NaN or an infinity gives NaN outputs for the whole row. The path
+ * needs scratch for the pieces, (4 * K/2 + 4 * K/16) * M + 4 * M bytes per matrix (256-byte
+ * aligned parts), allocated by the first call of a size (outside stream capture) and
+ * kept, or owned by a plan.
+ *
+ * TL_PATH_BF16_EXACT. CUDA cores decode each weight to bf16 (exact: an E2M1 value times
+ * an E4M3 scale has at most 6 significant bits) and the bf16 tensor-core MMA takes it
+ * with X as given, so products are exact and only the fp32 sums round. Slower: the
+ * decode is CUDA-core bound.
+ *
+ * tl_set_gemm_path() returns TL_ERR_INVALID_VALUE for any other value. The setting is
+ * process-wide; change it only while no call is in flight. */
+#define TL_PATH_BLOCK_SCALED 0
+#define TL_PATH_BF16_EXACT 1
+tl_status tl_set_gemm_path(int path);
+int tl_get_gemm_path(void);
+
 /* Create the per-device state of `device` (workspace, status word). Idempotent.
  * Does not change the calling thread's current device. */
 tl_status tl_init(int device);
@@ -82,9 +116,9 @@ void tl_shutdown(void);
  *   global_scale       finite
  *   y      device bf16 [M][N], 16-byte aligned; must not overlap x or W
  *   N      >= 1;  K  > 0 and K % 256 == 0
- * Kernel: the tensor-core path (tcgen05, A = dequantised W in tensor memory,
- * B = X in shared memory, fp32 accumulator in tensor memory), persistent
- * stream-K over all SMs; split-K partials are combined in fixed k order. */
+ * Kernel: the selected tensor-core path (tl_set_gemm_path; tcgen05 MMAs with the
+ * fp32 accumulator in tensor memory), persistent stream-K over all SMs; split-K
+ * partials are combined in fixed k order. */
 tl_status tl_nvfp4_verify_gemm(const void* x, int M, const void* w_codes, const void* w_scales,
                                float global_scale, void* y, int N, int K, void* stream);
 

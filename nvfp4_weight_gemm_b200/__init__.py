@@ -12,7 +12,8 @@ import ctypes
 from . import _lib
 from ._lib import Matrix, TlError, check
 
-__all__ = ["verify_gemm", "verify_gemm_simt", "verify_stack", "verify_stack_host", "Plan", "dequant",
+__all__ = ["verify_gemm", "verify_gemm_simt", "set_gemm_path", "get_gemm_path", "gemm_path", "PATH_BLOCK_SCALED",
+           "PATH_BF16_EXACT", "verify_stack", "verify_stack_host", "Plan", "dequant",
            "quantize", "check_device_error", "init", "num_sms", "Matrix", "TlError"]
 
 
@@ -32,6 +33,38 @@ def init(device: int = 0) -> None:
 
 def num_sms(device: int = 0) -> int:
     return _lib.lib().tl_num_sms(device)
+
+
+PATH_BLOCK_SCALED = _lib.TL_PATH_BLOCK_SCALED
+PATH_BF16_EXACT = _lib.TL_PATH_BF16_EXACT
+
+
+def set_gemm_path(path: int) -> None:
+    """Select the tensor-core path of verify_gemm, verify_stack(_host) and new plans:
+    PATH_BLOCK_SCALED (default; FP4 block-scaled MMA, within the stated tolerance) or
+    PATH_BF16_EXACT (CUDA-core decode to bf16, exact products)."""
+    check(_lib.lib().tl_set_gemm_path(path))
+
+
+def get_gemm_path() -> int:
+    return _lib.lib().tl_get_gemm_path()
+
+
+class gemm_path:
+    """Context manager: `with gemm_path(PATH_BF16_EXACT): ...` restores the previous path on exit."""
+
+    def __init__(self, path: int):
+        self.path = path
+        self.prev = None
+
+    def __enter__(self):
+        self.prev = get_gemm_path()
+        set_gemm_path(self.path)
+        return self
+
+    def __exit__(self, *exc):
+        set_gemm_path(self.prev)
+        return False
 
 
 def _gemm(name, x, codes, scales, global_scale, y=None, stream=None):

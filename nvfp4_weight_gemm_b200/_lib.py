@@ -26,8 +26,12 @@ EXPORTS = (
     "tl_nvfp4_verify_stack", "tl_nvfp4_verify_stack_host", "tl_nvfp4_plan_create",
     "tl_nvfp4_plan_run", "tl_nvfp4_plan_run_host", "tl_nvfp4_plan_destroy", "tl_nvfp4_dequant",
     "tl_nvfp4_quantize", "tl_check_device_error", "tl_selftest_bounded_wait", "tl_num_sms", "tl_status_string",
-    "tl_last_error_message",
+    "tl_last_error_message", "tl_set_gemm_path", "tl_get_gemm_path",
 )
+
+# Tensor-core paths (tl_set_gemm_path).
+TL_PATH_BLOCK_SCALED = 0
+TL_PATH_BF16_EXACT = 1
 
 
 class TlError(RuntimeError):
@@ -74,6 +78,8 @@ def lib() -> ctypes.CDLL:
             "tl_num_sms": [i],
             "tl_status_string": [i],
             "tl_last_error_message": [],
+            "tl_set_gemm_path": [i],
+            "tl_get_gemm_path": [],
         }
         for name, args in sig.items():
             fn = getattr(L, name)

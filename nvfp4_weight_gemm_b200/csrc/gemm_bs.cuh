@@ -1,0 +1,460 @@
+// gemm_bs.cuh -- block-scaled tensor-core NVFP4 verify GEMM for sm_100a (no CUDA-core dequant).
+//
+// Y[M,N] = X[M,K] . dequant(W)[N,K]^T for M <= 32 (TandemLLM docs v0.12.0, "What TandemLLM is",
+// section 1.2). W is already E2M1 with one E4M3 scale per 16 k, which is what
+// tcgen05.mma.kind::mxf4nvf4.block_scale consumes: the weight tile goes from HBM (TMA) into
+// shared memory and from there straight into the tensor core, with no decode on the CUDA
+// cores. X is brought into the same form beforehand (xsplit.cuh): per row a power of two and
+// TC_PIECES FP4 pieces with E4M3 scales. The pieces are stacked along the MMA's N dimension,
+// so one MMA per 64-k chunk serves every X row and every piece:
+//
+//   D[n][p * NX + m] = sum_k  w[n][k] * piece_p[m][k]        (fp32, in tensor memory)
+//   Y[m][n]          = bf16( (sum_p 4^-p D[n][p * NX + m]) * g * factor[m] )
+//
+//   * Work. As in gemm_tc.cuh: 128 weight rows x 256 k per tile, one global tile list cut into
+//     equal contiguous shares (stream-K); a split n-tile is reduced by its last contributor in
+//     k order, so every output has one fixed reduction order.
+//   * Roles, 12 warps.
+//     - Warp 0: TMA of W codes, W scales, X piece codes and X piece scales into a ring of
+//       stages (one 3-D copy each, from four lanes at once).
+//     - Warps 4..7: copy the tile's scales into tensor memory in the layout the MMA reads:
+//       lane 32q + l, columns 4c .. 4c+3 hold the scale words (four 16-k blocks each) of rows
+//       l, l + 32, l + 64, l + 96 for 64-k chunk c, for W and for the stacked X pieces.
+//       A W scale byte with the sign bit set (the MMA's scales are unsigned) is handled
+//       exactly: the codes of that block are negated in shared memory and the scale's sign is
+//       cleared.
+//     - Warp 1: one elected lane issues the four MMAs of a tile (M = 128, N = TC_PIECES * NX,
+//       K = 64 each) into the segment's accumulator.
+//     - Warps 8..11: the epilogue sums the pieces in fixed order and writes Y (or a partial).
+//
+// Every mbarrier wait is bounded; a wait that runs out records a status code and the CTA
+// winds down.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include "ptx.cuh"
+#include "gemm_tc.cuh"
+#include "xsplit.cuh"
+
+namespace tl {
+
+constexpr int BS_THREADS = 384;   // 12 warps
+constexpr int BS_SF_COLS = 32;    // tensor-memory columns of scales per stage (16 for W, 16 for X)
+
+struct alignas(64) BsMat {
+    CUtensorMap tm_codes;   // uint8 {K/2, N, 1}, box 128 B x 128 rows x 1, 128-byte swizzle
+    CUtensorMap tm_scales;  // uint8 {K/16, N, 1}, box 16 B x 128 rows x 1
+    CUtensorMap tm_xc;      // uint8 {K/2, M, TC_PIECES}, box 128 B x NX rows x TC_PIECES, 128-byte swizzle
+    CUtensorMap tm_xs;      // uint8 {K/16, M, TC_PIECES}, box 16 B x NX rows x TC_PIECES
+    const float* xfactor;   // [M], 2^-e per X row (NaN for a non-finite row)
+    __nv_bfloat16* y;
+    float g;                // the weight's tensor scale
+    int N;
+    int k_tiles;
+    int n_tiles;
+    long long tile_begin;
+};
+
+struct BsParams {
+    const BsMat* mats;      // device table, or nullptr to use `one`
+    int n_mats;
+    int M;
+    long long total_tiles;
+    float* partials;        // [2 * gridDim.x][32][128] fp32
+    unsigned* counters;     // [4 * gridDim.x], zero between launches
+    int* err;
+    BsMat one;
+};
+
+template <int NX>
+struct BsCfg {
+    static constexpr int CODES_BYTES = TC_BLOCK_N * (TC_BLOCK_K / 2);        // 16384
+    static constexpr int XC_BYTES = TC_PIECES * NX * (TC_BLOCK_K / 2);       // 8192 / 16384
+    static constexpr int SCALES_BYTES = TC_BLOCK_N * (TC_BLOCK_K / 16);      // 2048
+    static constexpr int XS_BYTES = TC_PIECES * NX * (TC_BLOCK_K / 16);      // 1024 / 2048
+    static constexpr int XC_OFF = CODES_BYTES;
+    static constexpr int SC_OFF = XC_OFF + XC_BYTES;
+    static constexpr int XS_OFF = SC_OFF + SCALES_BYTES;
+    static constexpr int STAGE_BYTES = XS_OFF + XS_BYTES;                    // 27648 / 36864
+    static constexpr int STAGES = (NX == 32) ? 6 : 8;
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 512 /*barriers*/;
+    static constexpr int N_MMA = TC_PIECES * NX;                             // 64 / 128
+    static constexpr int ACC_BUFS = 2;
+    static constexpr int SF_COL0 = 256;
+    static constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | ((uint32_t)(N_MMA >> 3) << 17) | (0u << 23) |
+                                      ((uint32_t)(TC_BLOCK_N >> 4) << 24);   // E2M1 x E2M1, UE4M3 scales
+    static_assert(STAGE_BYTES % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
+    static_assert(ACC_BUFS * N_MMA <= SF_COL0, "accumulators must fit below the scale columns");
+    static_assert(SF_COL0 + STAGES * BS_SF_COLS <= TC_TMEM_COLS, "tensor memory budget");
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+        ::"r"(taddr),
+          "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+          "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem], kind::mxf4nvf4 with one UE4M3 scale per 16 k from tensor memory.
+__device__ __forceinline__ void mma_bs_f4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
+// y[i][n] = bf16((v[i] * g) * factor[i]) for i < M (`y` already points at column n). All
+// factors are read before the first store, so the loads are not serialised behind stores.
+template <int NX>
+__device__ __forceinline__ void bs_store_rows(float (&v)[NX], int M, float g, const float* factor,
+                                              __nv_bfloat16* y, int ldy) {
+#pragma unroll
+    for (int i = 0; i < NX; ++i)
+        if (i < M) v[i] = (v[i] * g) * __ldg(factor + i);
+#pragma unroll
+    for (int i = 0; i < NX; ++i)
+        if (i < M) y[(long long)i * ldy] = __float2bfloat16_rn(v[i]);
+}
+
+template <int NX>
+__global__ void __launch_bounds__(BS_THREADS, 1)
+gemm_bs_kernel(const __grid_constant__ BsParams p) {
+    using C = BsCfg<NX>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+    uint64_t* full = bars;                          // [STAGES] all bytes of the stage landed
+    uint64_t* sfready = full + C::STAGES;           // [STAGES] scales of the stage in tensor memory (4 warps)
+    uint64_t* empty = sfready + C::STAGES;          // [STAGES] stage and its scale columns read by the MMAs
+    uint64_t* accfull = empty + C::STAGES;          // [2] accumulator complete
+    uint64_t* accempty = accfull + 2;               // [2] accumulator read (4 epilogue warps)
+    uint64_t* drain = accempty + 2;                 // [1] every MMA finished
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const BsMat* mats = p.mats ? p.mats : &p.one;
+    const long long ctas = gridDim.x;
+    const long long t_begin = tc_range_start(blockIdx.x, p.total_tiles, ctas);
+    const long long t_end = tc_range_start(blockIdx.x + 1, p.total_tiles, ctas);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < C::STAGES; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&sfready[i], 4);
+            mbar_init(&empty[i], 1);
+        }
+        for (int i = 0; i < C::ACC_BUFS; ++i) { mbar_init(&accfull[i], 1); mbar_init(&accempty[i], 4); }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, TC_TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        // Lanes 0..3 copy W codes, W scales, X piece codes and X piece scales of a stage with one
+        // converged rank-3 load; the whole warp waits for the stage.
+        const uint64_t pol = (lane < 2) ? policy_evict_first() : policy_evict_last();
+        const uint32_t dst_off = (lane == 0) ? 0u : (lane == 1) ? (uint32_t)C::SC_OFF
+                               : (lane == 2) ? (uint32_t)C::XC_OFF : (uint32_t)C::XS_OFF;
+        const uint32_t smem0 = smem_u32(smem);
+        int s = 0;
+        uint32_t ph = 0, issued = 0, last_ph = 0;
+        // segment walk over BsMat (the same tile list as TcSegIter's)
+        long long t = t_begin;
+        int mi = 0;
+        {
+            int lo = 0, hi = p.n_mats - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (mats[mid].tile_begin <= t_begin) lo = mid; else hi = mid - 1;
+            }
+            mi = lo;
+        }
+        bool ok = true;
+        while (ok && t < t_end) {
+            while (mi + 1 < p.n_mats && mats[mi + 1].tile_begin <= t) ++mi;
+            const BsMat& m = mats[mi];
+            const long long local = t - m.tile_begin;
+            const int ntile = (int)(local / m.k_tiles);
+            const int k0 = (int)(local % m.k_tiles);
+            const long long rem = t_end - t;
+            const int k1 = (int)((m.k_tiles - k0) < rem ? m.k_tiles : k0 + rem);
+            const void* tmap = (lane == 0) ? (const void*)&m.tm_codes : (lane == 1) ? (const void*)&m.tm_scales
+                             : (lane == 2) ? (const void*)&m.tm_xc : (const void*)&m.tm_xs;
+            const int c1 = (lane < 2) ? ntile * TC_BLOCK_N : 0;
+            for (int kt = k0; kt < k1; ++kt) {
+                const bool got = tc_wait(&empty[s], ph ^ 1u, abort_flag);
+                if (!__all_sync(0xFFFFFFFFu, got)) {
+                    if (lane == 0) tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_PRODUCER);
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)C::STAGE_BYTES);
+                __syncwarp();
+                const int c0 = (lane == 0 || lane == 2) ? kt * (TC_BLOCK_K / 2) : kt * (TC_BLOCK_K / 16);
+                if (lane < 4)
+                    tma_load_3d_s(smem0 + (uint32_t)(s * C::STAGE_BYTES) + dst_off, tmap, &full[s], c0, c1, 0, pol);
+                issued |= 1u << s;
+                last_ph = (last_ph & ~(1u << s)) | (ph << s);
+                if (++s == C::STAGES) { s = 0; ph ^= 1u; }
+            }
+            t += k1 - k0;
+        }
+        if (lane == 0) {
+            for (int i = 0; i < C::STAGES; ++i)
+                if ((issued >> i) & 1u)
+                    if (!mbar_wait(&full[i], (last_ph >> i) & 1u, TL_WAIT_LIMIT))
+                        tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_DRAIN);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (whole warp, elected lane)
+        const bool leader = elect_one();
+        int s = 0, acc = 0;
+        uint32_t ph = 0, accph = 0;
+        const uint64_t desc_w0 = smem_desc_k_sw128(smem_u32(smem));
+        const uint64_t desc_x0 = smem_desc_k_sw128(smem_u32(smem + C::XC_OFF));
+        long long t = t_begin;
+        int mi = 0;
+        {
+            int lo = 0, hi = p.n_mats - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (mats[mid].tile_begin <= t_begin) lo = mid; else hi = mid - 1;
+            }
+            mi = lo;
+        }
+        bool ok = true;
+        while (ok && t < t_end) {
+            while (mi + 1 < p.n_mats && mats[mi + 1].tile_begin <= t) ++mi;
+            const BsMat& m = mats[mi];
+            const long long local = t - m.tile_begin;
+            const int k0 = (int)(local % m.k_tiles);
+            const long long rem = t_end - t;
+            const int k1 = (int)((m.k_tiles - k0) < rem ? m.k_tiles : k0 + rem);
+            if (!__all_sync(0xFFFFFFFFu, tc_wait(&accempty[acc], accph ^ 1u, abort_flag))) {
+                if (leader) tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_MMA);
+                break;
+            }
+            tc_fence_after();
+            const uint32_t d_tmem = tmem + (uint32_t)(C::N_MMA * acc);
+            uint32_t first = 1;
+            for (int kt = k0; kt < k1; ++kt) {
+                if (!__all_sync(0xFFFFFFFFu, tc_wait(&full[s], ph, abort_flag) &&
+                                                 tc_wait(&sfready[s], ph, abort_flag))) {
+                    if (leader) tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_MMA);
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint64_t sdesc = (uint64_t)((s * C::STAGE_BYTES) >> 4);
+                const uint32_t sf = tmem + (uint32_t)(C::SF_COL0 + BS_SF_COLS * s);
+                if (leader) {
+#pragma unroll
+                    for (int kc = 0; kc < 4; ++kc)
+                        mma_bs_f4(d_tmem, desc_w0 + sdesc + (uint64_t)(2 * kc), desc_x0 + sdesc + (uint64_t)(2 * kc),
+                                  C::IDESC, sf + 4u * kc, sf + 16u + 4u * kc, (kc == 0) ? (first ^ 1u) : 1u);
+                    mma_commit(&empty[s]);
+                }
+                __syncwarp();
+                first = 0;
+                if (++s == C::STAGES) { s = 0; ph ^= 1u; }
+            }
+            if (!ok) break;
+            if (leader) mma_commit(&accfull[acc]);
+            __syncwarp();
+            if (++acc == C::ACC_BUFS) { acc = 0; accph ^= 1u; }
+            t += k1 - k0;
+        }
+        if (leader) mma_commit(drain);
+        __syncwarp();
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(drain, 0, TL_WAIT_LIMIT)) && lane == 0)
+            tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_DRAIN);
+    } else if (warp >= 4 && warp < 8) {
+        // ------------------------------------------------------------ scales into tensor memory
+        const int q = warp & 3;                         // this warp's tensor-memory lane quarter
+        const uint32_t t_lane = tmem + ((uint32_t)(32 * q) << 16);
+        const long long ntiles = t_end - t_begin;
+        int s = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        for (long long n = 0; ok && n < ntiles; ++n) {
+            if (!__all_sync(0xFFFFFFFFu, tc_wait(&full[s], ph, abort_flag))) {
+                if (lane == 0) tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_DEQUANT);
+                ok = false;
+                break;
+            }
+            uint8_t* st = smem + s * C::STAGE_BYTES;
+            uint4 wa[4], wb[4];
+#pragma unroll
+            for (int gq = 0; gq < 4; ++gq) {
+                const int r = lane + 32 * gq;
+                wa[gq] = *reinterpret_cast<const uint4*>(st + C::SC_OFF + 16 * r);
+                wb[gq] = (r < C::N_MMA) ? *reinterpret_cast<const uint4*>(st + C::XS_OFF + 16 * r) : make_uint4(0, 0, 0, 0);
+            }
+            // a scale byte with the sign bit set: negate that block's codes, keep |scale|
+            uint32_t neg = 0;
+#pragma unroll
+            for (int gq = 0; gq < 4; ++gq) neg |= (wa[gq].x | wa[gq].y | wa[gq].z | wa[gq].w) & 0x80808080u;
+            if (__any_sync(0xFFFFFFFFu, neg != 0u)) {
+                if (q == 0) {
+#pragma unroll
+                    for (int gq = 0; gq < 4; ++gq) {
+                        const int r = lane + 32 * gq;
+                        const uint32_t w4[4] = {wa[gq].x, wa[gq].y, wa[gq].z, wa[gq].w};
+#pragma unroll
+                        for (int b = 0; b < 16; ++b) {
+                            if ((w4[b >> 2] >> (8 * (b & 3) + 7)) & 1u) {
+                                // block b = bytes 8b .. 8b+7 of row r: 16-byte chunk b/2, half (b&1)
+                                uint2* c = reinterpret_cast<uint2*>(st + r * 128 + ((((b >> 1) ^ (r & 7))) << 4) + 8 * (b & 1));
+                                const uint2 v = *c;
+                                *c = make_uint2(v.x ^ 0x88888888u, v.y ^ 0x88888888u);
+                            }
+                        }
+                    }
+                    fence_proxy_async_smem();
+                }
+#pragma unroll
+                for (int gq = 0; gq < 4; ++gq) {
+                    wa[gq].x &= 0x7F7F7F7Fu; wa[gq].y &= 0x7F7F7F7Fu; wa[gq].z &= 0x7F7F7F7Fu; wa[gq].w &= 0x7F7F7F7Fu;
+                }
+            }
+            // column 4c + gq: scale word c (four 16-k blocks of chunk c) of row lane + 32 gq
+            uint32_t ca[16], cb[16];
+#pragma unroll
+            for (int gq = 0; gq < 4; ++gq) {
+                ca[0 + gq] = wa[gq].x; ca[4 + gq] = wa[gq].y; ca[8 + gq] = wa[gq].z; ca[12 + gq] = wa[gq].w;
+                cb[0 + gq] = wb[gq].x; cb[4 + gq] = wb[gq].y; cb[8 + gq] = wb[gq].z; cb[12 + gq] = wb[gq].w;
+            }
+            const uint32_t col = t_lane + (uint32_t)(C::SF_COL0 + BS_SF_COLS * s);
+            tmem_st16(col, ca);
+            tmem_st16(col + 16u, cb);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sfready[s]);
+            if (++s == C::STAGES) { s = 0; ph ^= 1u; }
+        }
+    } else if (warp >= 8) {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;
+        const int r = 32 * q + lane;
+        const uint32_t t_lane = tmem + ((uint32_t)(32 * q) << 16);
+        const int M = p.M;
+        int acc = 0;
+        uint32_t accph = 0;
+        long long t = t_begin;
+        int mi = 0;
+        {
+            int lo = 0, hi = p.n_mats - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (mats[mid].tile_begin <= t_begin) lo = mid; else hi = mid - 1;
+            }
+            mi = lo;
+        }
+        while (t < t_end) {
+            while (mi + 1 < p.n_mats && mats[mi + 1].tile_begin <= t) ++mi;
+            const BsMat& m = mats[mi];
+            const long long local = t - m.tile_begin;
+            const int ntile = (int)(local / m.k_tiles);
+            const int k0 = (int)(local % m.k_tiles);
+            const long long rem = t_end - t;
+            const int k1 = (int)((m.k_tiles - k0) < rem ? m.k_tiles : k0 + rem);
+            const long long seg_t0 = t;
+            t += k1 - k0;
+            // the matrix's fields in registers: stores to Y must not force them to be re-read
+            __nv_bfloat16* const yp = m.y;
+            const float gm = m.g;
+            const float* const xf = m.xfactor;
+            const int N = m.N;
+            if (!tc_wait(&accfull[acc], accph, abort_flag)) {
+                tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_EPILOGUE);
+                break;
+            }
+            tc_fence_after();
+            const int n = ntile * TC_BLOCK_N + r;
+            const bool whole = (k0 == 0 && k1 == m.k_tiles);
+            const long long ta = m.tile_begin + (long long)ntile * m.k_tiles;
+            const int my_slot = 2 * (int)blockIdx.x + (seg_t0 == t_begin ? 0 : 1);
+            float* mine = p.partials + (size_t)my_slot * (32 * TC_BLOCK_N);
+            // sum the pieces in order: v[mm] = sum_p 4^-p D[p * NX + mm] (exact scalings)
+            float v[NX];
+#pragma unroll
+            for (int i = 0; i < NX; ++i) v[i] = 0.0f;
+#pragma unroll
+            for (int pc = 0; pc < TC_PIECES; ++pc) {
+#pragma unroll
+                for (int c0 = 0; c0 < NX; c0 += 16) {
+                    uint32_t raw[16];
+                    tmem_ld16(t_lane + (uint32_t)(C::N_MMA * acc + pc * NX + c0), raw);
+                    tmem_wait_ld();
+                    const float unit = 1.0f / (float)(1 << (2 * pc));
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[c0 + i] = fmaf(__uint_as_float(raw[i]), unit, v[c0 + i]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&accempty[acc]);
+            if (++acc == C::ACC_BUFS) { acc = 0; accph ^= 1u; }
+            if (whole) {
+                if (n < N) bs_store_rows<NX>(v, M, gm, xf, yp + n, N);
+                continue;
+            }
+#pragma unroll
+            for (int i = 0; i < NX; ++i)
+                if (i < M) mine[i * TC_BLOCK_N + r] = v[i];
+            // split n-tile: the last contributor for these 32 rows adds all partials in k (CTA) order
+            const long long tb = ta + m.k_tiles;
+            const int f = tc_cta_of(ta, p.total_tiles, ctas);
+            const int l = tc_cta_of(tb - 1, p.total_tiles, ctas);
+            __threadfence();
+            __syncwarp();
+            unsigned old = 0;
+            if (lane == 0) old = atomicAdd(&p.counters[4 * f + q], 1u);
+            old = __shfl_sync(0xFFFFFFFFu, old, 0);
+            if (old == (unsigned)(l - f)) {
+                __threadfence();
+                for (int i = 0; i < NX; ++i) v[i] = 0.0f;
+                for (int c = f; c <= l; ++c) {
+                    const long long cs = tc_range_start(c, p.total_tiles, ctas);
+                    const int slot = 2 * c + ((ta > cs ? ta : cs) == cs ? 0 : 1);
+                    const float* part = p.partials + (size_t)slot * (32 * TC_BLOCK_N);
+#pragma unroll
+                    for (int i = 0; i < NX; ++i)
+                        if (i < M) v[i] += __ldcg(&part[i * TC_BLOCK_N + r]);
+                }
+                if (n < N) bs_store_rows<NX>(v, M, gm, xf, yp + n, N);
+                if (lane == 0) p.counters[4 * f + q] = 0u;   // ready for the next launch
+            }
+        }
+    }
+    __syncwarp();
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TC_TMEM_COLS);
+    }
+}
+
+}  // namespace tl

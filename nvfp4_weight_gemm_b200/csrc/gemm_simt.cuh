@@ -3,8 +3,9 @@
 // The plain form of Y[M,N] = X[M,K] . dequant(W)[N,K]^T: each warp streams one weight
 // row, lanes take 16-element K blocks in turn (lane l: blocks l, l+32, ...), every lane
 // keeps an fp32 accumulator per X row, a fixed xor-butterfly adds the lanes. Per block:
-// s = sum_j x[m,16b+j] * e2m1[n,16b+j], then acc += s * e4m3[n,b]; the tensor scale is
-// applied once in the epilogue. Used for the smallest M, where the row count leaves the
+// s = sum_j x[m,16b+j] * e2m1[n,16b+j], then acc += s * (e4m3[n,b] * g): the tensor scale
+// goes in with the block scale, so the running sum keeps the magnitude of the result and
+// cannot overflow fp32 where Y itself does not. Used for the smallest M, where the row count leaves the
 // tensor core idle, and as a second GPU path for cross-checks.
 #pragma once
 #include <cstdint>
@@ -31,7 +32,7 @@ gemm_simt_kernel(const __nv_bfloat16* __restrict__ x, int M, const uint8_t* __re
 
     for (int b = lane; b < nb; b += 32) {
         const uint2 c = crow[b];
-        const float s = e4m3_to_float(srow[b]);
+        const float s = e4m3_to_float(srow[b]) * g;
         float v[16];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -64,7 +65,7 @@ gemm_simt_kernel(const __nv_bfloat16* __restrict__ x, int M, const uint8_t* __re
     // lane m writes row m (each lane holds every sum after the butterfly)
 #pragma unroll
     for (int m = 0; m < MAXM; ++m)
-        if (m == lane && m < M) y[(int64_t)m * N + n] = __float2bfloat16_rn(acc[m] * g);
+        if (m == lane && m < M) y[(int64_t)m * N + n] = __float2bfloat16_rn(acc[m]);
 }
 
 }  // namespace tl

@@ -559,6 +559,9 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
             }
             tc_fence_after();
             const TcMat& m = mats[sg.mat];
+            // the matrix's fields in registers: stores to Y must not force them to be re-read
+            __nv_bfloat16* const yp = m.y;
+            const float g_out = m.g_out;
             const int N = m.N;
             const int n = sg.ntile * TC_BLOCK_N + r;
             const bool whole = (sg.k0 == 0 && sg.k1 == m.k_tiles);
@@ -589,7 +592,7 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
                 if (n < N) {
 #pragma unroll
                     for (int i = 0; i < NX; ++i)
-                        if (i < M) m.y[(long long)i * N + n] = __float2bfloat16_rn(v[i] * m.g_out);
+                        if (i < M) yp[(long long)i * N + n] = __float2bfloat16_rn(v[i] * g_out);
                 }
             } else {
 #pragma unroll
@@ -626,7 +629,7 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
                     if (n < N) {
 #pragma unroll
                         for (int i = 0; i < 16; ++i)
-                            if (c0 + i < M) m.y[(long long)(c0 + i) * N + n] = __float2bfloat16_rn(v[i] * m.g_out);
+                            if (c0 + i < M) yp[(long long)(c0 + i) * N + n] = __float2bfloat16_rn(v[i] * g_out);
                     }
                 }
                 if (lane == 0) p.counters[4 * f + q] = 0u;   // ready for the next launch

@@ -19,6 +19,7 @@
 
 #include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
+#include "gemm_bs.cuh"
 #include "kernels_aux.cuh"
 
 namespace {
@@ -45,8 +46,8 @@ constexpr int kMaxDevices = 64;
 constexpr int kStackCacheSlots = 8;
 
 struct StackCacheEntry {
-    std::vector<unsigned char> key;   // host bytes of the TcMat table
-    tl::TcMat* table = nullptr;       // device copy
+    std::vector<unsigned char> key;   // host bytes of a descriptor table
+    void* table = nullptr;            // device copy
     unsigned long long last_use = 0;
 };
 
@@ -58,12 +59,15 @@ struct DevState {
     unsigned* counters = nullptr;  // [4 * num_sms]
     unsigned* qscratch = nullptr;  // quantiser absmax + non-finite flag
     bool smem_attr_set = false;
+    unsigned char* xs_buf = nullptr;   // X pieces of the block-scaled path (calls without a plan)
+    size_t xs_cap = 0;
     StackCacheEntry cache[kStackCacheSlots];
     unsigned long long use_clock = 0;
 };
 
 std::mutex g_mu;
 DevState g_dev[kMaxDevices];
+int g_path = TL_PATH_BLOCK_SCALED;   // which tensor-core path the GEMM entry points take
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 tl_status load_encode_fn() {
@@ -225,10 +229,10 @@ tl_status check_M(int M) {
     return TL_OK;
 }
 
-// Device table of a stack's TcMat array: reused while the same matrices come back.
-tl_status stack_table(DevState& d, const std::vector<tl::TcMat>& mats, cudaStream_t stream, const tl::TcMat** out) {
-    const size_t bytes = mats.size() * sizeof(tl::TcMat);
-    const unsigned char* key = reinterpret_cast<const unsigned char*>(mats.data());
+// Device copy of a stack's descriptor table (host bytes `key`): reused while the same
+// matrices come back.
+tl_status device_table(DevState& d, const void* key_, size_t bytes, cudaStream_t stream, const void** out) {
+    const unsigned char* key = static_cast<const unsigned char*>(key_);
     std::lock_guard<std::mutex> lk(g_mu);
     ++d.use_clock;
     for (auto& e : d.cache) {
@@ -256,6 +260,13 @@ tl_status stack_table(DevState& d, const std::vector<tl::TcMat>& mats, cudaStrea
     victim->last_use = d.use_clock;
     *out = victim->table;
     return TL_OK;
+}
+
+tl_status stack_table(DevState& d, const std::vector<tl::TcMat>& mats, cudaStream_t stream, const tl::TcMat** out) {
+    const void* t = nullptr;
+    tl_status st = device_table(d, mats.data(), mats.size() * sizeof(tl::TcMat), stream, &t);
+    *out = static_cast<const tl::TcMat*>(t);
+    return st;
 }
 
 // Validate a stack and build its launch parameters (host side only, plus the
@@ -310,6 +321,9 @@ tl_status build_params(const tl_nvfp4_matrix* mats, int n_mats, int M, const uns
     return TL_OK;
 }
 
+tl_status run_stack_bs(const tl_nvfp4_matrix* mats, int n_mats, int M, const unsigned char* x_dev,
+                       unsigned char* y_dev, void* stream_, DevState* d);
+
 tl_status run_stack(const tl_nvfp4_matrix* mats, int n_mats, int M, const unsigned char* x_dev,
                     unsigned char* y_dev, void* stream_) {
     DevState* d = nullptr;
@@ -317,12 +331,170 @@ tl_status run_stack(const tl_nvfp4_matrix* mats, int n_mats, int M, const unsign
     std::vector<tl::TcMat> tbl;
     tl_status st = build_params(mats, n_mats, M, x_dev, y_dev, &d, &p, &tbl);
     if (st != TL_OK || M == 0) return st;
+    if (g_path == TL_PATH_BLOCK_SCALED) return run_stack_bs(mats, n_mats, M, x_dev, y_dev, stream_, d);
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
     if (n_mats > 1) {
         st = stack_table(*d, tbl, stream, &p.mats);
         if (st != TL_OK) return st;
     }
     return launch_tc_any(*d, p, stream);
+}
+
+
+// ---------------------------------------------------------------------------
+// The block-scaled path: X split into FP4 pieces, then W and the pieces straight into the
+// tensor core (gemm_bs.cuh, xsplit.cuh).
+
+size_t round256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// Bytes of the X pieces (codes, scales, row factors) of one matrix with M rows and K columns.
+size_t xs_bytes_of(int M, int K) {
+    return round256((size_t)tl::TC_PIECES * M * (K / 2)) + round256((size_t)tl::TC_PIECES * M * (K / 16)) +
+           round256((size_t)4 * M);
+}
+
+size_t xs_bytes_total(const tl_nvfp4_matrix* mats, int n_mats, int M) {
+    size_t t = 0;
+    for (int i = 0; i < n_mats; ++i) t += xs_bytes_of(M, mats[i].K);
+    return t;
+}
+
+// BsMat of one matrix whose X pieces live at `xs` (layout of xs_bytes_of).
+tl_status build_bs_mat(tl::BsMat* m, tl::XSplitMat* xm, const void* x, int M, int NX, const void* codes,
+                       const void* scales, float g, void* y, int N, int K, long long tile_begin, unsigned char* xs) {
+    memset(m, 0, sizeof *m);
+    const cuuint64_t n = (cuuint64_t)N, k = (cuuint64_t)K, mm = (cuuint64_t)M, P = (cuuint64_t)tl::TC_PIECES;
+    unsigned char* xc = xs;
+    unsigned char* xsc = xc + round256((size_t)P * M * (K / 2));
+    float* xf = reinterpret_cast<float*>(xsc + round256((size_t)P * M * (K / 16)));
+    tl_status st = encode_3d(&m->tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, {k / 2, n, 1}, {k / 2, n * (k / 2)},
+                             {tl::TC_BLOCK_K / 2, tl::TC_BLOCK_N, 1}, CU_TENSOR_MAP_SWIZZLE_128B, "codes");
+    if (st != TL_OK) return st;
+    st = encode_3d(&m->tm_scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, scales, {k / 16, n, 1}, {k / 16, n * (k / 16)},
+                   {tl::TC_BLOCK_K / 16, tl::TC_BLOCK_N, 1}, CU_TENSOR_MAP_SWIZZLE_NONE, "scales");
+    if (st != TL_OK) return st;
+    // X pieces: {K/2 bytes, M rows, pieces}; a box {128, NX, pieces} stacks the pieces of a tile
+    // as the MMA's N = pieces x NX rows (rows >= M read zero)
+    st = encode_3d(&m->tm_xc, CU_TENSOR_MAP_DATA_TYPE_UINT8, xc, {k / 2, mm, P}, {k / 2, mm * (k / 2)},
+                   {tl::TC_BLOCK_K / 2, (cuuint32_t)NX, (cuuint32_t)P}, CU_TENSOR_MAP_SWIZZLE_128B, "X piece codes");
+    if (st != TL_OK) return st;
+    st = encode_3d(&m->tm_xs, CU_TENSOR_MAP_DATA_TYPE_UINT8, xsc, {k / 16, mm, P}, {k / 16, mm * (k / 16)},
+                   {tl::TC_BLOCK_K / 16, (cuuint32_t)NX, (cuuint32_t)P}, CU_TENSOR_MAP_SWIZZLE_NONE, "X piece scales");
+    if (st != TL_OK) return st;
+    m->xfactor = xf;
+    m->y = static_cast<__nv_bfloat16*>(y);
+    m->g = g;
+    m->N = N;
+    m->k_tiles = K / tl::TC_BLOCK_K;
+    m->n_tiles = (N + tl::TC_BLOCK_N - 1) / tl::TC_BLOCK_N;
+    m->tile_begin = tile_begin;
+    xm->x = static_cast<const __nv_bfloat16*>(x);
+    xm->codes = xc;
+    xm->scales = xsc;
+    xm->factor = xf;
+    xm->K = K;
+    return TL_OK;
+}
+
+struct BsLaunch {
+    tl::BsParams bp;
+    tl::XSplitParams xp;
+    std::vector<tl::BsMat> tbl;
+    std::vector<tl::XSplitMat> xtbl;
+};
+
+// Validate (as build_params) and build the block-scaled launch of a stack whose X pieces go to
+// `xs` (xs_bytes_total bytes).
+tl_status build_bs(const tl_nvfp4_matrix* mats, int n_mats, int M, const unsigned char* x_dev, unsigned char* y_dev,
+                   unsigned char* xs, BsLaunch* L) {
+    const int NX = M <= 16 ? 16 : 32;
+    L->tbl.assign(n_mats, tl::BsMat());
+    L->xtbl.assign(n_mats, tl::XSplitMat());
+    long long tiles = 0;
+    size_t xoff = 0, yoff = 0, soff = 0;
+    for (int i = 0; i < n_mats; ++i) {
+        const tl_nvfp4_matrix& m = mats[i];
+        const void* x = x_dev ? static_cast<const void*>(x_dev + xoff) : m.x;
+        void* y = y_dev ? static_cast<void*>(y_dev + yoff) : m.y;
+        tl_status st = build_bs_mat(&L->tbl[i], &L->xtbl[i], x, M, NX, m.w_codes, m.w_scales, m.global_scale, y,
+                                    m.N, m.K, tiles, xs + soff);
+        if (st != TL_OK) return st;
+        tiles += (long long)L->tbl[i].n_tiles * L->tbl[i].k_tiles;
+        xoff += (size_t)2 * M * m.K;
+        yoff += (size_t)2 * M * m.N;
+        soff += xs_bytes_of(M, m.K);
+    }
+    memset(&L->bp, 0, sizeof L->bp);
+    L->bp.n_mats = n_mats;
+    L->bp.M = M;
+    L->bp.total_tiles = tiles;
+    L->bp.mats = nullptr;
+    if (n_mats == 1) L->bp.one = L->tbl[0];
+    memset(&L->xp, 0, sizeof L->xp);
+    L->xp.n_mats = n_mats;
+    L->xp.M = M;
+    L->xp.mats = nullptr;
+    if (n_mats == 1) L->xp.one = L->xtbl[0];
+    return TL_OK;
+}
+
+template <int NX>
+tl_status launch_bs_gemm(DevState& d, tl::BsParams& p, cudaStream_t stream) {
+    using C = tl::BsCfg<NX>;
+    TL_CUDA(cudaFuncSetAttribute(tl::gemm_bs_kernel<NX>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
+    const long long grid = p.total_tiles < d.num_sms ? p.total_tiles : d.num_sms;
+    p.partials = d.partials;
+    p.counters = d.counters;
+    p.err = d.err;
+    tl::gemm_bs_kernel<NX><<<(unsigned)grid, tl::BS_THREADS, C::SMEM_BYTES, stream>>>(p);
+    TL_CUDA(cudaGetLastError());
+    return TL_OK;
+}
+
+// The X split, then the GEMM, on `stream`.
+tl_status launch_bs(DevState& d, tl::BsParams bp, const tl::XSplitParams& xp, cudaStream_t stream) {
+    tl::x_split_kernel<<<dim3((unsigned)xp.M, (unsigned)xp.n_mats), tl::XS_THREADS, 0, stream>>>(xp);
+    TL_CUDA(cudaGetLastError());
+    return (bp.M <= 16) ? launch_bs_gemm<16>(d, bp, stream) : launch_bs_gemm<32>(d, bp, stream);
+}
+
+// Grow the per-device X-piece scratch to `bytes` (never inside a graph capture).
+tl_status ensure_xs(DevState& d, size_t bytes, cudaStream_t stream) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (d.xs_cap >= bytes) return TL_OK;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    TL_CUDA(cudaStreamIsCapturing(stream, &cs));
+    if (cs != cudaStreamCaptureStatusNone)
+        return fail(TL_ERR_UNSUPPORTED, "the block-scaled path must run once at this size before graph capture");
+    if (d.xs_buf) {
+        TL_CUDA(cudaDeviceSynchronize());   // a kernel in flight may still use the old buffer
+        TL_CUDA(cudaFree(d.xs_buf));
+        d.xs_buf = nullptr;
+        d.xs_cap = 0;
+    }
+    TL_CUDA(cudaMalloc(&d.xs_buf, bytes));
+    d.xs_cap = bytes;
+    return TL_OK;
+}
+
+tl_status run_stack_bs(const tl_nvfp4_matrix* mats, int n_mats, int M, const unsigned char* x_dev,
+                       unsigned char* y_dev, void* stream_, DevState* d) {
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    tl_status st = ensure_xs(*d, xs_bytes_total(mats, n_mats, M), stream);
+    if (st != TL_OK) return st;
+    BsLaunch L;
+    st = build_bs(mats, n_mats, M, x_dev, y_dev, d->xs_buf, &L);
+    if (st != TL_OK) return st;
+    if (n_mats > 1) {
+        const void* t = nullptr;
+        st = device_table(*d, L.tbl.data(), L.tbl.size() * sizeof(tl::BsMat), stream, &t);
+        if (st != TL_OK) return st;
+        L.bp.mats = static_cast<const tl::BsMat*>(t);
+        st = device_table(*d, L.xtbl.data(), L.xtbl.size() * sizeof(tl::XSplitMat), stream, &t);
+        if (st != TL_OK) return st;
+        L.xp.mats = static_cast<const tl::XSplitMat*>(t);
+    }
+    return launch_bs(*d, L.bp, L.xp, stream);
 }
 
 
@@ -432,12 +604,49 @@ extern "C" tl_status tl_nvfp4_verify_gemm_noalloc(const void* x, int M, const vo
 struct tl_nvfp4_plan_st {
     int device = 0;
     DevState* d = nullptr;
+    int path = TL_PATH_BLOCK_SCALED;  // fixed when the plan is made
     tl::TcParams params;
     tl::TcMat* table = nullptr;       // device copy when n_mats > 1
+    tl::BsParams bparams;             // block-scaled path
+    tl::XSplitParams xparams;
+    void* bs_tables = nullptr;        // device copies of the BsMat and XSplitMat tables (n_mats > 1)
+    unsigned char* xs = nullptr;      // the plan's own X-piece scratch
     const void* x_base = nullptr;     // packed X_i buffer (or nullptr if not packed)
     void* y_base = nullptr;           // packed Y_i buffer (or nullptr if not packed)
     size_t x_bytes = 0, y_bytes = 0;
 };
+
+namespace {
+
+// The block-scaled launch of a plan: own X-piece scratch and own device tables, so that a plan
+// never shares memory with another plan or with calls made without one.
+tl_status plan_build_bs(tl_nvfp4_plan plan, const tl_nvfp4_matrix* mats, int n_mats, int M) {
+    TL_CUDA(cudaMalloc(&plan->xs, xs_bytes_total(mats, n_mats, M)));
+    BsLaunch L;
+    tl_status st = build_bs(mats, n_mats, M, nullptr, nullptr, plan->xs, &L);
+    if (st != TL_OK) return st;
+    if (n_mats > 1) {
+        const size_t b1 = round256(L.tbl.size() * sizeof(tl::BsMat));
+        const size_t b2 = L.xtbl.size() * sizeof(tl::XSplitMat);
+        TL_CUDA(cudaMalloc(&plan->bs_tables, b1 + b2));
+        unsigned char* t = static_cast<unsigned char*>(plan->bs_tables);
+        TL_CUDA(cudaMemcpy(t, L.tbl.data(), L.tbl.size() * sizeof(tl::BsMat), cudaMemcpyHostToDevice));
+        TL_CUDA(cudaMemcpy(t + b1, L.xtbl.data(), b2, cudaMemcpyHostToDevice));
+        L.bp.mats = reinterpret_cast<const tl::BsMat*>(t);
+        L.xp.mats = reinterpret_cast<const tl::XSplitMat*>(t + b1);
+    }
+    plan->bparams = L.bp;
+    plan->xparams = L.xp;
+    return TL_OK;
+}
+
+tl_status plan_launch(tl_nvfp4_plan plan, cudaStream_t s) {
+    if (plan->path == TL_PATH_BLOCK_SCALED) return launch_bs(*plan->d, plan->bparams, plan->xparams, s);
+    tl::TcParams p = plan->params;
+    return launch_tc_any(*plan->d, p, s);
+}
+
+}  // namespace
 
 extern "C" {
 
@@ -454,12 +663,18 @@ tl_status tl_nvfp4_plan_create(const tl_nvfp4_matrix* mats, int n_mats, int M, t
     TL_CUDA(cudaGetDevice(&plan->device));
     plan->d = d;
     plan->params = p;
-    if (n_mats > 1) {
+    plan->path = g_path;
+    if (plan->path == TL_PATH_BLOCK_SCALED) {
+        st = plan_build_bs(plan, mats, n_mats, M);
+        if (st != TL_OK) {
+            tl_nvfp4_plan_destroy(plan);
+            return st;
+        }
+    } else if (n_mats > 1) {
         const size_t bytes = tbl.size() * sizeof(tl::TcMat);
         if (cudaMalloc(&plan->table, bytes) != cudaSuccess ||
             cudaMemcpy(plan->table, tbl.data(), bytes, cudaMemcpyHostToDevice) != cudaSuccess) {
-            if (plan->table) cudaFree(plan->table);
-            delete plan;
+            tl_nvfp4_plan_destroy(plan);
             return fail(TL_ERR_CUDA, "uploading the plan's descriptor table failed");
         }
         plan->params.mats = plan->table;
@@ -483,8 +698,7 @@ tl_status tl_nvfp4_plan_create(const tl_nvfp4_matrix* mats, int n_mats, int M, t
 
 tl_status tl_nvfp4_plan_run(tl_nvfp4_plan plan, void* stream) {
     if (!plan) return fail(TL_ERR_INVALID_VALUE, "plan is null");
-    tl::TcParams p = plan->params;
-    return launch_tc_any(*plan->d, p, static_cast<cudaStream_t>(stream));
+    return plan_launch(plan, static_cast<cudaStream_t>(stream));
 }
 
 tl_status tl_nvfp4_plan_run_host(tl_nvfp4_plan plan, const void* x_host, void* y_host, void* stream) {
@@ -494,8 +708,7 @@ tl_status tl_nvfp4_plan_run_host(tl_nvfp4_plan plan, const void* x_host, void* y
         return fail(TL_ERR_INVALID_VALUE, "the plan's X and Y buffers are not packed back to back");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     TL_CUDA(cudaMemcpyAsync(const_cast<void*>(plan->x_base), x_host, plan->x_bytes, cudaMemcpyHostToDevice, s));
-    tl::TcParams p = plan->params;
-    tl_status st = launch_tc_any(*plan->d, p, s);
+    tl_status st = plan_launch(plan, s);
     if (st != TL_OK) return st;
     TL_CUDA(cudaMemcpyAsync(y_host, plan->y_base, plan->y_bytes, cudaMemcpyDeviceToHost, s));
     return TL_OK;
@@ -503,16 +716,31 @@ tl_status tl_nvfp4_plan_run_host(tl_nvfp4_plan plan, const void* x_host, void* y
 
 tl_status tl_nvfp4_plan_destroy(tl_nvfp4_plan plan) {
     if (!plan) return TL_OK;
-    if (plan->table) {
+    if (plan->table || plan->bs_tables || plan->xs) {
         int prev = 0;
         cudaGetDevice(&prev);
         cudaSetDevice(plan->device);
         cudaDeviceSynchronize();
-        cudaFree(plan->table);
+        if (plan->table) cudaFree(plan->table);
+        if (plan->bs_tables) cudaFree(plan->bs_tables);
+        if (plan->xs) cudaFree(plan->xs);
         cudaSetDevice(prev);
     }
     delete plan;
     return TL_OK;
+}
+
+tl_status tl_set_gemm_path(int path) {
+    if (path != TL_PATH_BLOCK_SCALED && path != TL_PATH_BF16_EXACT)
+        return fail(TL_ERR_INVALID_VALUE, "unknown GEMM path %d", path);
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_path = path;
+    return TL_OK;
+}
+
+int tl_get_gemm_path(void) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    return g_path;
 }
 
 tl_status tl_init(int device) {
@@ -537,6 +765,7 @@ void tl_shutdown(void) {
         cudaFree(d.qscratch);
         for (auto& e : d.cache)
             if (e.table) cudaFree(e.table);
+        if (d.xs_buf) cudaFree(d.xs_buf);
         d = DevState();
     }
     cudaSetDevice(prev);

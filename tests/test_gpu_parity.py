@@ -3,10 +3,13 @@
 Bars (all written here):
   * dequantised weights and quantiser output: bit-exact;
   * Y: |y - y_ref| <= 1e-3 * sum_k |x_k w_k| + 2^-8 * |y_ref| per element (fp32 accumulation,
-    one bf16 rounding: the 2^-8 term covers the output rounding);
+    one bf16 rounding: the 2^-8 term covers the output rounding), on every GEMM path: the
+    block-scaled tensor-core path (X as FP4 pieces), the exact bf16 tensor-core path and the
+    CUDA-core path; NaN only where the reference is NaN;
   * cases whose exact result is representable (identity, one-hot, small integers): bit-exact
-    against bf16(y_ref);
-  * determinism: repeated runs bit-identical.
+    against bf16(y_ref) on the exact paths (bf16 tensor-core, CUDA-core), within the
+    tolerance on the block-scaled one;
+  * determinism: repeated runs bit-identical on every path.
 """
 
 import numpy as np
@@ -56,11 +59,18 @@ def bf16_round(a):
 
 
 def assert_within_tol(y, y_ref, a_ref, what=""):
+    """The per-element bar; a NaN (or infinity) passes only where the reference has the same."""
+    y, y_ref, a_ref = np.asarray(y), np.asarray(y_ref), np.asarray(a_ref)
     tol = 1e-3 * a_ref + 2.0 ** -8 * np.abs(y_ref)
-    err = np.abs(y - y_ref)
-    bad = err > tol
-    assert not bad.any(), (f"{what}: {bad.sum()} of {bad.size} outside tolerance; worst excess "
-                           f"{np.max(err - tol):.3e} at {np.unravel_index(np.argmax(err - tol), err.shape)}")
+    with np.errstate(invalid="ignore"):
+        err = np.abs(y - y_ref)
+        same_special = (np.isnan(y) & np.isnan(y_ref)) | (np.isinf(y) & (y == y_ref))
+        bad = ~((err <= tol) | same_special)
+    if bad.any():
+        excess = np.where(bad, np.nan_to_num(err - tol, nan=np.inf), -np.inf)
+        at = np.unravel_index(np.argmax(excess), excess.shape)
+        raise AssertionError(f"{what}: {bad.sum()} of {bad.size} outside tolerance; worst at {at}: "
+                             f"y={y[at]!r} ref={y_ref[at]!r} tol={tol[at]!r}")
 
 
 def make_weight(N, K, seed, tid, dist="normal"):
@@ -69,14 +79,52 @@ def make_weight(N, K, seed, tid, dist="normal"):
     return w, codes, scales, g
 
 
-def run_both_paths(x_bits, codes, scales, g):
+TC_PATHS = {"block-scaled": tl.PATH_BLOCK_SCALED, "bf16-exact": tl.PATH_BF16_EXACT}
+
+# The block-scaled path writes each X element as four FP4 pieces with per-16-block scales: an
+# element is off by at most (1.125/6)^4 of its block's largest |x| (each piece leaves at most
+# one E4M3 rounding step above 1/6 of the block's residual), plus a floor far below the row's
+# largest |x|. That error is spread over every term of a dense row of W, so the standard
+# tolerance holds there; a row of W with a single nonzero (identity, one-hot) sees it alone.
+SPLIT_RHO = 1.01 * (1.125 / 6.0) ** 4
+SPLIT_FLOOR = 2.0 ** -20
+
+
+def split_bound(x_bits, codes, scales, g):
+    """Standard tolerance plus the block-scaled split's own error bound, per output (fp64)."""
+    xf = np.abs(synth.bf16_bits_to_f32(x_bits).astype(np.float64))
+    M, K = xf.shape
+    blk = np.repeat(xf.reshape(M, K // 16, 16).max(axis=2), 16, axis=1)     # block max per element
+    _, wq = oracle.dequant(codes, scales, g, want_wq=True)
+    aw = np.abs(wq) * abs(g)
+    return SPLIT_RHO * (blk @ aw.T) + SPLIT_FLOOR * xf.max(axis=1, keepdims=True) * aw.sum(axis=1)[None, :]
+
+
+def assert_within_bound(y, y_ref, bound, what=""):
+    with np.errstate(invalid="ignore"):
+        bad = ~(np.abs(y - y_ref) <= bound)
+    assert not bad.any(), f"{what}: {bad.sum()} of {bad.size} outside the bound"
+
+
+def gemm_on(path, x, c, s, g):
+    with tl.gemm_path(TC_PATHS[path]):
+        return tl.verify_gemm(x, c, s, g)
+
+
+def run_paths(x_bits, codes, scales, g):
+    """Y from every path: {"block-scaled", "bf16-exact", "simt"} -> fp64 host arrays."""
     x = dev_bf16(x_bits)
     c, s = dev_u8(codes), dev_u8(scales)
-    y_tc = tl.verify_gemm(x, c, s, g)
-    y_simt = tl.verify_gemm_simt(x, c, s, g)
+    out = {p: gemm_on(p, x, c, s, g) for p in TC_PATHS}
+    out["simt"] = tl.verify_gemm_simt(x, c, s, g)
     torch.cuda.synchronize()
     tl.check_device_error()
-    return host_f64(y_tc), host_f64(y_simt)
+    return {k: host_f64(v) for k, v in out.items()}
+
+
+def assert_all_within_tol(ys, y_ref, a_ref, what=""):
+    for path, y in ys.items():
+        assert_within_tol(y, y_ref, a_ref, f"{what} [{path}]")
 
 
 # ------------------------------------------------------------------ format kernels
@@ -126,9 +174,7 @@ def test_tiny_config_both_paths():
     _, codes, scales, g = make_weight(256, 512, 0, 0)
     x = synth.x_bf16(8, 512, seed=0)
     y_ref, a_ref = oracle.gemm(x, codes, scales, g)
-    y_tc, y_simt = run_both_paths(x, codes, scales, g)
-    assert_within_tol(y_tc, y_ref, a_ref, "tensor-core")
-    assert_within_tol(y_simt, y_ref, a_ref, "simt")
+    assert_all_within_tol(run_paths(x, codes, scales, g), y_ref, a_ref, "tiny")
 
 
 @pytest.mark.parametrize("M", [1, 2, 7, 8, 15, 16, 17, 24, 31, 32])
@@ -137,42 +183,43 @@ def test_ragged_split_k_all_row_counts(M):
     _, codes, scales, g = make_weight(677, 2304, 2, 1)
     x = synth.x_bf16(M, 2304, seed=2, tensor_id=synth.X_ID_BASE + M)
     y_ref, a_ref = oracle.gemm(x, codes, scales, g)
-    y_tc, y_simt = run_both_paths(x, codes, scales, g)
-    assert_within_tol(y_tc, y_ref, a_ref, f"tensor-core M={M}")
-    assert_within_tol(y_simt, y_ref, a_ref, f"simt M={M}")
+    assert_all_within_tol(run_paths(x, codes, scales, g), y_ref, a_ref, f"M={M}")
 
 
+@pytest.mark.parametrize("path", list(TC_PATHS))
 @pytest.mark.parametrize("M", [1, 8, 16, 24, 32])
-def test_attention_projection_full(M):
+def test_attention_projection_full(M, path):
     _, codes, scales, g = make_weight(5120, 5120, 0, 2)
     x = synth.x_bf16(M, 5120, seed=0, tensor_id=synth.X_ID_BASE + 2)
     y_ref, a_ref = oracle.gemm(x, codes, scales, g)
-    y = host_f64(tl.verify_gemm(dev_bf16(x), dev_u8(codes), dev_u8(scales), g))
+    y = host_f64(gemm_on(path, dev_bf16(x), dev_u8(codes), dev_u8(scales), g))
     tl.check_device_error()
-    assert_within_tol(y, y_ref, a_ref, f"attn M={M}")
+    assert_within_tol(y, y_ref, a_ref, f"attn M={M} [{path}]")
 
 
-def _sampled_check(N, K, dist, Ms, tid):
+def _sampled_check(N, K, dist, Ms, tid, path):
     _, codes, scales, g = make_weight(N, K, 0, tid, dist)
     c, s = dev_u8(codes), dev_u8(scales)
     rng = np.random.default_rng(tid)
     for M in Ms:
         x = synth.x_bf16(M, K, seed=0, tensor_id=synth.X_ID_BASE + tid)
-        y = host_f64(tl.verify_gemm(dev_bf16(x), c, s, g))
+        y = host_f64(gemm_on(path, dev_bf16(x), c, s, g))
         tl.check_device_error()
         mi = rng.integers(0, M, 4096)
         ni = np.concatenate([rng.integers(0, N, 4000), np.arange(N - 96, N)])
         y_ref, a_ref = oracle.gemm_sampled(x, codes, scales, g, mi, ni)
-        assert_within_tol(y[mi, ni], y_ref, a_ref, f"{N}x{K} M={M}")
+        assert_within_tol(y[mi, ni], y_ref, a_ref, f"{N}x{K} M={M} [{path}]")
         assert np.isfinite(y).all()
 
 
-def test_mlp_gate_up_sampled():
-    _sampled_check(34816, 5120, "normal", [1, 13, 32], 10)
+@pytest.mark.parametrize("path", list(TC_PATHS))
+def test_mlp_gate_up_sampled(path):
+    _sampled_check(34816, 5120, "normal", [1, 13, 32], 10, path)
 
 
-def test_mlp_down_heavy_tail_sampled():
-    _sampled_check(5120, 17408, "t4", [1, 19, 32], 11)
+@pytest.mark.parametrize("path", list(TC_PATHS))
+def test_mlp_down_heavy_tail_sampled(path):
+    _sampled_check(5120, 17408, "t4", [1, 19, 32], 11, path)
 
 
 # ------------------------------------------------------------------ exact special cases
@@ -185,9 +232,11 @@ def test_identity_weight_returns_x_exactly():
     scales = np.full((K, K // 16), 0x38, dtype=np.uint8)
     for M in (3, 32):
         x = synth.x_bf16(M, K, seed=5, tensor_id=M)
-        y_tc, y_simt = run_both_paths(x, codes, scales, 1.0)
+        ys = run_paths(x, codes, scales, 1.0)
         xf = synth.bf16_bits_to_f32(x).astype(np.float64)
-        assert np.array_equal(y_tc, xf) and np.array_equal(y_simt, xf)
+        assert np.array_equal(ys["bf16-exact"], xf) and np.array_equal(ys["simt"], xf)
+        bound = 1e-3 * np.abs(xf) + 2.0 ** -8 * np.abs(xf) + split_bound(x, codes, scales, 1.0)
+        assert_within_bound(ys["block-scaled"], xf, bound, "identity [block-scaled]")
 
 
 def test_one_hot_weight_exact():
@@ -200,10 +249,12 @@ def test_one_hot_weight_exact():
         codes[n, k // 2] |= (0xD if k % 2 == 0 else 0xD0)   # -3.0
     scales = np.full((N, K // 16), 0x30, dtype=np.uint8)    # 0.5
     x = synth.x_bf16(20, K, seed=6)
-    y_ref, _ = oracle.gemm(x, codes, scales, 0.25)
-    y_tc, y_simt = run_both_paths(x, codes, scales, 0.25)
+    y_ref, a_ref = oracle.gemm(x, codes, scales, 0.25)
+    ys = run_paths(x, codes, scales, 0.25)
     want = bf16_round(y_ref)
-    assert np.array_equal(y_tc, want) and np.array_equal(y_simt, want)
+    assert np.array_equal(ys["bf16-exact"], want) and np.array_equal(ys["simt"], want)
+    bound = 1e-3 * a_ref + 2.0 ** -8 * np.abs(y_ref) + split_bound(x, codes, scales, 0.25)
+    assert_within_bound(ys["block-scaled"], y_ref, bound, "one-hot [block-scaled]")
 
 
 def test_small_integer_exact():
@@ -213,10 +264,11 @@ def test_small_integer_exact():
     codes = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
     scales = np.full((N, K // 16), 0x38, dtype=np.uint8)
     g = 2.0 ** -3
-    y_ref, _ = oracle.gemm(x, codes, scales, g)
-    y_tc, y_simt = run_both_paths(x, codes, scales, g)
+    y_ref, a_ref = oracle.gemm(x, codes, scales, g)
+    ys = run_paths(x, codes, scales, g)
     want = bf16_round(y_ref)
-    assert np.array_equal(y_tc, want) and np.array_equal(y_simt, want)
+    assert np.array_equal(ys["bf16-exact"], want) and np.array_equal(ys["simt"], want)
+    assert_within_tol(ys["block-scaled"], y_ref, a_ref, "small integers [block-scaled]")
 
 
 def test_subnormal_scales_and_zero_blocks():
@@ -228,20 +280,90 @@ def test_subnormal_scales_and_zero_blocks():
     scales[:, ::7] = rng.integers(0, 8, scales[:, ::7].shape)
     x = synth.x_bf16(M, K, seed=12)
     y_ref, a_ref = oracle.gemm(x, codes, scales, 0.5)
-    y_tc, y_simt = run_both_paths(x, codes, scales, 0.5)
-    assert_within_tol(y_tc, y_ref, a_ref, "tensor-core")
-    assert_within_tol(y_simt, y_ref, a_ref, "simt")
+    assert_all_within_tol(run_paths(x, codes, scales, 0.5), y_ref, a_ref, "subnormal scales")
+
+
+def test_negative_scales():
+    # E4M3 scale bytes with the sign bit set (0x80..0xFE): the block's weights change sign
+    rng = np.random.default_rng(13)
+    M, N, K = 17, 384, 1536
+    codes = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    scales = rng.integers(0x28, 0x48, (N, K // 16), dtype=np.uint8)
+    neg = rng.random((N, K // 16)) < 0.4
+    scales[neg] |= 0x80
+    scales[5, :] |= 0x80                   # a whole row of negative scales
+    scales[7, 3] = 0x80                    # -0
+    x = synth.x_bf16(M, K, seed=13)
+    y_ref, a_ref = oracle.gemm(x, codes, scales, 0.125)
+    assert_all_within_tol(run_paths(x, codes, scales, 0.125), y_ref, a_ref, "negative scales")
+
+
+def test_nan_scale_gives_nan_column():
+    # a NaN scale (0x7F or 0xFF) makes every output of that weight row NaN, as in the reference
+    rng = np.random.default_rng(14)
+    M, N, K = 8, 256, 1024
+    codes = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    scales = rng.integers(0x30, 0x40, (N, K // 16), dtype=np.uint8)
+    scales[3, 10] = 0x7F
+    scales[200, 63] = 0xFF
+    codes[200, 63 * 8:64 * 8] = 0          # NaN times zero codes is still NaN
+    x = synth.x_bf16(M, K, seed=14)
+    y_ref, a_ref = oracle.gemm(x, codes, scales, 1.0)
+    assert np.isnan(y_ref[:, [3, 200]]).all() and np.isfinite(np.delete(y_ref, [3, 200], axis=1)).all()
+    assert_all_within_tol(run_paths(x, codes, scales, 1.0), y_ref, a_ref, "NaN scale")
+
+
+def test_nonfinite_x_row():
+    # a NaN in X makes that row NaN on every path; the other rows are unaffected
+    _, codes, scales, g = make_weight(256, 512, 15, 15)
+    x = synth.x_bf16(5, 512, seed=15)
+    x[2, 100] = 0x7FC0                     # bf16 NaN
+    y_ref, a_ref = oracle.gemm(x, codes, scales, g)
+    assert np.isnan(y_ref[2]).all()
+    assert_all_within_tol(run_paths(x, codes, scales, g), y_ref, a_ref, "NaN in X")
+
+
+@pytest.mark.parametrize("ratio", [1e2, 1e4, 1e6])
+def test_outlier_channels_in_x(ratio):
+    # a few channels far larger than the rest (large activation outliers), and rows at the
+    # extremes of the bf16 range
+    _, codes, scales, g = make_weight(640, 4096, 16, 16)
+    rng = np.random.default_rng(16)
+    xf = synth.bf16_bits_to_f32(synth.x_bf16(12, 4096, seed=16)).astype(np.float64)
+    cols = rng.choice(4096, 6, replace=False)
+    xf[:, cols] *= ratio
+    xf[10] *= 2.0 ** -100
+    xf[11] *= 2.0 ** 100
+    x = synth.f32_to_bf16_bits(xf.astype(np.float32))
+    y_ref, a_ref = oracle.gemm(x, codes, scales, g)
+    assert_all_within_tol(run_paths(x, codes, scales, g), y_ref, a_ref, f"outliers x{ratio:g}")
 
 
 # ------------------------------------------------------------------ determinism, stack, host path
 
-def test_repeat_runs_bit_identical():
+@pytest.mark.parametrize("path", list(TC_PATHS))
+def test_repeat_runs_bit_identical(path):
     _, codes, scales, g = make_weight(677, 2304, 2, 1)
     x = dev_bf16(synth.x_bf16(32, 2304, seed=4))
     c, s = dev_u8(codes), dev_u8(scales)
-    first = tl.verify_gemm(x, c, s, g).clone()
+    first = gemm_on(path, x, c, s, g).clone()
     for _ in range(5):
-        assert torch.equal(tl.verify_gemm(x, c, s, g), first)
+        assert torch.equal(gemm_on(path, x, c, s, g), first)
+    tl.check_device_error()
+
+
+@pytest.mark.parametrize("path", list(TC_PATHS))
+def test_rows_do_not_depend_on_M(path):
+    # row i of a call with M rows equals the same row computed alone, bit for bit
+    _, codes, scales, g = make_weight(677, 2304, 2, 1)
+    x = synth.x_bf16(32, 2304, seed=17)
+    c, s = dev_u8(codes), dev_u8(scales)
+    alone = [gemm_on(path, dev_bf16(x[i:i + 1]), c, s, g) for i in (0, 5, 15, 16, 31)]
+    for M in (16, 17, 32):
+        y = gemm_on(path, dev_bf16(x[:M]), c, s, g)
+        for j, i in enumerate((0, 5, 15, 16, 31)):
+            if i < M:
+                assert torch.equal(y[i:i + 1], alone[j]), (M, i)
     tl.check_device_error()
 
 
@@ -260,23 +382,51 @@ def _small_stack(M, n_layers=3):
     return ents, refs
 
 
+@pytest.mark.parametrize("path", list(TC_PATHS))
 @pytest.mark.parametrize("M", [8, 24])
-def test_stack_matches_oracle_and_single_calls(M):
+def test_stack_matches_oracle_and_single_calls(M, path):
     ents, refs = _small_stack(M)
     mats = tl.make_matrices(ents)
-    tl.verify_stack(mats, M)
+    with tl.gemm_path(TC_PATHS[path]):
+        tl.verify_stack(mats, M)
     torch.cuda.synchronize()
     tl.check_device_error()
     for (c, s, g, x, y), (y_ref, a_ref, _) in zip(ents, refs):
         assert_within_tol(host_f64(y), y_ref, a_ref, "stack")
     # the cached descriptor table is reused on the second call: same results
     ys = [e[4].clone() for e in ents]
-    tl.verify_stack(mats, M)
+    with tl.gemm_path(TC_PATHS[path]):
+        tl.verify_stack(mats, M)
     for e, y0 in zip(ents, ys):
         assert torch.equal(e[4], y0)
+    # a single call gives the same rows as the stack
+    c, s, g, x, y = ents[5]
+    assert torch.equal(gemm_on(path, x, c, s, g), y)
 
 
-def test_stack_host_buffers_end_to_end():
+@pytest.mark.parametrize("path", list(TC_PATHS))
+def test_plan_matches_stack(path):
+    M = 24
+    ents, refs = _small_stack(M, n_layers=2)
+    mats = tl.make_matrices(ents)
+    with tl.gemm_path(TC_PATHS[path]):
+        tl.verify_stack(mats, M)
+        ys = [e[4].clone() for e in ents]
+        plan = tl.Plan(ents, M)
+    for e in ents:
+        e[4].fill_(0)
+    with tl.gemm_path(TC_PATHS[path] ^ 1):   # a plan keeps the path it was made with
+        plan.run()
+        plan.run()
+    torch.cuda.synchronize()
+    tl.check_device_error()
+    for e, y0 in zip(ents, ys):
+        assert torch.equal(e[4], y0)
+    plan.close()
+
+
+@pytest.mark.parametrize("path", list(TC_PATHS))
+def test_stack_host_buffers_end_to_end(path):
     M = 16
     ents, refs = _small_stack(M, n_layers=2)
     xs = torch.cat([e[3].reshape(-1) for e in ents]).cpu().pin_memory()
@@ -285,7 +435,8 @@ def test_stack_host_buffers_end_to_end():
     y_dev = torch.empty(ytot, dtype=torch.bfloat16, device=DEV)
     y_host = torch.empty(ytot, dtype=torch.bfloat16).pin_memory()
     mats = tl.make_matrices([(c, s, g, None, None) for c, s, g, _, _ in ents])
-    tl.verify_stack_host(mats, M, xs, x_dev, y_host, y_dev)
+    with tl.gemm_path(TC_PATHS[path]):
+        tl.verify_stack_host(mats, M, xs, x_dev, y_host, y_dev)
     torch.cuda.synchronize()
     tl.check_device_error()
     off = 0
@@ -309,8 +460,7 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     _, codes, scales, g = make_weight(256, 512, 0, 0)
     x = synth.x_bf16(8, 512, seed=0)
     y_ref, a_ref = oracle.gemm(x, codes, scales, g)
-    y_tc, _ = run_both_paths(x, codes, scales, g)
-    assert_within_tol(y_tc, y_ref, a_ref, "after timeout")
+    assert_all_within_tol(run_paths(x, codes, scales, g), y_ref, a_ref, "after timeout")
 
 
 def test_zero_rows_is_a_no_op():
