@@ -5,26 +5,31 @@
 // tcgen05.mma.kind::mxf4nvf4.block_scale consumes: the weight tile goes from HBM (TMA) into
 // shared memory and from there straight into the tensor core, with no decode on the CUDA
 // cores. X is brought into the same form beforehand (xsplit.cuh): per row a power of two and
-// TC_PIECES FP4 pieces with E4M3 scales. The pieces are stacked along the MMA's N dimension,
-// so one MMA per 64-k chunk serves every X row and every piece:
+// TC_PIECES FP4 pieces with E4M3 scales. The rows' pieces are stacked along the MMA's N
+// dimension (row m's pieces adjacent; Mp = M rounded up to a multiple of 4, padding rows
+// zero), so one MMA per 64-k chunk serves every X row and every piece:
 //
-//   D[n][p * NX + m] = sum_k  w[n][k] * piece_p[m][k]        (fp32, in tensor memory)
-//   Y[m][n]          = bf16( (sum_p 4^-p D[n][p * NX + m]) * g * factor[m] )
+//   D[n][4 m + p] = sum_k  w[n][k] * piece_p[m][k]        (fp32, in tensor memory; N = 4 Mp)
+//   Y[m][n]       = bf16( (sum_p 4^-p D[n][4 m + p]) * g * factor[m] )
 //
 //   * Work. As in gemm_tc.cuh: 128 weight rows x 256 k per tile, one global tile list cut into
 //     equal contiguous shares (stream-K); a split n-tile is reduced by its last contributor in
 //     k order, so every output has one fixed reduction order.
 //   * Roles, 12 warps.
-//     - Warp 0: TMA of W codes, W scales, X piece codes and X piece scales into a ring of
-//       stages (one 3-D copy each, from four lanes at once).
+//     - Warp 0: copies into a ring of stages, four per tile from four lanes at once. Lanes 0
+//       and 1: a TMA tensor copy each of the tile's W codes and W scales. Lanes 2 and 3: one
+//       plain bulk copy each of the tile's X piece codes (4 Mp rows of 128 B) and X piece
+//       scales (4 Mp rows of 16 B), contiguous in the k-tile-major layout xsplit.cuh writes.
+//       Few, large copies: the copy engine's cost per request, not the bytes, is what a
+//       per-row layout ran into.
 //     - Warps 4..7: copy the tile's scales into tensor memory in the layout the MMA reads:
 //       lane 32q + l, columns 4c .. 4c+3 hold the scale words (four 16-k blocks each) of rows
 //       l, l + 32, l + 64, l + 96 for 64-k chunk c, for W and for the stacked X pieces.
 //       A W scale byte with the sign bit set (the MMA's scales are unsigned) is handled
 //       exactly: the codes of that block are negated in shared memory and the scale's sign is
 //       cleared.
-//     - Warp 1: one elected lane issues the four MMAs of a tile (M = 128, N = TC_PIECES * NX,
-//       K = 64 each) into the segment's accumulator.
+//     - Warp 1: one elected lane issues the four MMAs of a tile (M = 128, N = 4 Mp, K = 64
+//       each) into the segment's accumulator.
 //     - Warps 8..11: the epilogue sums the pieces in fixed order and writes Y (or a partial).
 //
 // Every mbarrier wait is bounded; a wait that runs out records a status code and the CTA
@@ -45,8 +50,8 @@ constexpr int BS_SF_COLS = 32;    // tensor-memory columns of scales per stage (
 struct alignas(64) BsMat {
     CUtensorMap tm_codes;   // uint8 {K/2, N, 1}, box 128 B x 128 rows x 1, 128-byte swizzle
     CUtensorMap tm_scales;  // uint8 {K/16, N, 1}, box 16 B x 128 rows x 1
-    CUtensorMap tm_xc;      // uint8 {K/2, M, TC_PIECES}, box 128 B x NX rows x TC_PIECES, 128-byte swizzle
-    CUtensorMap tm_xs;      // uint8 {K/16, M, TC_PIECES}, box 16 B x NX rows x TC_PIECES
+    const uint8_t* xc;      // X piece codes, [K/256][TC_PIECES][M][128] (swizzled rows, xsplit.cuh)
+    const uint8_t* xs;      // X piece scales, [K/256][TC_PIECES][M][16]
     const float* xfactor;   // [M], 2^-e per X row (NaN for a non-finite row)
     __nv_bfloat16* y;
     float g;                // the weight's tensor scale
@@ -60,6 +65,7 @@ struct BsParams {
     const BsMat* mats;      // device table, or nullptr to use `one`
     int n_mats;
     int M;
+    int Mp;                 // M rounded up to a multiple of 4: X rows per piece group in the layout
     long long total_tiles;
     float* partials;        // [2 * gridDim.x][32][128] fp32
     unsigned* counters;     // [4 * gridDim.x], zero between launches
@@ -73,18 +79,19 @@ struct BsCfg {
     static constexpr int XC_BYTES = TC_PIECES * NX * (TC_BLOCK_K / 2);       // 8192 / 16384
     static constexpr int SCALES_BYTES = TC_BLOCK_N * (TC_BLOCK_K / 16);      // 2048
     static constexpr int XS_BYTES = TC_PIECES * NX * (TC_BLOCK_K / 16);      // 1024 / 2048
-    static constexpr int XC_OFF = CODES_BYTES;
-    static constexpr int SC_OFF = XC_OFF + XC_BYTES;
-    static constexpr int XS_OFF = SC_OFF + SCALES_BYTES;
+    static constexpr int SC_OFF = CODES_BYTES;
+    static constexpr int XC_OFF = SC_OFF + SCALES_BYTES;                     // 18432: 1024-byte aligned
+    static constexpr int XS_OFF = XC_OFF + XC_BYTES;                         // X codes and scales adjoin
     static constexpr int STAGE_BYTES = XS_OFF + XS_BYTES;                    // 27648 / 36864
     static constexpr int STAGES = (NX == 32) ? 6 : 8;
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 512 /*barriers*/;
-    static constexpr int N_MMA = TC_PIECES * NX;                             // 64 / 128
+    static constexpr int N_MMA = TC_PIECES * NX;                             // largest N: 64 / 128
     static constexpr int ACC_BUFS = 2;
     static constexpr int SF_COL0 = 256;
-    static constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | ((uint32_t)(N_MMA >> 3) << 17) | (0u << 23) |
-                                      ((uint32_t)(TC_BLOCK_N >> 4) << 24);   // E2M1 x E2M1, UE4M3 scales
+    // E2M1 x E2M1, UE4M3 scales, M = 128; N (bits 17..22, N / 8) is added at run time
+    static constexpr uint32_t IDESC_BASE = (1u << 7) | (1u << 10) | (0u << 23) | ((uint32_t)(TC_BLOCK_N >> 4) << 24);
     static_assert(STAGE_BYTES % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
+    static_assert(XC_OFF % 1024 == 0, "X piece codes must start on a swizzle atom");
     static_assert(ACC_BUFS * N_MMA <= SF_COL0, "accumulators must fit below the scale columns");
     static_assert(SF_COL0 + STAGES * BS_SF_COLS <= TC_TMEM_COLS, "tensor memory budget");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -162,6 +169,12 @@ gemm_bs_kernel(const __grid_constant__ BsParams p) {
         tmem_alloc(tmem_slot, TC_TMEM_COLS);
         tmem_relinquish();
     }
+    // X rows past 4 Mp stay zero: the copies only ever write rows < 4 Mp
+    for (int i = threadIdx.x; i < C::STAGES * (C::XC_BYTES + C::XS_BYTES) / 16; i += BS_THREADS) {
+        const int st = i / ((C::XC_BYTES + C::XS_BYTES) / 16), o = 16 * (i % ((C::XC_BYTES + C::XS_BYTES) / 16));
+        *reinterpret_cast<uint4*>(smem + st * C::STAGE_BYTES + C::XC_OFF + o) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -172,8 +185,11 @@ gemm_bs_kernel(const __grid_constant__ BsParams p) {
         // Lanes 0..3 copy W codes, W scales, X piece codes and X piece scales of a stage with one
         // converged rank-3 load; the whole warp waits for the stage.
         const uint64_t pol = (lane < 2) ? policy_evict_first() : policy_evict_last();
+        // lane 2: X piece codes (4 Mp rows x 128 B), lane 3: X piece scales (4 Mp rows x 16 B)
+        const uint32_t xbytes = (uint32_t)(TC_PIECES * p.Mp) * ((lane == 2) ? 128u : 16u);
         const uint32_t dst_off = (lane == 0) ? 0u : (lane == 1) ? (uint32_t)C::SC_OFF
                                : (lane == 2) ? (uint32_t)C::XC_OFF : (uint32_t)C::XS_OFF;
+        const uint32_t stage_tx = (uint32_t)(C::CODES_BYTES + C::SCALES_BYTES) + (uint32_t)p.Mp * (TC_PIECES * (128 + 16));
         const uint32_t smem0 = smem_u32(smem);
         int s = 0;
         uint32_t ph = 0, issued = 0, last_ph = 0;
@@ -197,9 +213,9 @@ gemm_bs_kernel(const __grid_constant__ BsParams p) {
             const int k0 = (int)(local % m.k_tiles);
             const long long rem = t_end - t;
             const int k1 = (int)((m.k_tiles - k0) < rem ? m.k_tiles : k0 + rem);
-            const void* tmap = (lane == 0) ? (const void*)&m.tm_codes : (lane == 1) ? (const void*)&m.tm_scales
-                             : (lane == 2) ? (const void*)&m.tm_xc : (const void*)&m.tm_xs;
-            const int c1 = (lane < 2) ? ntile * TC_BLOCK_N : 0;
+            const void* tmap = (lane == 0) ? (const void*)&m.tm_codes : (const void*)&m.tm_scales;
+            const int c1 = ntile * TC_BLOCK_N;
+            const uint8_t* xsrc = (lane == 2) ? m.xc : m.xs;    // k-tile 0; k-tile kt is xbytes further each
             for (int kt = k0; kt < k1; ++kt) {
                 const bool got = tc_wait(&empty[s], ph ^ 1u, abort_flag);
                 if (!__all_sync(0xFFFFFFFFu, got)) {
@@ -207,11 +223,14 @@ gemm_bs_kernel(const __grid_constant__ BsParams p) {
                     ok = false;
                     break;
                 }
-                if (lane == 0) mbar_arrive_expect_tx(&full[s], (uint32_t)C::STAGE_BYTES);
+                if (lane == 0) mbar_arrive_expect_tx(&full[s], stage_tx);
                 __syncwarp();
-                const int c0 = (lane == 0 || lane == 2) ? kt * (TC_BLOCK_K / 2) : kt * (TC_BLOCK_K / 16);
-                if (lane < 4)
-                    tma_load_3d_s(smem0 + (uint32_t)(s * C::STAGE_BYTES) + dst_off, tmap, &full[s], c0, c1, 0, pol);
+                const uint32_t dst = smem0 + (uint32_t)(s * C::STAGE_BYTES) + dst_off;
+                if (lane < 2)
+                    tma_load_3d_s(dst, tmap, &full[s], (lane == 0) ? kt * (TC_BLOCK_K / 2) : kt * (TC_BLOCK_K / 16),
+                                  c1, 0, pol);
+                else if (lane < 4)
+                    bulk_load_s(dst, xsrc + (size_t)kt * xbytes, xbytes, &full[s], pol);
                 issued |= 1u << s;
                 last_ph = (last_ph & ~(1u << s)) | (ph << s);
                 if (++s == C::STAGES) { s = 0; ph ^= 1u; }
@@ -231,6 +250,7 @@ gemm_bs_kernel(const __grid_constant__ BsParams p) {
         uint32_t ph = 0, accph = 0;
         const uint64_t desc_w0 = smem_desc_k_sw128(smem_u32(smem));
         const uint64_t desc_x0 = smem_desc_k_sw128(smem_u32(smem + C::XC_OFF));
+        const uint32_t idesc = C::IDESC_BASE | ((uint32_t)(TC_PIECES * p.Mp) >> 3) << 17;
         long long t = t_begin;
         int mi = 0;
         {
@@ -270,7 +290,7 @@ gemm_bs_kernel(const __grid_constant__ BsParams p) {
 #pragma unroll
                     for (int kc = 0; kc < 4; ++kc)
                         mma_bs_f4(d_tmem, desc_w0 + sdesc + (uint64_t)(2 * kc), desc_x0 + sdesc + (uint64_t)(2 * kc),
-                                  C::IDESC, sf + 4u * kc, sf + 16u + 4u * kc, (kc == 0) ? (first ^ 1u) : 1u);
+                                  idesc, sf + 4u * kc, sf + 16u + 4u * kc, (kc == 0) ? (first ^ 1u) : 1u);
                     mma_commit(&empty[s]);
                 }
                 __syncwarp();
@@ -395,20 +415,25 @@ gemm_bs_kernel(const __grid_constant__ BsParams p) {
             const long long ta = m.tile_begin + (long long)ntile * m.k_tiles;
             const int my_slot = 2 * (int)blockIdx.x + (seg_t0 == t_begin ? 0 : 1);
             float* mine = p.partials + (size_t)my_slot * (32 * TC_BLOCK_N);
-            // sum the pieces in order: v[mm] = sum_p 4^-p D[p * NX + mm] (exact scalings)
+            // sum the pieces in order: v[m] = sum_p 4^-p D[4 m + p] (exact scalings); 16 columns
+            // hold rows 4c .. 4c+3
             float v[NX];
 #pragma unroll
-            for (int i = 0; i < NX; ++i) v[i] = 0.0f;
-#pragma unroll
-            for (int pc = 0; pc < TC_PIECES; ++pc) {
-#pragma unroll
-                for (int c0 = 0; c0 < NX; c0 += 16) {
+            for (int c = 0; c < NX / 4; ++c) {
+                if (4 * c < M) {
                     uint32_t raw[16];
-                    tmem_ld16(t_lane + (uint32_t)(C::N_MMA * acc + pc * NX + c0), raw);
+                    tmem_ld16(t_lane + (uint32_t)(C::N_MMA * acc + 16 * c), raw);
                     tmem_wait_ld();
-                    const float unit = 1.0f / (float)(1 << (2 * pc));
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) v[c0 + i] = fmaf(__uint_as_float(raw[i]), unit, v[c0 + i]);
+                    for (int j = 0; j < 4; ++j) {
+                        float a = __uint_as_float(raw[4 * j]);
+                        a = fmaf(__uint_as_float(raw[4 * j + 1]), 0.25f, a);
+                        a = fmaf(__uint_as_float(raw[4 * j + 2]), 0.0625f, a);
+                        v[4 * c + j] = fmaf(__uint_as_float(raw[4 * j + 3]), 0.015625f, a);
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) v[4 * c + j] = 0.0f;
                 }
             }
             tc_fence_before();

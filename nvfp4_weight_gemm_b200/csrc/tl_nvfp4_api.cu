@@ -347,9 +347,13 @@ tl_status run_stack(const tl_nvfp4_matrix* mats, int n_mats, int M, const unsign
 
 size_t round256(size_t v) { return (v + 255) & ~size_t(255); }
 
-// Bytes of the X pieces (codes, scales, row factors) of one matrix with M rows and K columns.
+int round4(int M) { return (M + 3) & ~3; }
+
+// Bytes of the X pieces (codes, scales, row factors) of one matrix with M rows and K columns;
+// the pieces are laid out for Mp = M rounded up to a multiple of 4 rows.
 size_t xs_bytes_of(int M, int K) {
-    return round256((size_t)tl::TC_PIECES * M * (K / 2)) + round256((size_t)tl::TC_PIECES * M * (K / 16)) +
+    const size_t Mp = (size_t)round4(M);
+    return round256((size_t)tl::TC_PIECES * Mp * (K / 2)) + round256((size_t)tl::TC_PIECES * Mp * (K / 16)) +
            round256((size_t)4 * M);
 }
 
@@ -363,24 +367,19 @@ size_t xs_bytes_total(const tl_nvfp4_matrix* mats, int n_mats, int M) {
 tl_status build_bs_mat(tl::BsMat* m, tl::XSplitMat* xm, const void* x, int M, int NX, const void* codes,
                        const void* scales, float g, void* y, int N, int K, long long tile_begin, unsigned char* xs) {
     memset(m, 0, sizeof *m);
-    const cuuint64_t n = (cuuint64_t)N, k = (cuuint64_t)K, mm = (cuuint64_t)M, P = (cuuint64_t)tl::TC_PIECES;
+    const cuuint64_t n = (cuuint64_t)N, k = (cuuint64_t)K, P = (cuuint64_t)tl::TC_PIECES, Mp = (cuuint64_t)round4(M);
     unsigned char* xc = xs;
-    unsigned char* xsc = xc + round256((size_t)P * M * (K / 2));
-    float* xf = reinterpret_cast<float*>(xsc + round256((size_t)P * M * (K / 16)));
+    unsigned char* xsc = xc + round256((size_t)P * Mp * (K / 2));
+    float* xf = reinterpret_cast<float*>(xsc + round256((size_t)P * Mp * (K / 16)));
     tl_status st = encode_3d(&m->tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, {k / 2, n, 1}, {k / 2, n * (k / 2)},
                              {tl::TC_BLOCK_K / 2, tl::TC_BLOCK_N, 1}, CU_TENSOR_MAP_SWIZZLE_128B, "codes");
     if (st != TL_OK) return st;
     st = encode_3d(&m->tm_scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, scales, {k / 16, n, 1}, {k / 16, n * (k / 16)},
                    {tl::TC_BLOCK_K / 16, tl::TC_BLOCK_N, 1}, CU_TENSOR_MAP_SWIZZLE_NONE, "scales");
     if (st != TL_OK) return st;
-    // X pieces: {K/2 bytes, M rows, pieces}; a box {128, NX, pieces} stacks the pieces of a tile
-    // as the MMA's N = pieces x NX rows (rows >= M read zero)
-    st = encode_3d(&m->tm_xc, CU_TENSOR_MAP_DATA_TYPE_UINT8, xc, {k / 2, mm, P}, {k / 2, mm * (k / 2)},
-                   {tl::TC_BLOCK_K / 2, (cuuint32_t)NX, (cuuint32_t)P}, CU_TENSOR_MAP_SWIZZLE_128B, "X piece codes");
-    if (st != TL_OK) return st;
-    st = encode_3d(&m->tm_xs, CU_TENSOR_MAP_DATA_TYPE_UINT8, xsc, {k / 16, mm, P}, {k / 16, mm * (k / 16)},
-                   {tl::TC_BLOCK_K / 16, (cuuint32_t)NX, (cuuint32_t)P}, CU_TENSOR_MAP_SWIZZLE_NONE, "X piece scales");
-    if (st != TL_OK) return st;
+    // X pieces: k-tile-major runs that the kernel fetches with plain bulk copies
+    m->xc = xc;
+    m->xs = xsc;
     m->xfactor = xf;
     m->y = static_cast<__nv_bfloat16*>(y);
     m->g = g;
@@ -427,12 +426,14 @@ tl_status build_bs(const tl_nvfp4_matrix* mats, int n_mats, int M, const unsigne
     memset(&L->bp, 0, sizeof L->bp);
     L->bp.n_mats = n_mats;
     L->bp.M = M;
+    L->bp.Mp = round4(M);
     L->bp.total_tiles = tiles;
     L->bp.mats = nullptr;
     if (n_mats == 1) L->bp.one = L->tbl[0];
     memset(&L->xp, 0, sizeof L->xp);
     L->xp.n_mats = n_mats;
     L->xp.M = M;
+    L->xp.Mp = round4(M);
     L->xp.mats = nullptr;
     if (n_mats == 1) L->xp.one = L->xtbl[0];
     return TL_OK;
@@ -453,7 +454,7 @@ tl_status launch_bs_gemm(DevState& d, tl::BsParams& p, cudaStream_t stream) {
 
 // The X split, then the GEMM, on `stream`.
 tl_status launch_bs(DevState& d, tl::BsParams bp, const tl::XSplitParams& xp, cudaStream_t stream) {
-    tl::x_split_kernel<<<dim3((unsigned)xp.M, (unsigned)xp.n_mats), tl::XS_THREADS, 0, stream>>>(xp);
+    tl::x_split_kernel<<<dim3((unsigned)xp.Mp, (unsigned)xp.n_mats), tl::XS_THREADS, 0, stream>>>(xp);
     TL_CUDA(cudaGetLastError());
     return (bp.M <= 16) ? launch_bs_gemm<16>(d, bp, stream) : launch_bs_gemm<32>(d, bp, stream);
 }

@@ -23,9 +23,15 @@
 // magnitude inside |y - y_ref| <= 1e-3 * sum|x w| + 2^-8 |y_ref|. A row whose largest |x| is
 // not finite gets a NaN factor, so its outputs are NaN.
 //
-// Layout written per matrix (all row-major, k pairs packed low nibble first like the weights):
-//   codes  [TC_PIECES][M][K/2]   bytes
-//   scales [TC_PIECES][M][K/16]  bytes
+// Layout written per matrix, k-tile major (a k-tile is 256 k), so that one k-tile of every
+// row and piece is one contiguous run that a single bulk copy brings into shared memory.
+// Mp is M rounded up to a multiple of 4; rows M .. Mp-1 are written as zeros. Row m's pieces
+// are adjacent: piece p of row m is "line" j = 4 m + p of the k-tile.
+//   codes  [K/256][Mp][TC_PIECES][128]  bytes: the line's 256 k of the tile, k pairs packed
+//                                       low nibble first like the weights; the 16-byte chunk
+//                                       c of line j is stored at chunk c ^ (j & 7), the 128-byte
+//                                       swizzle the tensor core's shared-memory descriptor reads
+//   scales [K/256][Mp][TC_PIECES][16]   bytes: the E4M3 scales of the tile's 16 blocks
 //   factor [M]                   float, 2^-e[m] (NaN for a non-finite row); piece p of row m
 //                                stands for factor[m] * 4^-p * (its codes times its scales)
 #pragma once
@@ -40,8 +46,8 @@ constexpr int TC_PIECES = 4;
 
 struct XSplitMat {
     const __nv_bfloat16* x;   // [M][K]
-    uint8_t* codes;           // [TC_PIECES][M][K/2]
-    uint8_t* scales;          // [TC_PIECES][M][K/16]
+    uint8_t* codes;           // [K/256][TC_PIECES][M][128], swizzled rows
+    uint8_t* scales;          // [K/256][TC_PIECES][M][16]
     float* factor;            // [M]
     int K;
 };
@@ -50,6 +56,7 @@ struct XSplitParams {
     const XSplitMat* mats;    // device table, or nullptr to use `one`
     int n_mats;
     int M;
+    int Mp;                   // M rounded up to a multiple of 4
     XSplitMat one;
 };
 
@@ -122,15 +129,16 @@ __device__ __forceinline__ float2 xs_e2m1x2_values(uint32_t byte) {
 
 constexpr int XS_THREADS = 128;
 
-// Grid (M, n_mats): one CTA per row of one matrix.
+// Grid (Mp, n_mats): one CTA per row of one matrix; rows M .. Mp-1 write zero pieces.
 __global__ void __launch_bounds__(XS_THREADS) x_split_kernel(const __grid_constant__ XSplitParams p) {
     __shared__ float red[XS_THREADS / 32];
     __shared__ int bad_sh;
     const XSplitMat& m = p.mats ? p.mats[blockIdx.y] : p.one;
     const int row = blockIdx.x;
     const int K = m.K;
-    const int M = p.M;
-    const __nv_bfloat16* x = m.x + (size_t)row * K;
+    const int M = p.M, Mp = p.Mp;
+    const bool pad_row = row >= M;
+    const __nv_bfloat16* x = m.x + (size_t)(pad_row ? 0 : row) * K;
     uint8_t* const codes = m.codes;
     uint8_t* const scales = m.scales;
     float* const factor = m.factor;
@@ -138,7 +146,7 @@ __global__ void __launch_bounds__(XS_THREADS) x_split_kernel(const __grid_consta
     if (threadIdx.x == 0) bad_sh = 0;
     float mx = 0.0f;
     bool bad = false;
-    for (int k8 = threadIdx.x; k8 < K / 8; k8 += XS_THREADS) {
+    for (int k8 = threadIdx.x; !pad_row && k8 < K / 8; k8 += XS_THREADS) {
         const uint4 v = __ldg(reinterpret_cast<const uint4*>(x) + k8);
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -157,26 +165,29 @@ __global__ void __launch_bounds__(XS_THREADS) x_split_kernel(const __grid_consta
 #pragma unroll
     for (int i = 1; i < XS_THREADS / 32; ++i) r = fmaxf(r, red[i]);
     __syncthreads();
-    const bool bad_row = bad_sh != 0;
+    const bool bad_row = bad_sh != 0 || pad_row;   // both write zero pieces
     int e = 0;                                  // r * 2^e in [2^7, 2^8)
     if (r > 0.0f && !bad_row) {
         int fe;
         frexpf(r, &fe);                         // r in [2^(fe-1), 2^fe)
         e = 8 - fe;
     }
-    if (threadIdx.x == 0) factor[row] = bad_row ? __int_as_float(0x7FC00000) : ldexpf(1.0f, -e);
+    if (threadIdx.x == 0 && !pad_row) factor[row] = bad_row ? __int_as_float(0x7FC00000) : ldexpf(1.0f, -e);
     // exact scaling by 2^e in two steps (each factor a normal power of two)
     const float p1 = ldexpf(1.0f, e / 2), p2 = ldexpf(1.0f, e - e / 2);
     // 2. four pieces per 16-k block, one thread per block
-    const size_t plane_c = (size_t)M * (K / 2), plane_s = (size_t)M * (K / 16);
-    uint8_t* crow = codes + (size_t)row * (K / 2);
-    uint8_t* srow = scales + (size_t)row * (K / 16);
     for (int b = threadIdx.x; b < K / 16; b += XS_THREADS) {
+        const int kt = b >> 4, bt = b & 15;       // k-tile, block within it
+        const size_t j0 = ((size_t)kt * Mp + (size_t)row) * TC_PIECES;   // line of piece 0
+        // piece p is line j0 + p; its 16-byte chunk bt/2 sits at chunk (bt/2) ^ ((j0 + p) & 7)
+        uint8_t* cline = codes + j0 * 128 + 8 * (bt & 1);
+        uint8_t* sdst = scales + j0 * 16 + bt;
+        const uint32_t chunk = (uint32_t)(bt >> 1), ph0 = (uint32_t)(j0 & 7);
         if (bad_row) {
 #pragma unroll
             for (int pc = 0; pc < TC_PIECES; ++pc) {
-                *reinterpret_cast<uint2*>(crow + pc * plane_c + 8 * b) = make_uint2(0u, 0u);
-                srow[pc * plane_s + b] = 0;
+                *reinterpret_cast<uint2*>(cline + pc * 128 + ((chunk ^ ((ph0 + pc) & 7u)) << 4)) = make_uint2(0u, 0u);
+                sdst[pc * 16] = 0;
             }
             continue;
         }
@@ -208,8 +219,8 @@ __global__ void __launch_bounds__(XS_THREADS) x_split_kernel(const __grid_consta
                 u[2 * j + 1] = 4.0f * fmaf(-q.y, s, u[2 * j + 1]);
                 if (j < 4) wlo |= byte << (8 * j); else whi |= byte << (8 * (j - 4));
             }
-            *reinterpret_cast<uint2*>(crow + pc * plane_c + 8 * b) = make_uint2(wlo, whi);
-            srow[pc * plane_s + b] = (uint8_t)sc;
+            *reinterpret_cast<uint2*>(cline + pc * 128 + ((chunk ^ ((ph0 + pc) & 7u)) << 4)) = make_uint2(wlo, whi);
+            sdst[pc * 16] = (uint8_t)sc;
         }
     }
 }
