@@ -96,7 +96,8 @@ def profiled_traffic_ratio():
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,"
+              "power.limit,temperature.gpu,temperature.memory,clocks.mem")
 
     def __init__(self, index: int):
         self.index = index
@@ -130,9 +131,13 @@ class ClockSampler:
         smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
-        pw = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        def num(i):
+            return [float(r[i]) for r in rows if len(r) > i and r[i].replace(".", "").isdigit()]
+        pw, lim, tg, tm, mem = num(3), num(9), num(10), num(11), num(12)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": reasons, "samples": len(rows), "power_w_max": max(pw) if pw else None}
+                "reasons": reasons, "samples": len(rows), "power_w_max": max(pw) if pw else None,
+                "power_limit_w": max(lim) if lim else None, "temp_gpu_c_max": max(tg) if tg else None,
+                "temp_mem_c_max": max(tm) if tm else None, "mem_mhz": statistics.median(mem) if mem else None}
 
 
 # --------------------------------------------------------------------------- CPU oracle sample
@@ -393,35 +398,47 @@ def main_gpu(args):
 
 
 def run_profile_case(args):
-    """Small case for ncu: one matrix (N x K), `--reps` launches of the tensor-core path at --M rows.
+    """Small case for ncu: one matrix (--profile-matrix NxK) or the first L layers of the stack
+    (--profile-layers L), `--reps` launches of one plan at --M rows.
 
     Inputs are drawn and packed on the device like the stack's; prints one summary line."""
     import torch
     import nvfp4_weight_gemm_b200 as tl
     import synth
-    N, K = (int(v) for v in args.profile_matrix.lower().split("x"))
     dev = torch.device("cuda:0")
     torch.cuda.set_device(dev)
     tl.init(0)
     tl.set_gemm_path(PATHS[args.path])
-    w = synth.w_f32_torch(N, K, 0, 0, dev)
-    codes, scales, g = tl.quantize(w)
-    del w
-    x = synth.x_bf16_torch(args.M, K, 0, synth.X_ID_BASE, dev)
-    y = torch.empty((args.M, N), dtype=torch.bfloat16, device=dev)
-    plan = tl.Plan([(codes, scales, g, x, y)], args.M)
+    if args.profile_matrix:
+        N, K = (int(v) for v in args.profile_matrix.lower().split("x"))
+        shapes = [(N, K, "normal")]
+        case = f"{N}x{K}"
+    else:
+        shapes = [(N, K, dist) for (layer, j, name, N, K, dist) in stack_shapes() if layer < args.profile_layers]
+        case = f"{args.profile_layers} layers"
+    ents = []
+    for i, (N, K, dist) in enumerate(shapes):
+        w = synth.w_f32_torch(N, K, 0, i, dev, dist)
+        codes, scales, g = tl.quantize(w)
+        del w
+        x = synth.x_bf16_torch(args.M, K, 0, synth.X_ID_BASE + i, dev)
+        ents.append((codes, scales, g, x, torch.empty((args.M, N), dtype=torch.bfloat16, device=dev)))
+    plan = tl.Plan(ents, args.M)
     for _ in range(args.reps):
         plan.run()
     torch.cuda.synchronize()
     tl.check_device_error()
     plan.close()
-    print(json.dumps({"profile_case": f"{N}x{K}", "M": args.M, "reps": args.reps, "path": args.path}), flush=True)
+    wb = sum(N * K // 2 + N * K // 16 for (N, K, _) in shapes)
+    print(json.dumps({"profile_case": case, "matrices": len(shapes), "w_bytes": wb, "M": args.M, "reps": args.reps,
+                      "path": args.path}), flush=True)
     return 0
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--profile-matrix", default=None, help="NxK: run one matrix --reps times (for ncu)")
+    ap.add_argument("--profile-layers", type=int, default=0, help="L: run the first L layers of the stack (for ncu)")
     ap.add_argument("--M", type=int, default=32)
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--gpus", type=int, default=1)
@@ -435,7 +452,7 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
-    if args.profile_matrix:
+    if args.profile_matrix or args.profile_layers:
         return run_profile_case(args)
     return main_gpu(args)
 

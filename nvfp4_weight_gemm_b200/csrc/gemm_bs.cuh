@@ -12,9 +12,16 @@
 //   D[n][4 m + p] = sum_k  w[n][k] * piece_p[m][k]        (fp32, in tensor memory; N = 4 Mp)
 //   Y[m][n]       = bf16( (sum_p 4^-p D[n][4 m + p]) * g * factor[m] )
 //
-//   * Work. As in gemm_tc.cuh: 128 weight rows x 256 k per tile, one global tile list cut into
-//     equal contiguous shares (stream-K); a split n-tile is reduced by its last contributor in
-//     k order, so every output has one fixed reduction order.
+//   * Work. A tile is 128 weight rows x 256 k; an n-tile is all k-tiles of 128 weight rows.
+//     The host lays out each CTA's work as a list of segments (k-tiles [k0, k1) of one
+//     n-tile), built from the matrices' shapes alone:
+//     - first, whole n-tiles dealt round-robin over the CTAs, so that at any moment the CTAs
+//       work on neighbouring n-tiles of one or two matrices and the X pieces they all read
+//       stay in L2;
+//     - then the remaining n-tiles as one list of k-tiles cut so that every CTA ends with the
+//       same number of k-tiles (stream-K). A cut n-tile ("split") is reduced by its last
+//       contributor, adding the parts in k order, so every output has one fixed reduction
+//       order that does not depend on M.
 //   * Roles, 12 warps.
 //     - Warp 0: copies into a ring of stages, four per tile from four lanes at once. Lanes 0
 //       and 1: a TMA tensor copy each of the tile's W codes and W scales. Lanes 2 and 3: one
@@ -50,15 +57,23 @@ constexpr int BS_SF_COLS = 32;    // tensor-memory columns of scales per stage (
 struct alignas(64) BsMat {
     CUtensorMap tm_codes;   // uint8 {K/2, N, 1}, box 128 B x 128 rows x 1, 128-byte swizzle
     CUtensorMap tm_scales;  // uint8 {K/16, N, 1}, box 16 B x 128 rows x 1
-    const uint8_t* xc;      // X piece codes, [K/256][TC_PIECES][M][128] (swizzled rows, xsplit.cuh)
-    const uint8_t* xs;      // X piece scales, [K/256][TC_PIECES][M][16]
+    const uint8_t* xc;      // X piece codes, [K/256][Mp][TC_PIECES][128] (swizzled lines, xsplit.cuh)
+    const uint8_t* xs;      // X piece scales, [K/256][Mp][TC_PIECES][16]
     const float* xfactor;   // [M], 2^-e per X row (NaN for a non-finite row)
     __nv_bfloat16* y;
     float g;                // the weight's tensor scale
     int N;
-    int k_tiles;
-    int n_tiles;
-    long long tile_begin;
+};
+
+// One stretch of a CTA's work: k-tiles [k0, k1) of n-tile `ntile` of matrix `mat`, in k order.
+struct BsSeg {
+    int mat;
+    int ntile;
+    uint16_t k0, k1;
+    int split;              // -1: the whole n-tile; else the split's index (its four counters)
+    int slot;               // split only: partial slot of this part; the split's parts use
+                            // slots slot - rank .. slot - rank + parts - 1, in k order
+    uint16_t rank, parts;
 };
 
 struct BsParams {
@@ -66,9 +81,10 @@ struct BsParams {
     int n_mats;
     int M;
     int Mp;                 // M rounded up to a multiple of 4: X rows per piece group in the layout
-    long long total_tiles;
-    float* partials;        // [2 * gridDim.x][32][128] fp32
-    unsigned* counters;     // [4 * gridDim.x], zero between launches
+    const BsSeg* segs;      // every CTA's segments, CTA by CTA
+    const int* seg_begin;   // [gridDim.x + 1]: CTA c runs segs[seg_begin[c] .. seg_begin[c+1])
+    float* partials;        // [slots][32][128] fp32
+    unsigned* counters;     // [4 * splits], zero between launches
     int* err;
     BsMat one;
 };
@@ -150,9 +166,7 @@ gemm_bs_kernel(const __grid_constant__ BsParams p) {
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const BsMat* mats = p.mats ? p.mats : &p.one;
-    const long long ctas = gridDim.x;
-    const long long t_begin = tc_range_start(blockIdx.x, p.total_tiles, ctas);
-    const long long t_end = tc_range_start(blockIdx.x + 1, p.total_tiles, ctas);
+    const int s_begin = __ldg(p.seg_begin + blockIdx.x), s_end = __ldg(p.seg_begin + blockIdx.x + 1);
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::STAGES; ++i) {
@@ -193,26 +207,11 @@ gemm_bs_kernel(const __grid_constant__ BsParams p) {
         const uint32_t smem0 = smem_u32(smem);
         int s = 0;
         uint32_t ph = 0, issued = 0, last_ph = 0;
-        // segment walk over BsMat (the same tile list as TcSegIter's)
-        long long t = t_begin;
-        int mi = 0;
-        {
-            int lo = 0, hi = p.n_mats - 1;
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (mats[mid].tile_begin <= t_begin) lo = mid; else hi = mid - 1;
-            }
-            mi = lo;
-        }
         bool ok = true;
-        while (ok && t < t_end) {
-            while (mi + 1 < p.n_mats && mats[mi + 1].tile_begin <= t) ++mi;
-            const BsMat& m = mats[mi];
-            const long long local = t - m.tile_begin;
-            const int ntile = (int)(local / m.k_tiles);
-            const int k0 = (int)(local % m.k_tiles);
-            const long long rem = t_end - t;
-            const int k1 = (int)((m.k_tiles - k0) < rem ? m.k_tiles : k0 + rem);
+        for (int si = s_begin; ok && si < s_end; ++si) {
+            const BsSeg sg = p.segs[si];
+            const BsMat& m = mats[sg.mat];
+            const int ntile = sg.ntile, k0 = sg.k0, k1 = sg.k1;
             const void* tmap = (lane == 0) ? (const void*)&m.tm_codes : (const void*)&m.tm_scales;
             const int c1 = ntile * TC_BLOCK_N;
             const uint8_t* xsrc = (lane == 2) ? m.xc : m.xs;    // k-tile 0; k-tile kt is xbytes further each
@@ -235,7 +234,6 @@ gemm_bs_kernel(const __grid_constant__ BsParams p) {
                 last_ph = (last_ph & ~(1u << s)) | (ph << s);
                 if (++s == C::STAGES) { s = 0; ph ^= 1u; }
             }
-            t += k1 - k0;
         }
         if (lane == 0) {
             for (int i = 0; i < C::STAGES; ++i)
@@ -251,24 +249,10 @@ gemm_bs_kernel(const __grid_constant__ BsParams p) {
         const uint64_t desc_w0 = smem_desc_k_sw128(smem_u32(smem));
         const uint64_t desc_x0 = smem_desc_k_sw128(smem_u32(smem + C::XC_OFF));
         const uint32_t idesc = C::IDESC_BASE | ((uint32_t)(TC_PIECES * p.Mp) >> 3) << 17;
-        long long t = t_begin;
-        int mi = 0;
-        {
-            int lo = 0, hi = p.n_mats - 1;
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (mats[mid].tile_begin <= t_begin) lo = mid; else hi = mid - 1;
-            }
-            mi = lo;
-        }
         bool ok = true;
-        while (ok && t < t_end) {
-            while (mi + 1 < p.n_mats && mats[mi + 1].tile_begin <= t) ++mi;
-            const BsMat& m = mats[mi];
-            const long long local = t - m.tile_begin;
-            const int k0 = (int)(local % m.k_tiles);
-            const long long rem = t_end - t;
-            const int k1 = (int)((m.k_tiles - k0) < rem ? m.k_tiles : k0 + rem);
+        for (int si = s_begin; ok && si < s_end; ++si) {
+            const BsSeg sg = p.segs[si];
+            const int k0 = sg.k0, k1 = sg.k1;
             if (!__all_sync(0xFFFFFFFFu, tc_wait(&accempty[acc], accph ^ 1u, abort_flag))) {
                 if (leader) tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_MMA);
                 break;
@@ -301,7 +285,6 @@ gemm_bs_kernel(const __grid_constant__ BsParams p) {
             if (leader) mma_commit(&accfull[acc]);
             __syncwarp();
             if (++acc == C::ACC_BUFS) { acc = 0; accph ^= 1u; }
-            t += k1 - k0;
         }
         if (leader) mma_commit(drain);
         __syncwarp();
@@ -311,7 +294,8 @@ gemm_bs_kernel(const __grid_constant__ BsParams p) {
         // ------------------------------------------------------------ scales into tensor memory
         const int q = warp & 3;                         // this warp's tensor-memory lane quarter
         const uint32_t t_lane = tmem + ((uint32_t)(32 * q) << 16);
-        const long long ntiles = t_end - t_begin;
+        long long ntiles = 0;
+        for (int si = s_begin; si < s_end; ++si) ntiles += p.segs[si].k1 - p.segs[si].k0;
         int s = 0;
         uint32_t ph = 0;
         bool ok = true;
@@ -380,26 +364,9 @@ gemm_bs_kernel(const __grid_constant__ BsParams p) {
         const int M = p.M;
         int acc = 0;
         uint32_t accph = 0;
-        long long t = t_begin;
-        int mi = 0;
-        {
-            int lo = 0, hi = p.n_mats - 1;
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (mats[mid].tile_begin <= t_begin) lo = mid; else hi = mid - 1;
-            }
-            mi = lo;
-        }
-        while (t < t_end) {
-            while (mi + 1 < p.n_mats && mats[mi + 1].tile_begin <= t) ++mi;
-            const BsMat& m = mats[mi];
-            const long long local = t - m.tile_begin;
-            const int ntile = (int)(local / m.k_tiles);
-            const int k0 = (int)(local % m.k_tiles);
-            const long long rem = t_end - t;
-            const int k1 = (int)((m.k_tiles - k0) < rem ? m.k_tiles : k0 + rem);
-            const long long seg_t0 = t;
-            t += k1 - k0;
+        for (int si = s_begin; si < s_end; ++si) {
+            const BsSeg sg = p.segs[si];
+            const BsMat& m = mats[sg.mat];
             // the matrix's fields in registers: stores to Y must not force them to be re-read
             __nv_bfloat16* const yp = m.y;
             const float gm = m.g;
@@ -410,11 +377,7 @@ gemm_bs_kernel(const __grid_constant__ BsParams p) {
                 break;
             }
             tc_fence_after();
-            const int n = ntile * TC_BLOCK_N + r;
-            const bool whole = (k0 == 0 && k1 == m.k_tiles);
-            const long long ta = m.tile_begin + (long long)ntile * m.k_tiles;
-            const int my_slot = 2 * (int)blockIdx.x + (seg_t0 == t_begin ? 0 : 1);
-            float* mine = p.partials + (size_t)my_slot * (32 * TC_BLOCK_N);
+            const int n = sg.ntile * TC_BLOCK_N + r;
             // sum the pieces in order: v[m] = sum_p 4^-p D[4 m + p] (exact scalings); 16 columns
             // hold rows 4c .. 4c+3
             float v[NX];
@@ -440,35 +403,34 @@ gemm_bs_kernel(const __grid_constant__ BsParams p) {
             __syncwarp();
             if (lane == 0) mbar_arrive(&accempty[acc]);
             if (++acc == C::ACC_BUFS) { acc = 0; accph ^= 1u; }
-            if (whole) {
+            if (sg.split < 0) {
                 if (n < N) bs_store_rows<NX>(v, M, gm, xf, yp + n, N);
                 continue;
             }
+            // a split n-tile: write this part; the last part to arrive (per 32-row quarter)
+            // adds all parts in k order and writes Y
+            float* mine = p.partials + (size_t)sg.slot * (32 * TC_BLOCK_N);
 #pragma unroll
             for (int i = 0; i < NX; ++i)
                 if (i < M) mine[i * TC_BLOCK_N + r] = v[i];
-            // split n-tile: the last contributor for these 32 rows adds all partials in k (CTA) order
-            const long long tb = ta + m.k_tiles;
-            const int f = tc_cta_of(ta, p.total_tiles, ctas);
-            const int l = tc_cta_of(tb - 1, p.total_tiles, ctas);
             __threadfence();
             __syncwarp();
             unsigned old = 0;
-            if (lane == 0) old = atomicAdd(&p.counters[4 * f + q], 1u);
+            if (lane == 0) old = atomicAdd(&p.counters[4 * sg.split + q], 1u);
             old = __shfl_sync(0xFFFFFFFFu, old, 0);
-            if (old == (unsigned)(l - f)) {
+            if (old == (unsigned)(sg.parts - 1)) {
                 __threadfence();
+#pragma unroll
                 for (int i = 0; i < NX; ++i) v[i] = 0.0f;
-                for (int c = f; c <= l; ++c) {
-                    const long long cs = tc_range_start(c, p.total_tiles, ctas);
-                    const int slot = 2 * c + ((ta > cs ? ta : cs) == cs ? 0 : 1);
-                    const float* part = p.partials + (size_t)slot * (32 * TC_BLOCK_N);
+                const float* part0 = p.partials + (size_t)(sg.slot - sg.rank) * (32 * TC_BLOCK_N);
+                for (int rk = 0; rk < sg.parts; ++rk) {
+                    const float* part = part0 + (size_t)rk * (32 * TC_BLOCK_N);
 #pragma unroll
                     for (int i = 0; i < NX; ++i)
                         if (i < M) v[i] += __ldcg(&part[i * TC_BLOCK_N + r]);
                 }
                 if (n < N) bs_store_rows<NX>(v, M, gm, xf, yp + n, N);
-                if (lane == 0) p.counters[4 * f + q] = 0u;   // ready for the next launch
+                if (lane == 0) p.counters[4 * sg.split + q] = 0u;   // ready for the next launch
             }
         }
     }

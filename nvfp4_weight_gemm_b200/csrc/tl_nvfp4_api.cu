@@ -10,6 +10,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -364,8 +365,8 @@ size_t xs_bytes_total(const tl_nvfp4_matrix* mats, int n_mats, int M) {
 }
 
 // BsMat of one matrix whose X pieces live at `xs` (layout of xs_bytes_of).
-tl_status build_bs_mat(tl::BsMat* m, tl::XSplitMat* xm, const void* x, int M, int NX, const void* codes,
-                       const void* scales, float g, void* y, int N, int K, long long tile_begin, unsigned char* xs) {
+tl_status build_bs_mat(tl::BsMat* m, tl::XSplitMat* xm, const void* x, int M, const void* codes,
+                       const void* scales, float g, void* y, int N, int K, unsigned char* xs) {
     memset(m, 0, sizeof *m);
     const cuuint64_t n = (cuuint64_t)N, k = (cuuint64_t)K, P = (cuuint64_t)tl::TC_PIECES, Mp = (cuuint64_t)round4(M);
     unsigned char* xc = xs;
@@ -384,9 +385,6 @@ tl_status build_bs_mat(tl::BsMat* m, tl::XSplitMat* xm, const void* x, int M, in
     m->y = static_cast<__nv_bfloat16*>(y);
     m->g = g;
     m->N = N;
-    m->k_tiles = K / tl::TC_BLOCK_K;
-    m->n_tiles = (N + tl::TC_BLOCK_N - 1) / tl::TC_BLOCK_N;
-    m->tile_begin = tile_begin;
     xm->x = static_cast<const __nv_bfloat16*>(x);
     xm->codes = xc;
     xm->scales = xsc;
@@ -395,18 +393,107 @@ tl_status build_bs_mat(tl::BsMat* m, tl::XSplitMat* xm, const void* x, int M, in
     return TL_OK;
 }
 
+// Each CTA's list of segments (gemm_bs.cuh): whole n-tiles dealt round-robin first, so that
+// the CTAs move through the matrices side by side and share the X pieces in L2; the last two
+// to three rounds' worth of n-tiles are cut into equal shares of k-tiles (stream-K), so every
+// CTA ends with the same number of k-tiles. Depends only on the shapes and the grid.
+struct BsSchedule {
+    std::vector<tl::BsSeg> segs;
+    std::vector<int> begin;   // [grid + 1]
+    int splits = 0;           // split n-tiles (four counters each)
+    int slots = 0;            // partial slots
+};
+
+void build_schedule(const tl_nvfp4_matrix* mats, int n_mats, int grid, BsSchedule* out) {
+    struct Unit { int mat, ntile, kt; };
+    std::vector<Unit> units;
+    for (int i = 0; i < n_mats; ++i) {
+        const int nt = (mats[i].N + tl::TC_BLOCK_N - 1) / tl::TC_BLOCK_N, kt = mats[i].K / tl::TC_BLOCK_K;
+        for (int j = 0; j < nt; ++j) units.push_back({i, j, kt});
+    }
+    const long long U = (long long)units.size(), G = grid;
+    const long long R = std::max(0LL, U / G - 2) * G;          // n-tiles dealt whole
+    std::vector<std::vector<tl::BsSeg>> per(grid);
+    std::vector<long long> load(grid, 0);
+    auto seg = [](const Unit& u, int k0, int k1) {
+        tl::BsSeg sg;
+        sg.mat = u.mat;
+        sg.ntile = u.ntile;
+        sg.k0 = (uint16_t)k0;
+        sg.k1 = (uint16_t)k1;
+        sg.split = -1;
+        sg.slot = 0;
+        sg.rank = 0;
+        sg.parts = 1;
+        return sg;
+    };
+    for (long long u = 0; u < R; ++u) {
+        per[u % G].push_back(seg(units[u], 0, units[u].kt));
+        load[u % G] += units[u].kt;
+    }
+    long long total = 0, rest = 0;
+    for (long long c = 0; c < G; ++c) total += load[c];
+    for (long long u = R; u < U; ++u) rest += units[u].kt;
+    total += rest;
+    const long long target = (total + G - 1) / G;
+    // cut the rest: CTA c takes target - load[c] k-tiles (the last CTA whatever is left)
+    struct Part { int cta; long long unit; int k0, k1; };
+    std::vector<Part> parts;
+    long long u = R;
+    int k = 0;
+    for (int c = 0; c < grid && u < U; ++c) {
+        long long need = (c == grid - 1) ? (1LL << 62) : target - load[c];
+        while (need > 0 && u < U) {
+            const int take = (int)std::min<long long>(need, units[u].kt - k);
+            parts.push_back({c, u, k, k + take});
+            k += take;
+            need -= take;
+            if (k == units[u].kt) { ++u; k = 0; }
+        }
+    }
+    out->splits = 0;
+    out->slots = 0;
+    for (size_t i = 0; i < parts.size();) {
+        size_t j = i;
+        while (j < parts.size() && parts[j].unit == parts[i].unit) ++j;
+        const Unit& un = units[parts[i].unit];
+        if (j - i == 1) {
+            per[parts[i].cta].push_back(seg(un, parts[i].k0, parts[i].k1));
+        } else {
+            const int split = out->splits++;
+            for (size_t r = i; r < j; ++r) {
+                tl::BsSeg sg = seg(un, parts[r].k0, parts[r].k1);
+                sg.split = split;
+                sg.slot = out->slots++;
+                sg.rank = (uint16_t)(r - i);
+                sg.parts = (uint16_t)(j - i);
+                per[parts[r].cta].push_back(sg);
+            }
+        }
+        i = j;
+    }
+    out->segs.clear();
+    out->begin.assign(grid + 1, 0);
+    for (int c = 0; c < grid; ++c) {
+        out->begin[c] = (int)out->segs.size();
+        out->segs.insert(out->segs.end(), per[c].begin(), per[c].end());
+    }
+    out->begin[grid] = (int)out->segs.size();
+}
+
 struct BsLaunch {
     tl::BsParams bp;
     tl::XSplitParams xp;
     std::vector<tl::BsMat> tbl;
     std::vector<tl::XSplitMat> xtbl;
+    BsSchedule sched;
+    int grid = 0;
 };
 
 // Validate (as build_params) and build the block-scaled launch of a stack whose X pieces go to
 // `xs` (xs_bytes_total bytes).
 tl_status build_bs(const tl_nvfp4_matrix* mats, int n_mats, int M, const unsigned char* x_dev, unsigned char* y_dev,
-                   unsigned char* xs, BsLaunch* L) {
-    const int NX = M <= 16 ? 16 : 32;
+                   unsigned char* xs, int num_sms, BsLaunch* L) {
     L->tbl.assign(n_mats, tl::BsMat());
     L->xtbl.assign(n_mats, tl::XSplitMat());
     long long tiles = 0;
@@ -415,10 +502,10 @@ tl_status build_bs(const tl_nvfp4_matrix* mats, int n_mats, int M, const unsigne
         const tl_nvfp4_matrix& m = mats[i];
         const void* x = x_dev ? static_cast<const void*>(x_dev + xoff) : m.x;
         void* y = y_dev ? static_cast<void*>(y_dev + yoff) : m.y;
-        tl_status st = build_bs_mat(&L->tbl[i], &L->xtbl[i], x, M, NX, m.w_codes, m.w_scales, m.global_scale, y,
-                                    m.N, m.K, tiles, xs + soff);
+        tl_status st = build_bs_mat(&L->tbl[i], &L->xtbl[i], x, M, m.w_codes, m.w_scales, m.global_scale, y,
+                                    m.N, m.K, xs + soff);
         if (st != TL_OK) return st;
-        tiles += (long long)L->tbl[i].n_tiles * L->tbl[i].k_tiles;
+        tiles += (long long)((m.N + tl::TC_BLOCK_N - 1) / tl::TC_BLOCK_N) * (m.K / tl::TC_BLOCK_K);
         xoff += (size_t)2 * M * m.K;
         yoff += (size_t)2 * M * m.N;
         soff += xs_bytes_of(M, m.K);
@@ -427,8 +514,12 @@ tl_status build_bs(const tl_nvfp4_matrix* mats, int n_mats, int M, const unsigne
     L->bp.n_mats = n_mats;
     L->bp.M = M;
     L->bp.Mp = round4(M);
-    L->bp.total_tiles = tiles;
     L->bp.mats = nullptr;
+    L->grid = (int)std::min<long long>(tiles, num_sms);
+    build_schedule(mats, n_mats, L->grid, &L->sched);
+    if (L->sched.slots > 2 * num_sms || L->sched.splits > num_sms)
+        return fail(TL_ERR_DEVICE_FAULT, "internal: schedule needs %d partial slots and %d splits", L->sched.slots,
+                    L->sched.splits);
     if (n_mats == 1) L->bp.one = L->tbl[0];
     memset(&L->xp, 0, sizeof L->xp);
     L->xp.n_mats = n_mats;
@@ -440,10 +531,9 @@ tl_status build_bs(const tl_nvfp4_matrix* mats, int n_mats, int M, const unsigne
 }
 
 template <int NX>
-tl_status launch_bs_gemm(DevState& d, tl::BsParams& p, cudaStream_t stream) {
+tl_status launch_bs_gemm(DevState& d, tl::BsParams& p, int grid, cudaStream_t stream) {
     using C = tl::BsCfg<NX>;
     TL_CUDA(cudaFuncSetAttribute(tl::gemm_bs_kernel<NX>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
-    const long long grid = p.total_tiles < d.num_sms ? p.total_tiles : d.num_sms;
     p.partials = d.partials;
     p.counters = d.counters;
     p.err = d.err;
@@ -452,11 +542,21 @@ tl_status launch_bs_gemm(DevState& d, tl::BsParams& p, cudaStream_t stream) {
     return TL_OK;
 }
 
-// The X split, then the GEMM, on `stream`.
-tl_status launch_bs(DevState& d, tl::BsParams bp, const tl::XSplitParams& xp, cudaStream_t stream) {
+// The X split, then the GEMM, on `stream` (bp.segs / bp.seg_begin already on the device).
+tl_status launch_bs(DevState& d, tl::BsParams bp, const tl::XSplitParams& xp, int grid, cudaStream_t stream) {
     tl::x_split_kernel<<<dim3((unsigned)xp.Mp, (unsigned)xp.n_mats), tl::XS_THREADS, 0, stream>>>(xp);
     TL_CUDA(cudaGetLastError());
-    return (bp.M <= 16) ? launch_bs_gemm<16>(d, bp, stream) : launch_bs_gemm<32>(d, bp, stream);
+    return (bp.M <= 16) ? launch_bs_gemm<16>(d, bp, grid, stream) : launch_bs_gemm<32>(d, bp, grid, stream);
+}
+
+// The schedule as one device blob: segments, then the per-CTA offsets.
+std::vector<unsigned char> schedule_blob(const BsSchedule& sc, size_t* begin_off) {
+    const size_t a = round256(sc.segs.size() * sizeof(tl::BsSeg));
+    std::vector<unsigned char> blob(a + sc.begin.size() * sizeof(int), 0);
+    memcpy(blob.data(), sc.segs.data(), sc.segs.size() * sizeof(tl::BsSeg));
+    memcpy(blob.data() + a, sc.begin.data(), sc.begin.size() * sizeof(int));
+    *begin_off = a;
+    return blob;
 }
 
 // Grow the per-device X-piece scratch to `bytes` (never inside a graph capture).
@@ -484,8 +584,17 @@ tl_status run_stack_bs(const tl_nvfp4_matrix* mats, int n_mats, int M, const uns
     tl_status st = ensure_xs(*d, xs_bytes_total(mats, n_mats, M), stream);
     if (st != TL_OK) return st;
     BsLaunch L;
-    st = build_bs(mats, n_mats, M, x_dev, y_dev, d->xs_buf, &L);
+    st = build_bs(mats, n_mats, M, x_dev, y_dev, d->xs_buf, d->num_sms, &L);
     if (st != TL_OK) return st;
+    {
+        size_t boff = 0;
+        const std::vector<unsigned char> blob = schedule_blob(L.sched, &boff);
+        const void* t = nullptr;
+        st = device_table(*d, blob.data(), blob.size(), stream, &t);
+        if (st != TL_OK) return st;
+        L.bp.segs = static_cast<const tl::BsSeg*>(t);
+        L.bp.seg_begin = reinterpret_cast<const int*>(static_cast<const unsigned char*>(t) + boff);
+    }
     if (n_mats > 1) {
         const void* t = nullptr;
         st = device_table(*d, L.tbl.data(), L.tbl.size() * sizeof(tl::BsMat), stream, &t);
@@ -495,7 +604,7 @@ tl_status run_stack_bs(const tl_nvfp4_matrix* mats, int n_mats, int M, const uns
         if (st != TL_OK) return st;
         L.xp.mats = static_cast<const tl::XSplitMat*>(t);
     }
-    return launch_bs(*d, L.bp, L.xp, stream);
+    return launch_bs(*d, L.bp, L.xp, L.grid, stream);
 }
 
 
@@ -610,7 +719,8 @@ struct tl_nvfp4_plan_st {
     tl::TcMat* table = nullptr;       // device copy when n_mats > 1
     tl::BsParams bparams;             // block-scaled path
     tl::XSplitParams xparams;
-    void* bs_tables = nullptr;        // device copies of the BsMat and XSplitMat tables (n_mats > 1)
+    int grid = 0;                     // CTAs of the block-scaled GEMM
+    void* bs_tables = nullptr;        // device copies of the BsMat and XSplitMat tables (n_mats > 1) and the schedule
     unsigned char* xs = nullptr;      // the plan's own X-piece scratch
     const void* x_base = nullptr;     // packed X_i buffer (or nullptr if not packed)
     void* y_base = nullptr;           // packed Y_i buffer (or nullptr if not packed)
@@ -624,25 +734,32 @@ namespace {
 tl_status plan_build_bs(tl_nvfp4_plan plan, const tl_nvfp4_matrix* mats, int n_mats, int M) {
     TL_CUDA(cudaMalloc(&plan->xs, xs_bytes_total(mats, n_mats, M)));
     BsLaunch L;
-    tl_status st = build_bs(mats, n_mats, M, nullptr, nullptr, plan->xs, &L);
+    tl_status st = build_bs(mats, n_mats, M, nullptr, nullptr, plan->xs, plan->d->num_sms, &L);
     if (st != TL_OK) return st;
+    // one device allocation: descriptor tables (n_mats > 1), then the schedule
+    size_t boff = 0;
+    const std::vector<unsigned char> blob = schedule_blob(L.sched, &boff);
+    const size_t b1 = n_mats > 1 ? round256(L.tbl.size() * sizeof(tl::BsMat)) : 0;
+    const size_t b2 = n_mats > 1 ? round256(L.xtbl.size() * sizeof(tl::XSplitMat)) : 0;
+    TL_CUDA(cudaMalloc(&plan->bs_tables, b1 + b2 + blob.size()));
+    unsigned char* t = static_cast<unsigned char*>(plan->bs_tables);
     if (n_mats > 1) {
-        const size_t b1 = round256(L.tbl.size() * sizeof(tl::BsMat));
-        const size_t b2 = L.xtbl.size() * sizeof(tl::XSplitMat);
-        TL_CUDA(cudaMalloc(&plan->bs_tables, b1 + b2));
-        unsigned char* t = static_cast<unsigned char*>(plan->bs_tables);
         TL_CUDA(cudaMemcpy(t, L.tbl.data(), L.tbl.size() * sizeof(tl::BsMat), cudaMemcpyHostToDevice));
-        TL_CUDA(cudaMemcpy(t + b1, L.xtbl.data(), b2, cudaMemcpyHostToDevice));
+        TL_CUDA(cudaMemcpy(t + b1, L.xtbl.data(), L.xtbl.size() * sizeof(tl::XSplitMat), cudaMemcpyHostToDevice));
         L.bp.mats = reinterpret_cast<const tl::BsMat*>(t);
         L.xp.mats = reinterpret_cast<const tl::XSplitMat*>(t + b1);
     }
+    TL_CUDA(cudaMemcpy(t + b1 + b2, blob.data(), blob.size(), cudaMemcpyHostToDevice));
+    L.bp.segs = reinterpret_cast<const tl::BsSeg*>(t + b1 + b2);
+    L.bp.seg_begin = reinterpret_cast<const int*>(t + b1 + b2 + boff);
     plan->bparams = L.bp;
     plan->xparams = L.xp;
+    plan->grid = L.grid;
     return TL_OK;
 }
 
 tl_status plan_launch(tl_nvfp4_plan plan, cudaStream_t s) {
-    if (plan->path == TL_PATH_BLOCK_SCALED) return launch_bs(*plan->d, plan->bparams, plan->xparams, s);
+    if (plan->path == TL_PATH_BLOCK_SCALED) return launch_bs(*plan->d, plan->bparams, plan->xparams, plan->grid, s);
     tl::TcParams p = plan->params;
     return launch_tc_any(*plan->d, p, s);
 }
