@@ -9,7 +9,8 @@
 // 1. e[m] is the power of two that brings the row's largest |x| into [2^7, 2^8).
 // 2. Piece p codes the block's remaining residual r, taken in units 4^-p times those of piece
 //    0 (u = 4^p r): s_p is the smallest E4M3 value with 6 * s_p >= max|u| (so no code
-//    saturates), c_p = RNE_e2m1(u / s_p), and u -= c_p * s_p.
+//    saturates), c_p = RNE_e2m1(u / s_p), and u -= c_p * s_p. (The kernel keeps r in piece 0's
+//    units and scales s_p instead; the powers of two make the two forms give the same bits.)
 //
 // Why 4^p: a piece leaves a residual of at most s_p <= 1.125 * max|u| / 6 (one E4M3 step of
 // rounding up), so 4 * residual <= 0.75 * max|u|: every piece's |u| stays below 2^8 and its
@@ -50,10 +51,12 @@ struct XSplitMat {
     uint8_t* scales;          // [K/256][TC_PIECES][M][16]
     float* factor;            // [M]
     int K;
+    int chunk0;               // first chunk of this matrix in the launch's chunk list
 };
 
 struct XSplitParams {
     const XSplitMat* mats;    // device table, or nullptr to use `one`
+    const uint16_t* chunk_mat;// [chunks]: the matrix of each chunk (with the table)
     int n_mats;
     int M;
     int Mp;                   // M rounded up to a multiple of 4
@@ -106,35 +109,37 @@ __host__ __device__ __forceinline__ uint32_t xs_e4m3_ceil_div6(float amax) {
     return code;
 }
 
-// Two floats to two E2M1 codes in one byte (round to nearest even, saturating at +-6):
-// lo lands in the low nibble.
-__device__ __forceinline__ uint32_t xs_cvt_e2m1x2(float lo, float hi) {
-    uint32_t r;
-    asm("{\n\t.reg .b8 b;\n\t"
-        "cvt.rn.satfinite.e2m1x2.f32 b, %2, %1;\n\t"
-        "cvt.u32.u8 %0, b;\n\t}"
-        : "=r"(r) : "f"(lo), "f"(hi));
-    return r;
+// Eight floats to eight E2M1 codes (round to nearest even, saturating at +-6), packed low
+// nibble first into one word, and the values of those codes as four f16 pairs (exact).
+__device__ __forceinline__ uint32_t xs_e2m1x8(const float (&q)[8], uint32_t (&h)[4]) {
+    uint32_t codes;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %8, %7;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %10, %9;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %12, %11;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %4, b3;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(codes), "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+        : "f"(q[0]), "f"(q[1]), "f"(q[2]), "f"(q[3]), "f"(q[4]), "f"(q[5]), "f"(q[6]), "f"(q[7]));
+    return codes;
 }
 
-// The two E2M1 values of a code byte (low nibble first) as floats.
-__device__ __forceinline__ float2 xs_e2m1x2_values(uint32_t byte) {
-    uint32_t h2;
-    asm("{\n\t.reg .b8 b;\n\t"
-        "cvt.u8.u32 b, %1;\n\t"
-        "cvt.rn.f16x2.e2m1x2 %0, b;\n\t}"
-        : "=r"(h2) : "r"(byte));
-    return __half22float2(*reinterpret_cast<const __half2*>(&h2));
-}
+constexpr int XS_THREADS = 256;
+constexpr int XS_CHUNK_BLOCKS = XS_THREADS;   // 16-k blocks per chunk: one per thread
 
-constexpr int XS_THREADS = 128;
-
-// Grid (Mp, n_mats): one CTA per row of one matrix; rows M .. Mp-1 write zero pieces.
+// Grid (Mp, chunks): one CTA per row and chunk of XS_CHUNK_BLOCKS 16-k blocks of one matrix (a
+// matrix has ceil(K/16 / XS_CHUNK_BLOCKS) chunks); rows M .. Mp-1 write zero pieces. Every CTA
+// of a row finds the row's largest |x| itself, so the chunks need no ordering among them.
 __global__ void __launch_bounds__(XS_THREADS) x_split_kernel(const __grid_constant__ XSplitParams p) {
     __shared__ float red[XS_THREADS / 32];
     __shared__ int bad_sh;
-    const XSplitMat& m = p.mats ? p.mats[blockIdx.y] : p.one;
+    const XSplitMat& m = p.mats ? p.mats[__ldg(p.chunk_mat + blockIdx.y)] : p.one;
     const int row = blockIdx.x;
+    const int chunk = (int)blockIdx.y - m.chunk0;
     const int K = m.K;
     const int M = p.M, Mp = p.Mp;
     const bool pad_row = row >= M;
@@ -146,6 +151,7 @@ __global__ void __launch_bounds__(XS_THREADS) x_split_kernel(const __grid_consta
     if (threadIdx.x == 0) bad_sh = 0;
     float mx = 0.0f;
     bool bad = false;
+#pragma unroll 4
     for (int k8 = threadIdx.x; !pad_row && k8 < K / 8; k8 += XS_THREADS) {
         const uint4 v = __ldg(reinterpret_cast<const uint4*>(x) + k8);
         const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -172,11 +178,12 @@ __global__ void __launch_bounds__(XS_THREADS) x_split_kernel(const __grid_consta
         frexpf(r, &fe);                         // r in [2^(fe-1), 2^fe)
         e = 8 - fe;
     }
-    if (threadIdx.x == 0 && !pad_row) factor[row] = bad_row ? __int_as_float(0x7FC00000) : ldexpf(1.0f, -e);
+    if (threadIdx.x == 0 && !pad_row && chunk == 0) factor[row] = bad_row ? __int_as_float(0x7FC00000) : ldexpf(1.0f, -e);
     // exact scaling by 2^e in two steps (each factor a normal power of two)
     const float p1 = ldexpf(1.0f, e / 2), p2 = ldexpf(1.0f, e - e / 2);
-    // 2. four pieces per 16-k block, one thread per block
-    for (int b = threadIdx.x; b < K / 16; b += XS_THREADS) {
+    // 2. four pieces per 16-k block, one thread per block of this chunk
+    const int b = chunk * XS_CHUNK_BLOCKS + (int)threadIdx.x;
+    if (b < K / 16) {
         const int kt = b >> 4, bt = b & 15;       // k-tile, block within it
         const size_t j0 = ((size_t)kt * Mp + (size_t)row) * TC_PIECES;   // line of piece 0
         // piece p is line j0 + p; its 16-byte chunk bt/2 sits at chunk (bt/2) ^ ((j0 + p) & 7)
@@ -189,8 +196,9 @@ __global__ void __launch_bounds__(XS_THREADS) x_split_kernel(const __grid_consta
                 *reinterpret_cast<uint2*>(cline + pc * 128 + ((chunk ^ ((ph0 + pc) & 7u)) << 4)) = make_uint2(0u, 0u);
                 sdst[pc * 16] = 0;
             }
-            continue;
+            return;
         }
+        // u: the block's residual, always in piece-0 units (x * 2^e)
         float u[16];
         {
             const uint4 v0 = __ldg(reinterpret_cast<const uint4*>(x) + 2 * b);
@@ -204,22 +212,30 @@ __global__ void __launch_bounds__(XS_THREADS) x_split_kernel(const __grid_consta
         }
 #pragma unroll
         for (int pc = 0; pc < TC_PIECES; ++pc) {
+            const float unit = (float)(1 << (2 * pc));          // piece pc's units: 4^-pc of piece 0's
             float amax = 0.0f;
 #pragma unroll
             for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(u[i]));
-            const uint32_t sc = xs_e4m3_ceil_div6(amax);
-            const float s = xs_e4m3_value(sc);
-            const float inv = (sc != 0u) ? 1.0f / s : 0.0f;
-            uint32_t wlo = 0, whi = 0;
+            const uint32_t sc = xs_e4m3_ceil_div6(amax * unit);
+            const float sv = xs_e4m3_value(sc);
+            const float s = sv * (1.0f / unit);                 // the scale in piece-0 units (exact)
+            const float inv = (sc != 0u) ? unit / sv : 0.0f;    // = 1 / s
+            uint32_t w[2];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const uint32_t byte = xs_cvt_e2m1x2(u[2 * j] * inv, u[2 * j + 1] * inv);
-                const float2 q = xs_e2m1x2_values(byte);
-                u[2 * j] = 4.0f * fmaf(-q.x, s, u[2 * j]);          // the next piece's units
-                u[2 * j + 1] = 4.0f * fmaf(-q.y, s, u[2 * j + 1]);
-                if (j < 4) wlo |= byte << (8 * j); else whi |= byte << (8 * (j - 4));
+            for (int hlf = 0; hlf < 2; ++hlf) {
+                float q[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) q[i] = u[8 * hlf + i] * inv;
+                uint32_t h[4];
+                w[hlf] = xs_e2m1x8(q, h);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 qv = __half22float2(*reinterpret_cast<const __half2*>(&h[i]));
+                    u[8 * hlf + 2 * i] = fmaf(-qv.x, s, u[8 * hlf + 2 * i]);
+                    u[8 * hlf + 2 * i + 1] = fmaf(-qv.y, s, u[8 * hlf + 2 * i + 1]);
+                }
             }
-            *reinterpret_cast<uint2*>(cline + pc * 128 + ((chunk ^ ((ph0 + pc) & 7u)) << 4)) = make_uint2(wlo, whi);
+            *reinterpret_cast<uint2*>(cline + pc * 128 + ((chunk ^ ((ph0 + pc) & 7u)) << 4)) = make_uint2(w[0], w[1]);
             sdst[pc * 16] = (uint8_t)sc;
         }
     }
