@@ -79,16 +79,24 @@ def source_hash():
     return h.hexdigest()[:16]
 
 
-def profiled_traffic_ratio():
-    """DRAM bytes / algorithmic bytes of the hot kernel, from the committed ncu summary, if it
-    was taken on this source (None otherwise)."""
+def profiled_traffic(shapes, path):
+    """DRAM bytes of the mean stack pass (M = 1..32), from the committed ncu record of the pass's
+    kernels at several M (ratio to the algorithmic bytes, linear in between), if it was taken on
+    this source and path (None otherwise)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
-    if d.get("source_hash") != source_hash():
+    if d.get("source_hash") != source_hash() or not d.get("kernels", "").startswith(KERNELS[path].split(" (")[0]):
         return None
-    return d.get("dram_over_algorithmic")
+    pts = sorted((int(m), v["ratio"]) for m, v in d["per_M"].items())
+
+    def ratio(M):
+        for (m0, r0), (m1, r1) in zip(pts, pts[1:]):
+            if m0 <= M <= m1:
+                return r0 + (r1 - r0) * (M - m0) / (m1 - m0)
+        return pts[0][1] if M < pts[0][0] else pts[-1][1]
+    return round(sum(ratio(M) * pass_bytes(shapes, M) for M in M_SWEEP) / len(M_SWEEP))
 
 
 # --------------------------------------------------------------------------- clocks
@@ -358,9 +366,8 @@ def main_gpu(args):
         peak, peak_kind = load_peaks()
         value = world * bytes_step * args.steps / (total_ms * 1e-3) / 1e9
         achieved = bytes_step * args.steps / (launch_ms_sum * 1e-3) / 1e9
-        ratio = profiled_traffic_ratio()
-        # per launch, like `achieved`: the mean algorithmic bytes of one stack pass x the ratio
-        traffic = None if ratio is None else round(ratio * bytes_step / len(M_SWEEP))
+        # per launch, like `achieved`: DRAM bytes of the mean stack pass
+        traffic = profiled_traffic(shapes, args.path)
         stair = {}
         for M in M_SWEEP:
             gbs = pass_bytes(shapes, M) / (per_M[M] * 1e-3) / 1e9

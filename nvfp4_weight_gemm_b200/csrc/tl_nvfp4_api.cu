@@ -390,7 +390,6 @@ tl_status build_bs_mat(tl::BsMat* m, tl::XSplitMat* xm, const void* x, int M, co
     xm->scales = xsc;
     xm->factor = xf;
     xm->K = K;
-    xm->chunk0 = 0;
     return TL_OK;
 }
 
@@ -487,7 +486,6 @@ struct BsLaunch {
     tl::XSplitParams xp;
     std::vector<tl::BsMat> tbl;
     std::vector<tl::XSplitMat> xtbl;
-    std::vector<uint16_t> chunk_mat;   // the split kernel's chunk -> matrix map
     BsSchedule sched;
     int grid = 0;
 };
@@ -523,14 +521,6 @@ tl_status build_bs(const tl_nvfp4_matrix* mats, int n_mats, int M, const unsigne
         return fail(TL_ERR_DEVICE_FAULT, "internal: schedule needs %d partial slots and %d splits", L->sched.slots,
                     L->sched.splits);
     if (n_mats == 1) L->bp.one = L->tbl[0];
-    L->chunk_mat.clear();
-    for (int i = 0; i < n_mats; ++i) {
-        L->xtbl[i].chunk0 = (int)L->chunk_mat.size();
-        const int nb = mats[i].K / 16, nc = (nb + tl::XS_CHUNK_BLOCKS - 1) / tl::XS_CHUNK_BLOCKS;
-        L->chunk_mat.insert(L->chunk_mat.end(), nc, (uint16_t)i);
-    }
-    if (L->chunk_mat.size() > 65535)
-        return fail(TL_ERR_UNSUPPORTED, "the stack's K values need %zu split chunks (> 65535)", L->chunk_mat.size());
     memset(&L->xp, 0, sizeof L->xp);
     L->xp.n_mats = n_mats;
     L->xp.M = M;
@@ -553,9 +543,8 @@ tl_status launch_bs_gemm(DevState& d, tl::BsParams& p, int grid, cudaStream_t st
 }
 
 // The X split, then the GEMM, on `stream` (bp.segs / bp.seg_begin already on the device).
-tl_status launch_bs(DevState& d, tl::BsParams bp, const tl::XSplitParams& xp, int chunks, int grid,
-                    cudaStream_t stream) {
-    tl::x_split_kernel<<<dim3((unsigned)xp.Mp, (unsigned)chunks), tl::XS_THREADS, 0, stream>>>(xp);
+tl_status launch_bs(DevState& d, tl::BsParams bp, const tl::XSplitParams& xp, int grid, cudaStream_t stream) {
+    tl::x_split_kernel<<<dim3((unsigned)xp.Mp, (unsigned)xp.n_mats), tl::XS_THREADS, 0, stream>>>(xp);
     TL_CUDA(cudaGetLastError());
     return (bp.M <= 16) ? launch_bs_gemm<16>(d, bp, grid, stream) : launch_bs_gemm<32>(d, bp, grid, stream);
 }
@@ -611,17 +600,11 @@ tl_status run_stack_bs(const tl_nvfp4_matrix* mats, int n_mats, int M, const uns
         st = device_table(*d, L.tbl.data(), L.tbl.size() * sizeof(tl::BsMat), stream, &t);
         if (st != TL_OK) return st;
         L.bp.mats = static_cast<const tl::BsMat*>(t);
-        // the XSplitMat table, then the chunk -> matrix map
-        const size_t a = round256(L.xtbl.size() * sizeof(tl::XSplitMat));
-        std::vector<unsigned char> blob(a + L.chunk_mat.size() * sizeof(uint16_t), 0);
-        memcpy(blob.data(), L.xtbl.data(), L.xtbl.size() * sizeof(tl::XSplitMat));
-        memcpy(blob.data() + a, L.chunk_mat.data(), L.chunk_mat.size() * sizeof(uint16_t));
-        st = device_table(*d, blob.data(), blob.size(), stream, &t);
+        st = device_table(*d, L.xtbl.data(), L.xtbl.size() * sizeof(tl::XSplitMat), stream, &t);
         if (st != TL_OK) return st;
         L.xp.mats = static_cast<const tl::XSplitMat*>(t);
-        L.xp.chunk_mat = reinterpret_cast<const uint16_t*>(static_cast<const unsigned char*>(t) + a);
     }
-    return launch_bs(*d, L.bp, L.xp, (int)L.chunk_mat.size(), L.grid, stream);
+    return launch_bs(*d, L.bp, L.xp, L.grid, stream);
 }
 
 
@@ -737,7 +720,6 @@ struct tl_nvfp4_plan_st {
     tl::BsParams bparams;             // block-scaled path
     tl::XSplitParams xparams;
     int grid = 0;                     // CTAs of the block-scaled GEMM
-    int chunks = 0;                   // CTAs per X row of the split kernel
     void* bs_tables = nullptr;        // device copies of the BsMat and XSplitMat tables (n_mats > 1) and the schedule
     unsigned char* xs = nullptr;      // the plan's own X-piece scratch
     const void* x_base = nullptr;     // packed X_i buffer (or nullptr if not packed)
@@ -758,19 +740,14 @@ tl_status plan_build_bs(tl_nvfp4_plan plan, const tl_nvfp4_matrix* mats, int n_m
     size_t boff = 0;
     const std::vector<unsigned char> blob = schedule_blob(L.sched, &boff);
     const size_t b1 = n_mats > 1 ? round256(L.tbl.size() * sizeof(tl::BsMat)) : 0;
-    const size_t b2 = n_mats > 1 ? round256(L.xtbl.size() * sizeof(tl::XSplitMat)) +
-                                       round256(L.chunk_mat.size() * sizeof(uint16_t)) : 0;
+    const size_t b2 = n_mats > 1 ? round256(L.xtbl.size() * sizeof(tl::XSplitMat)) : 0;
     TL_CUDA(cudaMalloc(&plan->bs_tables, b1 + b2 + blob.size()));
     unsigned char* t = static_cast<unsigned char*>(plan->bs_tables);
     if (n_mats > 1) {
         TL_CUDA(cudaMemcpy(t, L.tbl.data(), L.tbl.size() * sizeof(tl::BsMat), cudaMemcpyHostToDevice));
-        const size_t xa = round256(L.xtbl.size() * sizeof(tl::XSplitMat));
         TL_CUDA(cudaMemcpy(t + b1, L.xtbl.data(), L.xtbl.size() * sizeof(tl::XSplitMat), cudaMemcpyHostToDevice));
-        TL_CUDA(cudaMemcpy(t + b1 + xa, L.chunk_mat.data(), L.chunk_mat.size() * sizeof(uint16_t),
-                           cudaMemcpyHostToDevice));
         L.bp.mats = reinterpret_cast<const tl::BsMat*>(t);
         L.xp.mats = reinterpret_cast<const tl::XSplitMat*>(t + b1);
-        L.xp.chunk_mat = reinterpret_cast<const uint16_t*>(t + b1 + xa);
     }
     TL_CUDA(cudaMemcpy(t + b1 + b2, blob.data(), blob.size(), cudaMemcpyHostToDevice));
     L.bp.segs = reinterpret_cast<const tl::BsSeg*>(t + b1 + b2);
@@ -778,13 +755,11 @@ tl_status plan_build_bs(tl_nvfp4_plan plan, const tl_nvfp4_matrix* mats, int n_m
     plan->bparams = L.bp;
     plan->xparams = L.xp;
     plan->grid = L.grid;
-    plan->chunks = (int)L.chunk_mat.size();
     return TL_OK;
 }
 
 tl_status plan_launch(tl_nvfp4_plan plan, cudaStream_t s) {
-    if (plan->path == TL_PATH_BLOCK_SCALED)
-        return launch_bs(*plan->d, plan->bparams, plan->xparams, plan->chunks, plan->grid, s);
+    if (plan->path == TL_PATH_BLOCK_SCALED) return launch_bs(*plan->d, plan->bparams, plan->xparams, plan->grid, s);
     tl::TcParams p = plan->params;
     return launch_tc_any(*plan->d, p, s);
 }

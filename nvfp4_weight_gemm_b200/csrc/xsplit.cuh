@@ -51,12 +51,10 @@ struct XSplitMat {
     uint8_t* scales;          // [K/256][TC_PIECES][M][16]
     float* factor;            // [M]
     int K;
-    int chunk0;               // first chunk of this matrix in the launch's chunk list
 };
 
 struct XSplitParams {
     const XSplitMat* mats;    // device table, or nullptr to use `one`
-    const uint16_t* chunk_mat;// [chunks]: the matrix of each chunk (with the table)
     int n_mats;
     int M;
     int Mp;                   // M rounded up to a multiple of 4
@@ -129,17 +127,13 @@ __device__ __forceinline__ uint32_t xs_e2m1x8(const float (&q)[8], uint32_t (&h)
 }
 
 constexpr int XS_THREADS = 256;
-constexpr int XS_CHUNK_BLOCKS = XS_THREADS;   // 16-k blocks per chunk: one per thread
 
-// Grid (Mp, chunks): one CTA per row and chunk of XS_CHUNK_BLOCKS 16-k blocks of one matrix (a
-// matrix has ceil(K/16 / XS_CHUNK_BLOCKS) chunks); rows M .. Mp-1 write zero pieces. Every CTA
-// of a row finds the row's largest |x| itself, so the chunks need no ordering among them.
+// Grid (Mp, n_mats): one CTA per row of one matrix; rows M .. Mp-1 write zero pieces.
 __global__ void __launch_bounds__(XS_THREADS) x_split_kernel(const __grid_constant__ XSplitParams p) {
     __shared__ float red[XS_THREADS / 32];
     __shared__ int bad_sh;
-    const XSplitMat& m = p.mats ? p.mats[__ldg(p.chunk_mat + blockIdx.y)] : p.one;
+    const XSplitMat& m = p.mats ? p.mats[blockIdx.y] : p.one;
     const int row = blockIdx.x;
-    const int chunk = (int)blockIdx.y - m.chunk0;
     const int K = m.K;
     const int M = p.M, Mp = p.Mp;
     const bool pad_row = row >= M;
@@ -178,12 +172,11 @@ __global__ void __launch_bounds__(XS_THREADS) x_split_kernel(const __grid_consta
         frexpf(r, &fe);                         // r in [2^(fe-1), 2^fe)
         e = 8 - fe;
     }
-    if (threadIdx.x == 0 && !pad_row && chunk == 0) factor[row] = bad_row ? __int_as_float(0x7FC00000) : ldexpf(1.0f, -e);
+    if (threadIdx.x == 0 && !pad_row) factor[row] = bad_row ? __int_as_float(0x7FC00000) : ldexpf(1.0f, -e);
     // exact scaling by 2^e in two steps (each factor a normal power of two)
     const float p1 = ldexpf(1.0f, e / 2), p2 = ldexpf(1.0f, e - e / 2);
-    // 2. four pieces per 16-k block, one thread per block of this chunk
-    const int b = chunk * XS_CHUNK_BLOCKS + (int)threadIdx.x;
-    if (b < K / 16) {
+    // 2. four pieces per 16-k block, one thread per block
+    for (int b = threadIdx.x; b < K / 16; b += XS_THREADS) {
         const int kt = b >> 4, bt = b & 15;       // k-tile, block within it
         const size_t j0 = ((size_t)kt * Mp + (size_t)row) * TC_PIECES;   // line of piece 0
         // piece p is line j0 + p; its 16-byte chunk bt/2 sits at chunk (bt/2) ^ ((j0 + p) & 7)
@@ -196,7 +189,7 @@ __global__ void __launch_bounds__(XS_THREADS) x_split_kernel(const __grid_consta
                 *reinterpret_cast<uint2*>(cline + pc * 128 + ((chunk ^ ((ph0 + pc) & 7u)) << 4)) = make_uint2(0u, 0u);
                 sdst[pc * 16] = 0;
             }
-            return;
+            continue;
         }
         // u: the block's residual, always in piece-0 units (x * 2^e)
         float u[16];
