@@ -404,6 +404,40 @@ def test_stack_matches_oracle_and_single_calls(M, path):
     assert torch.equal(gemm_on(path, x, c, s, g), y)
 
 
+def test_large_stack_schedule_matches_oracle_and_repeats():
+    # enough n-tiles (more than 4 per SM) that the block-scaled schedule deals whole n-tiles
+    # round-robin before its stream-K tail, with several K and a ragged last n-tile; results
+    # must match the oracle and be bit-identical from run to run
+    M = 24
+    units = 4 * tl.num_sms(0) + 40
+    Ks = [256, 512, 768, 512]
+    per = (units + len(Ks) - 1) // len(Ks)
+    ents, refs = [], []
+    for j, K in enumerate(Ks):
+        N = per * 128 - (37 if j == 1 else 0)   # one ragged last n-tile
+        _, codes, scales, g = make_weight(N, K, 21, 200 + j)
+        x = synth.x_bf16(M, K, seed=21, tensor_id=synth.X_ID_BASE + 200 + j)
+        ents.append((dev_u8(codes), dev_u8(scales), g, dev_bf16(x), torch.empty((M, N), dtype=torch.bfloat16, device=DEV)))
+        refs.append((codes, scales, g, x))
+    mats = tl.make_matrices(ents)
+    with tl.gemm_path(tl.PATH_BLOCK_SCALED):
+        tl.verify_stack(mats, M)
+        torch.cuda.synchronize()
+        first = [e[4].clone() for e in ents]
+        for _ in range(3):
+            tl.verify_stack(mats, M)
+            for e, y0 in zip(ents, first):
+                assert torch.equal(e[4], y0)
+    tl.check_device_error()
+    rng = np.random.default_rng(21)
+    for (c, s, g, x, y), (codes, scales, gg, xb) in zip(ents, refs):
+        N = y.shape[1]
+        mi = rng.integers(0, M, 3000)
+        ni = np.concatenate([rng.integers(0, N, 2900), np.arange(N - 100, N)])
+        y_ref, a_ref = oracle.gemm_sampled(xb, codes, scales, gg, mi, ni)
+        assert_within_tol(host_f64(y)[mi, ni], y_ref, a_ref, "large stack")
+
+
 @pytest.mark.parametrize("path", list(TC_PATHS))
 def test_plan_matches_stack(path):
     M = 24
