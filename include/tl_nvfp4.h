@@ -30,9 +30,11 @@
  * stream) and do not synchronise, unless stated. The library keeps one small
  * per-device state (split-K workspace, error word, descriptor cache) created
  * by tl_init() or lazily by the first call on a device; call tl_init() before
- * capturing a stream into a CUDA graph. Entry points are thread-safe for
- * distinct streams; calls on one stream must not be interleaved from several
- * host threads without external ordering.
+ * capturing a stream into a CUDA graph. The host side of every entry point is
+ * thread-safe. On the GPU, launches of one device share its workspace (split-K
+ * partials and counters, the X pieces of calls made without a plan): calls whose
+ * kernels could overlap (different streams, or host threads without ordering)
+ * must be serialised by the caller, e.g. by issuing them on one stream.
  *
  * Errors. Every entry point validates its arguments first: on a violation it
  * launches nothing and returns a status; tl_last_error_message() then holds a
