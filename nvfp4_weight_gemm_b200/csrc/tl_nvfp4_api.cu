@@ -16,6 +16,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <queue>
 #include <vector>
 
 #include "gemm_simt.cuh"
@@ -393,10 +394,11 @@ tl_status build_bs_mat(tl::BsMat* m, tl::XSplitMat* xm, const void* x, int M, co
     return TL_OK;
 }
 
-// Each CTA's list of segments (gemm_bs.cuh): whole n-tiles dealt round-robin first, so that
-// the CTAs move through the matrices side by side and share the X pieces in L2; the last two
-// to three rounds' worth of n-tiles are cut into equal shares of k-tiles (stream-K), so every
-// CTA ends with the same number of k-tiles. Depends only on the shapes and the grid.
+// Each CTA's list of segments (gemm_bs.cuh): whole n-tiles dealt in order, each to the CTA with
+// the fewest k-tiles so far (round-robin when the n-tiles are alike), so that the CTAs move
+// through the matrices side by side and share the X pieces in L2; the last two to three rounds'
+// worth of n-tiles are cut into equal shares of k-tiles (stream-K), so every CTA ends with the
+// same number of k-tiles. Depends only on the shapes and the grid.
 struct BsSchedule {
     std::vector<tl::BsSeg> segs;
     std::vector<int> begin;   // [grid + 1]
@@ -412,7 +414,13 @@ void build_schedule(const tl_nvfp4_matrix* mats, int n_mats, int grid, BsSchedul
         for (int j = 0; j < nt; ++j) units.push_back({i, j, kt});
     }
     const long long U = (long long)units.size(), G = grid;
-    const long long R = std::max(0LL, U / G - 2) * G;          // n-tiles dealt whole
+    // n-tiles dealt whole: all but a tail of at least two per CTA and at least two of the
+    // largest n-tiles' k-tiles per CTA, enough to even out the dealt part
+    int max_kt = 1;
+    for (const Unit& un : units) max_kt = std::max(max_kt, un.kt);
+    long long R = std::max(0LL, U - 2 * G), tail = 0;
+    for (long long u = U - 1; u >= R; --u) tail += units[u].kt;
+    while (R > 0 && tail < 2 * G * max_kt) tail += units[--R].kt;
     std::vector<std::vector<tl::BsSeg>> per(grid);
     std::vector<long long> load(grid, 0);
     auto seg = [](const Unit& u, int k0, int k1) {
@@ -427,9 +435,17 @@ void build_schedule(const tl_nvfp4_matrix* mats, int n_mats, int grid, BsSchedul
         sg.parts = 1;
         return sg;
     };
+    // deal each whole n-tile, in order, to the CTA with the fewest k-tiles so far (the one that
+    // will be free first; ties to the lowest index): round-robin when the n-tiles are alike
+    std::priority_queue<std::pair<long long, int>, std::vector<std::pair<long long, int>>,
+                        std::greater<std::pair<long long, int>>> freeq;
+    for (int c = 0; c < grid; ++c) freeq.push({0LL, c});
     for (long long u = 0; u < R; ++u) {
-        per[u % G].push_back(seg(units[u], 0, units[u].kt));
-        load[u % G] += units[u].kt;
+        const int c = freeq.top().second;
+        freeq.pop();
+        per[c].push_back(seg(units[u], 0, units[u].kt));
+        load[c] += units[u].kt;
+        freeq.push({load[c], c});
     }
     long long total = 0, rest = 0;
     for (long long c = 0; c < G; ++c) total += load[c];

@@ -1,0 +1,110 @@
+// Host-only check of the block-scaled GEMM's work schedule (build_schedule in tl_nvfp4_api.cu):
+// every k-tile of every n-tile is covered exactly once, split n-tiles carry consistent ranks,
+// part counts, consecutive partial slots and k order, the workspace limits hold, and the
+// k-tiles per CTA are balanced. Built and run by tests/test_schedule.py; no GPU is touched.
+#include "../nvfp4_weight_gemm_b200/csrc/tl_nvfp4_api.cu"
+
+#include <algorithm>
+#include <cstdio>
+#include <map>
+#include <set>
+#include <utility>
+#include <vector>
+
+static int check(const std::vector<std::pair<int, int>>& shapes, int grid, double min_eff, bool verbose) {
+    std::vector<tl_nvfp4_matrix> mats;
+    for (auto& sh : shapes) {
+        tl_nvfp4_matrix m{};
+        m.N = sh.first;
+        m.K = sh.second;
+        mats.push_back(m);
+    }
+    BsSchedule sc;
+    build_schedule(mats.data(), (int)mats.size(), grid, &sc);
+    int bad = 0;
+    if ((int)sc.begin.size() != grid + 1 || sc.begin[0] != 0 || sc.begin[grid] != (int)sc.segs.size()) {
+        printf("per-CTA offsets malformed\n");
+        return 1;
+    }
+    std::map<std::pair<int, int>, std::vector<std::pair<int, int>>> cov;
+    std::map<int, std::vector<tl::BsSeg>> splits;
+    std::vector<long long> load(grid, 0);
+    for (int c = 0; c < grid; ++c) {
+        for (int i = sc.begin[c]; i < sc.begin[c + 1]; ++i) {
+            const tl::BsSeg& g = sc.segs[i];
+            cov[{g.mat, g.ntile}].push_back({g.k0, g.k1});
+            load[c] += g.k1 - g.k0;
+            if (g.k1 <= g.k0) { ++bad; printf("empty segment\n"); }
+            if (g.split >= 0) splits[g.split].push_back(g);
+            else if (g.k0 != 0 || g.k1 != mats[g.mat].K / 256) { ++bad; printf("whole segment is not whole\n"); }
+        }
+    }
+    long long total = 0;
+    for (size_t i = 0; i < mats.size(); ++i) {
+        const int nt = (mats[i].N + 127) / 128, kt = mats[i].K / 256;
+        total += (long long)nt * kt;
+        for (int j = 0; j < nt; ++j) {
+            auto v = cov[{(int)i, j}];
+            std::sort(v.begin(), v.end());
+            int k = 0;
+            for (auto& r : v) {
+                if (r.first != k) ++bad;
+                k = r.second;
+            }
+            if (k != kt) { ++bad; printf("coverage: matrix %zu n-tile %d\n", i, j); }
+        }
+    }
+    std::set<int> slots;
+    for (auto& kv : splits) {
+        auto& v = kv.second;
+        std::sort(v.begin(), v.end(), [](const tl::BsSeg& a, const tl::BsSeg& b) { return a.rank < b.rank; });
+        for (size_t r = 0; r < v.size(); ++r) {
+            if (v[r].rank != r || v[r].parts != v.size() || v[r].slot - v[r].rank != v[0].slot) {
+                ++bad;
+                printf("split bookkeeping\n");
+            }
+            if (r && v[r].k0 != v[r - 1].k1) { ++bad; printf("split parts out of k order\n"); }
+            if (!slots.insert(v[r].slot).second) { ++bad; printf("partial slot used twice\n"); }
+        }
+    }
+    if (sc.slots > 2 * grid || sc.splits > grid) { ++bad; printf("workspace limits exceeded\n"); }
+    const long long mx = *std::max_element(load.begin(), load.end());
+    const double eff = (double)total / grid / (double)mx;
+    const long long ideal = (total + grid - 1) / grid;
+    if (mx > ideal) { ++bad; printf("a CTA has %lld k-tiles, more than ceil(total / grid) = %lld\n", mx, ideal); }
+    if (eff < min_eff) { ++bad; printf("balance %.4f below %.4f\n", eff, min_eff); }
+    if (verbose || bad)
+        printf("%zu matrices, grid %d: %lld k-tiles, largest CTA share %lld (balance %.4f), %zu segments, "
+               "%d splits, %d slots, bad %d\n",
+               mats.size(), grid, total, mx, eff, sc.segs.size(), sc.splits, sc.slots, bad);
+    return bad;
+}
+
+int main() {
+    int bad = 0;
+    std::vector<std::pair<int, int>> stack;
+    for (int l = 0; l < 64; ++l) {
+        stack.push_back({7168, 5120});
+        stack.push_back({5120, 5120});
+        stack.push_back({34816, 5120});
+        stack.push_back({5120, 17408});
+    }
+    bad += check(stack, 148, 0.999, true);           // the 64-layer stack
+    bad += check({{5120, 5120}}, 148, 0.0, true);      // single matrices: one k-tile short at most
+    bad += check({{34816, 5120}}, 148, 0.0, true);
+    bad += check({{5120, 17408}}, 148, 0.0, true);
+    bad += check({{677, 2304}}, 54, 0.0, true);
+    bad += check({{256, 512}}, 4, 0.0, true);
+    srand(7);
+    for (int it = 0; it < 300; ++it) {
+        std::vector<std::pair<int, int>> sh;
+        const int n = 1 + rand() % 40;
+        for (int i = 0; i < n; ++i) sh.push_back({1 + rand() % 20000, 256 * (1 + rand() % 80)});
+        long long tiles = 0;
+        for (auto& s2 : sh) tiles += (long long)((s2.first + 127) / 128) * (s2.second / 256);
+        const int grid = (int)std::min<long long>(tiles, 1 + rand() % 160);
+        bad += check(sh, grid, 0.0, false);
+    }
+    printf("bad=%d\n", bad);
+    return bad != 0;
+}
