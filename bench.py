@@ -200,6 +200,23 @@ def run_reference(args):
     return 0
 
 
+# --------------------------------------------------------------------------- replicas
+
+def max_over_ranks(values, device, world):
+    """Element-wise maximum of per-rank timings over all ranks (every rank must call it)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_gbs(world, bytes_per_rank, ms):
+    """Whole-job GB/s of `world` replicas: every rank's bytes over the slowest rank's time."""
+    return world * bytes_per_rank / (ms * 1e-3) / 1e9
+
+
 # --------------------------------------------------------------------------- GPU arm
 
 def build_stack(dev, seed=0):
@@ -357,14 +374,11 @@ def main_gpu(args):
     tl.check_device_error(stream)
 
     # ---- reduce over ranks: max time, summed bytes
-    stats = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(stats, op=dist.ReduceOp.MAX)
-    total_ms, e2e_ms = stats.tolist()
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev, world)
 
     if rank == 0:
         peak, peak_kind = load_peaks()
-        value = world * bytes_step * args.steps / (total_ms * 1e-3) / 1e9
+        value = job_gbs(world, bytes_step * args.steps, total_ms)
         achieved = bytes_step * args.steps / (launch_ms_sum * 1e-3) / 1e9
         # per launch, like `achieved`: DRAM bytes of the mean stack pass
         traffic = profiled_traffic(shapes, args.path)
@@ -390,7 +404,7 @@ def main_gpu(args):
             "m_invariance_row_fraction": inv,
             "cpu_baseline": {"value": round(cb / cs / 1e9, 4), "unit": "GB/s", "cores": cthreads, "kind": "oracle",
                              "sample": CPU_SAMPLE_DESC},
-            "e2e": {"value": round(world * bytes_step / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+            "e2e": {"value": round(job_gbs(world, bytes_step, e2e_ms), 1), "unit": "GB/s",
                     "h2d_bytes_per_step": e2e_h2d, "d2h_bytes_per_step": e2e_d2h},
             "gpu_launches": n_launch * launches_per_pass,
             "clocks": clocks,
