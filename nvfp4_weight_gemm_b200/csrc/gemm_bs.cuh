@@ -89,27 +89,31 @@ struct BsParams {
     BsMat one;
 };
 
+// NX: the X rows a launch can hold (4, 8, 16, 24 or 32; the smallest >= Mp is used). Fewer X rows
+// leave room for more stages, and the ring's depth is what keeps enough weight bytes in flight.
 template <int NX>
 struct BsCfg {
     static constexpr int CODES_BYTES = TC_BLOCK_N * (TC_BLOCK_K / 2);        // 16384
-    static constexpr int XC_BYTES = TC_PIECES * NX * (TC_BLOCK_K / 2);       // 8192 / 16384
+    static constexpr int XC_BYTES = TC_PIECES * NX * (TC_BLOCK_K / 2);       // 2048 .. 16384
     static constexpr int SCALES_BYTES = TC_BLOCK_N * (TC_BLOCK_K / 16);      // 2048
-    static constexpr int XS_BYTES = TC_PIECES * NX * (TC_BLOCK_K / 16);      // 1024 / 2048
+    static constexpr int XS_BYTES = TC_PIECES * NX * (TC_BLOCK_K / 16);      // 256 .. 2048
     static constexpr int SC_OFF = CODES_BYTES;
     static constexpr int XC_OFF = SC_OFF + SCALES_BYTES;                     // 18432: 1024-byte aligned
     static constexpr int XS_OFF = XC_OFF + XC_BYTES;                         // X codes and scales adjoin
-    static constexpr int STAGE_BYTES = XS_OFF + XS_BYTES;                    // 27648 / 36864
-    static constexpr int STAGES = (NX == 32) ? 6 : 8;
+    static constexpr int STAGE_BYTES = (XS_OFF + XS_BYTES + 1023) / 1024 * 1024;
+    static constexpr int STAGES = (232448 - 1024 - 512) / STAGE_BYTES;       // 10, 9, 8, 7, 6
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 512 /*barriers*/;
-    static constexpr int N_MMA = TC_PIECES * NX;                             // largest N: 64 / 128
+    static constexpr int N_MMA = TC_PIECES * NX;                             // largest N: 16 .. 128
     static constexpr int ACC_BUFS = 2;
-    static constexpr int SF_COL0 = 256;
+    static constexpr int SF_COL0 = ACC_BUFS * N_MMA;                         // scale columns after the accumulators
     // E2M1 x E2M1, UE4M3 scales, M = 128; N (bits 17..22, N / 8) is added at run time
     static constexpr uint32_t IDESC_BASE = (1u << 7) | (1u << 10) | (0u << 23) | ((uint32_t)(TC_BLOCK_N >> 4) << 24);
     static_assert(STAGE_BYTES % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
     static_assert(XC_OFF % 1024 == 0, "X piece codes must start on a swizzle atom");
     static_assert(ACC_BUFS * N_MMA <= SF_COL0, "accumulators must fit below the scale columns");
     static_assert(SF_COL0 + STAGES * BS_SF_COLS <= TC_TMEM_COLS, "tensor memory budget");
+    static_assert(STAGES <= 32, "stage masks are 32 bits");
+    static_assert(NX % 4 == 0 && N_MMA % 16 == 0, "MMA N must be a multiple of 16");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 

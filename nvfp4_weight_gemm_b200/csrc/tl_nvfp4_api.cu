@@ -562,7 +562,11 @@ tl_status launch_bs_gemm(DevState& d, tl::BsParams& p, int grid, cudaStream_t st
 tl_status launch_bs(DevState& d, tl::BsParams bp, const tl::XSplitParams& xp, int grid, cudaStream_t stream) {
     tl::x_split_kernel<<<dim3((unsigned)xp.Mp, (unsigned)xp.n_mats), tl::XS_THREADS, 0, stream>>>(xp);
     TL_CUDA(cudaGetLastError());
-    return (bp.M <= 16) ? launch_bs_gemm<16>(d, bp, grid, stream) : launch_bs_gemm<32>(d, bp, grid, stream);
+    if (bp.Mp <= 4) return launch_bs_gemm<4>(d, bp, grid, stream);
+    if (bp.Mp <= 8) return launch_bs_gemm<8>(d, bp, grid, stream);
+    if (bp.Mp <= 16) return launch_bs_gemm<16>(d, bp, grid, stream);
+    if (bp.Mp <= 24) return launch_bs_gemm<24>(d, bp, grid, stream);
+    return launch_bs_gemm<32>(d, bp, grid, stream);
 }
 
 // The schedule as one device blob: segments, then the per-CTA offsets.
