@@ -7,7 +7,7 @@
  * weight once (TandemLLM docs v0.12.0, "What TandemLLM is", section 1.2; the
  * StairCut research page, "What it says"). Each projection of that pass is
  *
- *     Y[M,N] = X[M,K] . dequant(W)[N,K]^T,      1 <= M <= 32,
+ *     Y[M,N] = X[M,K] . dequant(W)[N,K]^T,      1 <= M <= 32 (up to 128 served),
  *
  * with W stored as NVFP4: four bits a weight and one scale per 16 weights
  * (same page, section 1.2). At the bit level:
@@ -55,7 +55,7 @@ typedef enum {
     TL_OK = 0,
     TL_ERR_INVALID_VALUE = 1,   /* a size or pointer argument is out of range */
     TL_ERR_MISALIGNED = 2,      /* a pointer is not 16-byte aligned */
-    TL_ERR_UNSUPPORTED = 3,     /* valid request this build does not serve (e.g. M > 32) */
+    TL_ERR_UNSUPPORTED = 3,     /* valid request this build does not serve (e.g. M > 128) */
     TL_ERR_CUDA = 4,            /* a CUDA runtime/driver call failed */
     TL_ERR_TIMEOUT = 5,         /* a device-side wait ran past its iteration limit */
     TL_ERR_NOT_INITIALIZED = 6, /* no usable device / state */
@@ -63,8 +63,11 @@ typedef enum {
     TL_ERR_DEVICE_FAULT = 8     /* the device status word holds an internal error */
 } tl_status;
 
-/* Largest number of draft-tree rows one call serves. */
-#define TL_NVFP4_MAX_M 32
+/* Largest number of X rows one call serves. One launch serves up to 64 rows on the
+ * block-scaled path and 32 on the exact and CUDA-core paths; a call with more rows runs as
+ * groups of rows, each streaming the weights again. Plans take at most one launch's rows;
+ * tl_nvfp4_verify_gemm_noalloc() takes at most 32. */
+#define TL_NVFP4_MAX_M 128
 /* K must be a positive multiple of this. */
 #define TL_NVFP4_K_ALIGN 256
 /* Largest number of matrices one tl_nvfp4_verify_stack() call takes. */
@@ -113,7 +116,7 @@ void tl_shutdown(void);
 
 /* Y = X . dequant(W)^T for one weight matrix (see the top of this file).
  *   x      device bf16 [M][K], 16-byte aligned
- *   M      0..32 (0 is a no-op returning TL_OK; > 32 returns TL_ERR_UNSUPPORTED)
+ *   M      0..TL_NVFP4_MAX_M (0 is a no-op returning TL_OK; more returns TL_ERR_UNSUPPORTED)
  *   w_codes, w_scales  device, 16-byte aligned, layouts above
  *   global_scale       finite
  *   y      device bf16 [M][N], 16-byte aligned; must not overlap x or W

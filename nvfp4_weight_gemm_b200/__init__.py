@@ -1,4 +1,4 @@
-"""NVFP4 verify GEMM for B200: Y[M,N] = X[M,K] . dequant(W)[N,K]^T, M <= 32.
+"""NVFP4 verify GEMM for B200: Y[M,N] = X[M,K] . dequant(W)[N,K]^T, M <= 128.
 
 Thin Python layer over libtl_nvfp4.so (the C ABI in include/tl_nvfp4.h). Torch tensors
 are used for device memory and streams only; every step of the computation runs in the

@@ -52,7 +52,7 @@
 namespace tl {
 
 constexpr int BS_THREADS = 384;   // 12 warps
-constexpr int BS_SF_COLS = 32;    // tensor-memory columns of scales per stage (16 for W, 16 for X)
+constexpr int BS_PART_ROWS = 64;  // X rows of one split-K partial slot ([64][128] fp32)
 
 struct alignas(64) BsMat {
     CUtensorMap tm_codes;   // uint8 {K/2, N, 1}, box 128 B x 128 rows x 1, 128-byte swizzle
@@ -89,8 +89,10 @@ struct BsParams {
     BsMat one;
 };
 
-// NX: the X rows a launch can hold (4, 8, 16, 24 or 32; the smallest >= Mp is used). Fewer X rows
-// leave room for more stages, and the ring's depth is what keeps enough weight bytes in flight.
+// NX: the X rows a launch can hold (4, 8, 16, 24, 32 or 64; the smallest >= Mp is used). Fewer X
+// rows leave room for more stages, and the ring's depth is what keeps enough weight bytes in
+// flight. Above 32 rows the X lines are two MMA operands of up to 128 lines each (the MMA shape
+// and scale layout used at every size), with one accumulator buffer.
 template <int NX>
 struct BsCfg {
     static constexpr int CODES_BYTES = TC_BLOCK_N * (TC_BLOCK_K / 2);        // 16384
@@ -103,15 +105,20 @@ struct BsCfg {
     static constexpr int STAGE_BYTES = (XS_OFF + XS_BYTES + 1023) / 1024 * 1024;
     static constexpr int STAGES = (232448 - 1024 - 512) / STAGE_BYTES;       // 10, 9, 8, 7, 6
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 512 /*barriers*/;
-    static constexpr int N_MMA = TC_PIECES * NX;                             // largest N: 16 .. 128
-    static constexpr int ACC_BUFS = 2;
+    static constexpr int N_MMA = TC_PIECES * NX;                             // X lines: 16 .. 256
+    static constexpr int XH = (NX > 32) ? 2 : 1;                             // MMAs per 64-k chunk (128 lines each)
+    static constexpr int ACC_BUFS = (NX > 32) ? 1 : 2;
+    static constexpr int SF_COLS = 16 + 16 * XH;                             // scale columns per stage: W, X halves
     static constexpr int SF_COL0 = ACC_BUFS * N_MMA;                         // scale columns after the accumulators
+    static constexpr int RG = (NX + 31) / 32;                                // epilogue row groups
+    static constexpr int GR = (NX < 32) ? NX : 32;                           // rows per group
     // E2M1 x E2M1, UE4M3 scales, M = 128; N (bits 17..22, N / 8) is added at run time
     static constexpr uint32_t IDESC_BASE = (1u << 7) | (1u << 10) | (0u << 23) | ((uint32_t)(TC_BLOCK_N >> 4) << 24);
     static_assert(STAGE_BYTES % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
     static_assert(XC_OFF % 1024 == 0, "X piece codes must start on a swizzle atom");
     static_assert(ACC_BUFS * N_MMA <= SF_COL0, "accumulators must fit below the scale columns");
-    static_assert(SF_COL0 + STAGES * BS_SF_COLS <= TC_TMEM_COLS, "tensor memory budget");
+    static_assert(SF_COL0 + STAGES * SF_COLS <= TC_TMEM_COLS, "tensor memory budget");
+    static_assert(NX <= BS_PART_ROWS, "partial slots hold 64 rows");
     static_assert(STAGES <= 32, "stage masks are 32 bits");
     static_assert(NX % 4 == 0 && N_MMA % 16 == 0, "MMA N must be a multiple of 16");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -252,7 +259,11 @@ gemm_bs_kernel(const __grid_constant__ BsParams p) {
         uint32_t ph = 0, accph = 0;
         const uint64_t desc_w0 = smem_desc_k_sw128(smem_u32(smem));
         const uint64_t desc_x0 = smem_desc_k_sw128(smem_u32(smem + C::XC_OFF));
-        const uint32_t idesc = C::IDESC_BASE | ((uint32_t)(TC_PIECES * p.Mp) >> 3) << 17;
+        // X lines 0..127 and 128..4 Mp - 1 (above 32 rows) are two MMAs into accumulator columns
+        // 0..127 and 128..
+        const uint32_t lines = (uint32_t)(TC_PIECES * p.Mp);
+        const uint32_t idesc = C::IDESC_BASE | ((lines < 128u ? lines : 128u) >> 3) << 17;
+        const uint32_t idesc_hi = C::IDESC_BASE | ((lines > 128u ? lines - 128u : 16u) >> 3) << 17;
         bool ok = true;
         for (int si = s_begin; ok && si < s_end; ++si) {
             const BsSeg sg = p.segs[si];
@@ -273,12 +284,17 @@ gemm_bs_kernel(const __grid_constant__ BsParams p) {
                 }
                 tc_fence_after();
                 const uint64_t sdesc = (uint64_t)((s * C::STAGE_BYTES) >> 4);
-                const uint32_t sf = tmem + (uint32_t)(C::SF_COL0 + BS_SF_COLS * s);
+                const uint32_t sf = tmem + (uint32_t)(C::SF_COL0 + C::SF_COLS * s);
                 if (leader) {
 #pragma unroll
-                    for (int kc = 0; kc < 4; ++kc)
+                    for (int kc = 0; kc < 4; ++kc) {
                         mma_bs_f4(d_tmem, desc_w0 + sdesc + (uint64_t)(2 * kc), desc_x0 + sdesc + (uint64_t)(2 * kc),
                                   idesc, sf + 4u * kc, sf + 16u + 4u * kc, (kc == 0) ? (first ^ 1u) : 1u);
+                        if (C::XH > 1 && lines > 128u)
+                            mma_bs_f4(d_tmem + 128u, desc_w0 + sdesc + (uint64_t)(2 * kc),
+                                      desc_x0 + sdesc + (uint64_t)((128 * 128) >> 4) + (uint64_t)(2 * kc), idesc_hi,
+                                      sf + 4u * kc, sf + 32u + 4u * kc, (kc == 0) ? (first ^ 1u) : 1u);
+                    }
                     mma_commit(&empty[s]);
                 }
                 __syncwarp();
@@ -310,13 +326,10 @@ gemm_bs_kernel(const __grid_constant__ BsParams p) {
                 break;
             }
             uint8_t* st = smem + s * C::STAGE_BYTES;
-            uint4 wa[4], wb[4];
+            uint4 wa[4];
 #pragma unroll
-            for (int gq = 0; gq < 4; ++gq) {
-                const int r = lane + 32 * gq;
-                wa[gq] = *reinterpret_cast<const uint4*>(st + C::SC_OFF + 16 * r);
-                wb[gq] = (r < C::N_MMA) ? *reinterpret_cast<const uint4*>(st + C::XS_OFF + 16 * r) : make_uint4(0, 0, 0, 0);
-            }
+            for (int gq = 0; gq < 4; ++gq)
+                wa[gq] = *reinterpret_cast<const uint4*>(st + C::SC_OFF + 16 * (lane + 32 * gq));
             // a scale byte with the sign bit set: negate that block's codes, keep |scale|
             uint32_t neg = 0;
 #pragma unroll
@@ -345,15 +358,25 @@ gemm_bs_kernel(const __grid_constant__ BsParams p) {
                 }
             }
             // column 4c + gq: scale word c (four 16-k blocks of chunk c) of row lane + 32 gq
-            uint32_t ca[16], cb[16];
+            uint32_t ca[16];
 #pragma unroll
             for (int gq = 0; gq < 4; ++gq) {
                 ca[0 + gq] = wa[gq].x; ca[4 + gq] = wa[gq].y; ca[8 + gq] = wa[gq].z; ca[12 + gq] = wa[gq].w;
-                cb[0 + gq] = wb[gq].x; cb[4 + gq] = wb[gq].y; cb[8 + gq] = wb[gq].z; cb[12 + gq] = wb[gq].w;
             }
-            const uint32_t col = t_lane + (uint32_t)(C::SF_COL0 + BS_SF_COLS * s);
+            const uint32_t col = t_lane + (uint32_t)(C::SF_COL0 + C::SF_COLS * s);
             tmem_st16(col, ca);
-            tmem_st16(col + 16u, cb);
+#pragma unroll
+            for (int h = 0; h < C::XH; ++h) {
+                uint32_t cb[16];
+#pragma unroll
+                for (int gq = 0; gq < 4; ++gq) {
+                    const int rx = 128 * h + lane + 32 * gq;   // X line
+                    const uint4 wb = (rx < C::N_MMA) ? *reinterpret_cast<const uint4*>(st + C::XS_OFF + 16 * rx)
+                                                     : make_uint4(0, 0, 0, 0);
+                    cb[0 + gq] = wb.x; cb[4 + gq] = wb.y; cb[8 + gq] = wb.z; cb[12 + gq] = wb.w;
+                }
+                tmem_st16(col + 16u + 16u * h, cb);
+            }
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -382,41 +405,50 @@ gemm_bs_kernel(const __grid_constant__ BsParams p) {
             }
             tc_fence_after();
             const int n = sg.ntile * TC_BLOCK_N + r;
-            // sum the pieces in order: v[m] = sum_p 4^-p D[4 m + p] (exact scalings); 16 columns
-            // hold rows 4c .. 4c+3
-            float v[NX];
+            const uint32_t acc_col = (uint32_t)(C::N_MMA * acc);
+            float* part = p.partials + (size_t)sg.slot * (BS_PART_ROWS * TC_BLOCK_N);   // split only
+            // Rows in groups of up to 32 (registers): sum the pieces in order,
+            // v[m] = sum_p 4^-p D[4 m + p] (exact scalings), 16 columns holding rows 4c .. 4c+3;
+            // the accumulator is handed back after the last group's reads.
+#pragma unroll 1
+            for (int g = 0; g < C::RG; ++g) {
+                float v[C::GR];
 #pragma unroll
-            for (int c = 0; c < NX / 4; ++c) {
-                if (4 * c < M) {
-                    uint32_t raw[16];
-                    tmem_ld16(t_lane + (uint32_t)(C::N_MMA * acc + 16 * c), raw);
-                    tmem_wait_ld();
+                for (int c = 0; c < C::GR / 4; ++c) {
+                    if (32 * g + 4 * c < M) {
+                        uint32_t raw[16];
+                        tmem_ld16(t_lane + acc_col + (uint32_t)(16 * (8 * g + c)), raw);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        float a = __uint_as_float(raw[4 * j]);
-                        a = fmaf(__uint_as_float(raw[4 * j + 1]), 0.25f, a);
-                        a = fmaf(__uint_as_float(raw[4 * j + 2]), 0.0625f, a);
-                        v[4 * c + j] = fmaf(__uint_as_float(raw[4 * j + 3]), 0.015625f, a);
+                        for (int j = 0; j < 4; ++j) {
+                            float a = __uint_as_float(raw[4 * j]);
+                            a = fmaf(__uint_as_float(raw[4 * j + 1]), 0.25f, a);
+                            a = fmaf(__uint_as_float(raw[4 * j + 2]), 0.0625f, a);
+                            v[4 * c + j] = fmaf(__uint_as_float(raw[4 * j + 3]), 0.015625f, a);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) v[4 * c + j] = 0.0f;
                     }
+                }
+                if (g == C::RG - 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&accempty[acc]);
+                    if (++acc == C::ACC_BUFS) { acc = 0; accph ^= 1u; }
+                }
+                const int mg = M - 32 * g;                  // rows of this group that exist
+                if (sg.split < 0) {
+                    if (n < N && mg > 0) bs_store_rows<C::GR>(v, mg, gm, xf + 32 * g, yp + (long long)(32 * g) * N + n, N);
                 } else {
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) v[4 * c + j] = 0.0f;
+                    for (int i = 0; i < C::GR; ++i)
+                        if (i < mg) part[(32 * g + i) * TC_BLOCK_N + r] = v[i];
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&accempty[acc]);
-            if (++acc == C::ACC_BUFS) { acc = 0; accph ^= 1u; }
-            if (sg.split < 0) {
-                if (n < N) bs_store_rows<NX>(v, M, gm, xf, yp + n, N);
-                continue;
-            }
-            // a split n-tile: write this part; the last part to arrive (per 32-row quarter)
-            // adds all parts in k order and writes Y
-            float* mine = p.partials + (size_t)sg.slot * (32 * TC_BLOCK_N);
-#pragma unroll
-            for (int i = 0; i < NX; ++i)
-                if (i < M) mine[i * TC_BLOCK_N + r] = v[i];
+            if (sg.split < 0) continue;
+            // a split n-tile: the last part to arrive (per 32-row quarter of weight rows) adds all
+            // parts in k order and writes Y
             __threadfence();
             __syncwarp();
             unsigned old = 0;
@@ -424,16 +456,21 @@ gemm_bs_kernel(const __grid_constant__ BsParams p) {
             old = __shfl_sync(0xFFFFFFFFu, old, 0);
             if (old == (unsigned)(sg.parts - 1)) {
                 __threadfence();
+                const float* part0 = p.partials + (size_t)(sg.slot - sg.rank) * (BS_PART_ROWS * TC_BLOCK_N);
+#pragma unroll 1
+                for (int g = 0; g < C::RG; ++g) {
+                    const int mg = M - 32 * g;
+                    float v[C::GR];
 #pragma unroll
-                for (int i = 0; i < NX; ++i) v[i] = 0.0f;
-                const float* part0 = p.partials + (size_t)(sg.slot - sg.rank) * (32 * TC_BLOCK_N);
-                for (int rk = 0; rk < sg.parts; ++rk) {
-                    const float* part = part0 + (size_t)rk * (32 * TC_BLOCK_N);
+                    for (int i = 0; i < C::GR; ++i) v[i] = 0.0f;
+                    for (int rk = 0; rk < sg.parts; ++rk) {
+                        const float* pp = part0 + (size_t)rk * (BS_PART_ROWS * TC_BLOCK_N);
 #pragma unroll
-                    for (int i = 0; i < NX; ++i)
-                        if (i < M) v[i] += __ldcg(&part[i * TC_BLOCK_N + r]);
+                        for (int i = 0; i < C::GR; ++i)
+                            if (i < mg) v[i] += __ldcg(&pp[(32 * g + i) * TC_BLOCK_N + r]);
+                    }
+                    if (n < N && mg > 0) bs_store_rows<C::GR>(v, mg, gm, xf + 32 * g, yp + (long long)(32 * g) * N + n, N);
                 }
-                if (n < N) bs_store_rows<NX>(v, M, gm, xf, yp + n, N);
                 if (lane == 0) p.counters[4 * sg.split + q] = 0u;   // ready for the next launch
             }
         }

@@ -57,7 +57,7 @@ struct DevState {
     bool ready = false;
     int num_sms = 0;
     int* err = nullptr;            // device status word
-    float* partials = nullptr;     // [2 * num_sms][32][128]
+    float* partials = nullptr;     // [2 * num_sms][64][128]
     unsigned* counters = nullptr;  // [4 * num_sms]
     unsigned* qscratch = nullptr;  // quantiser absmax + non-finite flag
     bool smem_attr_set = false;
@@ -106,7 +106,7 @@ tl_status init_locked(int device) {
             break;
         }
         d.num_sms = sms;
-        const size_t pbytes = (size_t)2 * sms * 32 * tl::TC_BLOCK_N * sizeof(float);
+        const size_t pbytes = (size_t)2 * sms * tl::BS_PART_ROWS * tl::TC_BLOCK_N * sizeof(float);
         if (cudaMalloc(&d.err, 64) != cudaSuccess || cudaMalloc(&d.partials, pbytes) != cudaSuccess ||
             cudaMalloc(&d.counters, (size_t)4 * sms * sizeof(unsigned)) != cudaSuccess ||
             cudaMalloc(&d.qscratch, 64) != cudaSuccess) {
@@ -225,9 +225,14 @@ tl_status launch_tc_any(DevState& d, tl::TcParams& p, cudaStream_t stream) {
     return (p.M <= 16) ? launch_tc<16>(d, p, stream) : launch_tc<32>(d, p, stream);
 }
 
-tl_status check_M(int M) {
+// Rows one launch serves: the block-scaled GEMM 64, the exact and CUDA-core kernels 32. Calls with
+// more rows (up to TL_NVFP4_MAX_M) run as groups of rows, each streaming the weights again.
+constexpr int kBsMaxRows = 64;
+constexpr int kExactMaxRows = 32;
+
+tl_status check_M(int M, int limit = TL_NVFP4_MAX_M) {
     if (M < 0) return fail(TL_ERR_INVALID_VALUE, "M = %d is negative", M);
-    if (M > TL_NVFP4_MAX_M) return fail(TL_ERR_UNSUPPORTED, "M = %d > %d rows is not served", M, TL_NVFP4_MAX_M);
+    if (M > limit) return fail(TL_ERR_UNSUPPORTED, "M = %d > %d rows is not served here", M, limit);
     return TL_OK;
 }
 
@@ -275,7 +280,7 @@ tl_status stack_table(DevState& d, const std::vector<tl::TcMat>& mats, cudaStrea
 // state lookup). `table_out` receives the TcMat array when n_mats > 1.
 tl_status build_params(const tl_nvfp4_matrix* mats, int n_mats, int M, const unsigned char* x_dev,
                        unsigned char* y_dev, DevState** dstate, tl::TcParams* p, std::vector<tl::TcMat>* table_out) {
-    tl_status st = check_M(M);
+    tl_status st = check_M(M, g_path == TL_PATH_BLOCK_SCALED ? kBsMaxRows : kExactMaxRows);
     if (st != TL_OK) return st;
     if (!mats) return fail(TL_ERR_INVALID_VALUE, "mats is null");
     if (n_mats < 1 || n_mats > TL_NVFP4_MAX_STACK)
@@ -298,6 +303,7 @@ tl_status build_params(const tl_nvfp4_matrix* mats, int n_mats, int M, const uns
     if (M == 0) return TL_OK;
     st = current_state(dstate);
     if (st != TL_OK) return st;
+    if (g_path == TL_PATH_BLOCK_SCALED) return TL_OK;   // the block-scaled launch builds its own tables
     const int NX = M <= 16 ? 16 : 32;
     std::vector<tl::TcMat>& tbl = *table_out;
     tbl.assign(n_mats, tl::TcMat());
@@ -326,8 +332,50 @@ tl_status build_params(const tl_nvfp4_matrix* mats, int n_mats, int M, const uns
 tl_status run_stack_bs(const tl_nvfp4_matrix* mats, int n_mats, int M, const unsigned char* x_dev,
                        unsigned char* y_dev, void* stream_, DevState* d);
 
+tl_status run_stack_rows(const tl_nvfp4_matrix* mats, int n_mats, int M, const unsigned char* x_dev,
+                         unsigned char* y_dev, void* stream_);
+
+// A stack with more rows than one launch serves: validate it whole, then run it as groups of
+// rows (rows r0 .. r0 + Mg - 1 of every X_i and Y_i), each group one launch.
 tl_status run_stack(const tl_nvfp4_matrix* mats, int n_mats, int M, const unsigned char* x_dev,
                     unsigned char* y_dev, void* stream_) {
+    const int lim = (g_path == TL_PATH_BLOCK_SCALED) ? kBsMaxRows : kExactMaxRows;
+    if (M <= lim) return run_stack_rows(mats, n_mats, M, x_dev, y_dev, stream_);
+    tl_status st = check_M(M);
+    if (st != TL_OK) return st;
+    if (!mats) return fail(TL_ERR_INVALID_VALUE, "mats is null");
+    if (n_mats < 1 || n_mats > TL_NVFP4_MAX_STACK)
+        return fail(TL_ERR_INVALID_VALUE, "n_mats = %d outside [1, %d]", n_mats, TL_NVFP4_MAX_STACK);
+    std::vector<tl_nvfp4_matrix> full(mats, mats + n_mats), grp(n_mats);
+    size_t xoff = 0, yoff = 0;
+    for (int i = 0; i < n_mats; ++i) {
+        if (x_dev) full[i].x = x_dev + xoff;
+        if (y_dev) full[i].y = y_dev + yoff;
+        st = check_matrix(full[i].x, M, full[i].w_codes, full[i].w_scales, full[i].global_scale, full[i].y, full[i].N,
+                          full[i].K, true);
+        if (st != TL_OK) {
+            char why[sizeof g_msg];
+            memcpy(why, g_msg, sizeof why);
+            return fail(st, "matrix %d: %s", i, why);
+        }
+        xoff += (size_t)2 * M * mats[i].K;
+        yoff += (size_t)2 * M * mats[i].N;
+    }
+    for (int r0 = 0; r0 < M; r0 += lim) {
+        const int mg = std::min(lim, M - r0);
+        for (int i = 0; i < n_mats; ++i) {
+            grp[i] = full[i];
+            grp[i].x = static_cast<const unsigned char*>(full[i].x) + (size_t)2 * r0 * full[i].K;
+            grp[i].y = static_cast<unsigned char*>(full[i].y) + (size_t)2 * r0 * full[i].N;
+        }
+        st = run_stack_rows(grp.data(), n_mats, mg, nullptr, nullptr, stream_);
+        if (st != TL_OK) return st;
+    }
+    return TL_OK;
+}
+
+tl_status run_stack_rows(const tl_nvfp4_matrix* mats, int n_mats, int M, const unsigned char* x_dev,
+                         unsigned char* y_dev, void* stream_) {
     DevState* d = nullptr;
     tl::TcParams p;
     std::vector<tl::TcMat> tbl;
@@ -566,7 +614,8 @@ tl_status launch_bs(DevState& d, tl::BsParams bp, const tl::XSplitParams& xp, in
     if (bp.Mp <= 8) return launch_bs_gemm<8>(d, bp, grid, stream);
     if (bp.Mp <= 16) return launch_bs_gemm<16>(d, bp, grid, stream);
     if (bp.Mp <= 24) return launch_bs_gemm<24>(d, bp, grid, stream);
-    return launch_bs_gemm<32>(d, bp, grid, stream);
+    if (bp.Mp <= 32) return launch_bs_gemm<32>(d, bp, grid, stream);
+    return launch_bs_gemm<64>(d, bp, grid, stream);
 }
 
 // The schedule as one device blob: segments, then the per-CTA offsets.
@@ -692,7 +741,7 @@ tl_status noalloc_setup(int device, NoAllocDevice** out) {
 
 extern "C" tl_status tl_nvfp4_verify_gemm_noalloc(const void* x, int M, const void* w_codes, const void* w_scales,
                                                   float global_scale, void* y, int N, int K, void* stream) {
-    tl_status st = check_M(M);
+    tl_status st = check_M(M, kExactMaxRows);
     if (st != TL_OK) return st;
     st = check_matrix(x, M, w_codes, w_scales, global_scale, y, N, K, true);
     if (st != TL_OK) return st;
@@ -936,13 +985,18 @@ tl_status tl_nvfp4_verify_gemm_simt(const void* x, int M, const void* w_codes, c
     auto ss = static_cast<const uint8_t*>(w_scales);
     auto ys = static_cast<__nv_bfloat16*>(y);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (M <= 8)
-        tl::gemm_simt_kernel<8><<<grid, tl::SIMT_WARPS * 32, 0, s>>>(xs, M, cs, ss, global_scale, ys, N, K);
-    else if (M <= 16)
-        tl::gemm_simt_kernel<16><<<grid, tl::SIMT_WARPS * 32, 0, s>>>(xs, M, cs, ss, global_scale, ys, N, K);
-    else
-        tl::gemm_simt_kernel<32><<<grid, tl::SIMT_WARPS * 32, 0, s>>>(xs, M, cs, ss, global_scale, ys, N, K);
-    TL_CUDA(cudaGetLastError());
+    for (int r0 = 0; r0 < M; r0 += kExactMaxRows) {   // groups of at most 32 rows
+        const int mg = std::min(kExactMaxRows, M - r0);
+        const __nv_bfloat16* xg = xs + (size_t)r0 * K;
+        __nv_bfloat16* yg = ys + (size_t)r0 * N;
+        if (mg <= 8)
+            tl::gemm_simt_kernel<8><<<grid, tl::SIMT_WARPS * 32, 0, s>>>(xg, mg, cs, ss, global_scale, yg, N, K);
+        else if (mg <= 16)
+            tl::gemm_simt_kernel<16><<<grid, tl::SIMT_WARPS * 32, 0, s>>>(xg, mg, cs, ss, global_scale, yg, N, K);
+        else
+            tl::gemm_simt_kernel<32><<<grid, tl::SIMT_WARPS * 32, 0, s>>>(xg, mg, cs, ss, global_scale, yg, N, K);
+        TL_CUDA(cudaGetLastError());
+    }
     return TL_OK;
 }
 

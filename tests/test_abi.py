@@ -53,7 +53,7 @@ def _gemm(L, x=A, M=8, c=A + 4096, s=A + 8192, g=1.0, y=A + (1 << 16), N=256, K=
 
 
 @pytest.mark.parametrize("kw,status", [
-    (dict(M=33), 3), (dict(M=-1), 1), (dict(K=100), 1), (dict(K=0), 1), (dict(K=128), 1),
+    (dict(M=129), 3), (dict(M=-1), 1), (dict(K=100), 1), (dict(K=0), 1), (dict(K=128), 1),
     (dict(N=0), 1), (dict(c=A + 8), 2), (dict(s=A + 4), 2), (dict(x=A + 2), 2), (dict(y=A + 6), 2),
     (dict(c=0), 1), (dict(g=float("nan")), 1), (dict(g=float("inf")), 1), (dict(y=A), 1),
 ])
@@ -63,7 +63,7 @@ def test_verify_gemm_rejects(L, kw, status):
 
 
 def test_simt_path_validates_the_same_way(L):
-    assert L.tl_nvfp4_verify_gemm_simt(A, 40, A, A, ctypes.c_float(1.0), A, 8, 256, None) == 3
+    assert L.tl_nvfp4_verify_gemm_simt(A, 129, A, A, ctypes.c_float(1.0), A, 8, 256, None) == 3
     assert L.tl_nvfp4_verify_gemm_simt(A, 4, A, A, ctypes.c_float(1.0), A + 1, 8, 256, None) == 2
 
 
@@ -72,7 +72,7 @@ def test_stack_rejects_bad_counts(L):
     arr = (Matrix * 1)()
     assert L.tl_nvfp4_verify_stack(arr, 0, 8, None) == 1
     assert L.tl_nvfp4_verify_stack(arr, 5000, 8, None) == 1
-    assert L.tl_nvfp4_verify_stack(arr, 1, 33, None) == 3
+    assert L.tl_nvfp4_verify_stack(arr, 1, 129, None) == 3
     arr[0] = Matrix(A + 8, A, A, A + (1 << 16), 1.0, 256, 512)
     assert L.tl_nvfp4_verify_stack(arr, 1, 8, None) == 2
 

@@ -186,6 +186,16 @@ def test_ragged_split_k_all_row_counts(M):
     assert_all_within_tol(run_paths(x, codes, scales, g), y_ref, a_ref, f"M={M}")
 
 
+@pytest.mark.parametrize("M", [33, 48, 64, 65, 100, 128])
+def test_more_rows_than_one_launch(M):
+    # above 32 rows: one 64-row launch on the block-scaled path (two 128-line MMAs per chunk),
+    # groups of rows beyond that; groups of 32 rows on the exact and CUDA-core paths
+    _, codes, scales, g = make_weight(677, 2304, 2, 1)
+    x = synth.x_bf16(M, 2304, seed=22, tensor_id=synth.X_ID_BASE + 300 + M)
+    y_ref, a_ref = oracle.gemm(x, codes, scales, g)
+    assert_all_within_tol(run_paths(x, codes, scales, g), y_ref, a_ref, f"M={M}")
+
+
 @pytest.mark.parametrize("path", list(TC_PATHS))
 @pytest.mark.parametrize("M", [1, 8, 16, 24, 32])
 def test_attention_projection_full(M, path):
@@ -356,12 +366,12 @@ def test_repeat_runs_bit_identical(path):
 def test_rows_do_not_depend_on_M(path):
     # row i of a call with M rows equals the same row computed alone, bit for bit
     _, codes, scales, g = make_weight(677, 2304, 2, 1)
-    x = synth.x_bf16(32, 2304, seed=17)
+    x = synth.x_bf16(48, 2304, seed=17)
     c, s = dev_u8(codes), dev_u8(scales)
-    alone = [gemm_on(path, dev_bf16(x[i:i + 1]), c, s, g) for i in (0, 5, 15, 16, 31)]
-    for M in (16, 17, 32):
+    alone = [gemm_on(path, dev_bf16(x[i:i + 1]), c, s, g) for i in (0, 5, 15, 16, 31, 40)]
+    for M in (16, 17, 32, 48):
         y = gemm_on(path, dev_bf16(x[:M]), c, s, g)
-        for j, i in enumerate((0, 5, 15, 16, 31)):
+        for j, i in enumerate((0, 5, 15, 16, 31, 40)):
             if i < M:
                 assert torch.equal(y[i:i + 1], alone[j]), (M, i)
     tl.check_device_error()
@@ -457,6 +467,34 @@ def test_plan_matches_stack(path):
     for e, y0 in zip(ents, ys):
         assert torch.equal(e[4], y0)
     plan.close()
+
+
+def test_plan_row_limits():
+    # a plan is one launch: up to 64 rows on the block-scaled path, 32 on the exact one
+    ents, _ = _small_stack(48, n_layers=1)
+    with tl.gemm_path(tl.PATH_BLOCK_SCALED):
+        plan = tl.Plan(ents, 48)
+        plan.run()
+        torch.cuda.synchronize()
+        plan.close()
+    tl.check_device_error()
+    with tl.gemm_path(tl.PATH_BF16_EXACT):
+        with pytest.raises(tl.TlError) as ei:
+            tl.Plan(ents, 48)
+    assert ei.value.status == 3
+
+
+@pytest.mark.parametrize("path", list(TC_PATHS))
+@pytest.mark.parametrize("M", [8, 48])
+def test_stack_rows_above_32(M, path):
+    ents, refs = _small_stack(M, n_layers=1)
+    mats = tl.make_matrices(ents)
+    with tl.gemm_path(TC_PATHS[path]):
+        tl.verify_stack(mats, M)
+    torch.cuda.synchronize()
+    tl.check_device_error()
+    for (c, s, g, x, y), (y_ref, a_ref, _) in zip(ents, refs):
+        assert_within_tol(host_f64(y), y_ref, a_ref, f"stack M={M} [{path}]")
 
 
 @pytest.mark.parametrize("path", list(TC_PATHS))
