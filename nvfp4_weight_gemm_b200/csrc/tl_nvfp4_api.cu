@@ -454,11 +454,13 @@ struct BsSchedule {
     int slots = 0;            // partial slots
 };
 
-void build_schedule(const tl_nvfp4_matrix* mats, int n_mats, int grid, BsSchedule* out) {
+// tile_rows: weight rows of an n-tile (128, or 256 when a stage holds two weight tiles).
+void build_schedule(const tl_nvfp4_matrix* mats, int n_mats, int grid, BsSchedule* out,
+                    int tile_rows = tl::TC_BLOCK_N) {
     struct Unit { int mat, ntile, kt; };
     std::vector<Unit> units;
     for (int i = 0; i < n_mats; ++i) {
-        const int nt = (mats[i].N + tl::TC_BLOCK_N - 1) / tl::TC_BLOCK_N, kt = mats[i].K / tl::TC_BLOCK_K;
+        const int nt = (mats[i].N + tile_rows - 1) / tile_rows, kt = mats[i].K / tl::TC_BLOCK_K;
         for (int j = 0; j < nt; ++j) units.push_back({i, j, kt});
     }
     const long long U = (long long)units.size(), G = grid;
@@ -545,6 +547,14 @@ void build_schedule(const tl_nvfp4_matrix* mats, int n_mats, int grid, BsSchedul
     out->begin[grid] = (int)out->segs.size();
 }
 
+// The X rows of the launch that serves Mp rows, and its weight tiles per stage: two (one X
+// stage for 256 weight rows) from TL_BS_WT2_MIN_NX rows up to 32.
+#ifndef TL_BS_WT2_MIN_NX
+#define TL_BS_WT2_MIN_NX 8
+#endif
+constexpr int bs_nx(int Mp) { return Mp <= 4 ? 4 : Mp <= 8 ? 8 : Mp <= 16 ? 16 : Mp <= 24 ? 24 : Mp <= 32 ? 32 : 64; }
+constexpr int bs_wt(int nx) { return (nx >= TL_BS_WT2_MIN_NX && nx <= 32) ? 2 : 1; }
+
 struct BsLaunch {
     tl::BsParams bp;
     tl::XSplitParams xp;
@@ -562,6 +572,7 @@ tl_status build_bs(const tl_nvfp4_matrix* mats, int n_mats, int M, const unsigne
     L->xtbl.assign(n_mats, tl::XSplitMat());
     long long tiles = 0;
     size_t xoff = 0, yoff = 0, soff = 0;
+    const int tile_rows = tl::TC_BLOCK_N * bs_wt(bs_nx(round4(M)));
     for (int i = 0; i < n_mats; ++i) {
         const tl_nvfp4_matrix& m = mats[i];
         const void* x = x_dev ? static_cast<const void*>(x_dev + xoff) : m.x;
@@ -569,18 +580,22 @@ tl_status build_bs(const tl_nvfp4_matrix* mats, int n_mats, int M, const unsigne
         tl_status st = build_bs_mat(&L->tbl[i], &L->xtbl[i], x, M, m.w_codes, m.w_scales, m.global_scale, y,
                                     m.N, m.K, xs + soff);
         if (st != TL_OK) return st;
-        tiles += (long long)((m.N + tl::TC_BLOCK_N - 1) / tl::TC_BLOCK_N) * (m.K / tl::TC_BLOCK_K);
+        tiles += (long long)((m.N + tile_rows - 1) / tile_rows) * (m.K / tl::TC_BLOCK_K);
         xoff += (size_t)2 * M * m.K;
         yoff += (size_t)2 * M * m.N;
         soff += xs_bytes_of(M, m.K);
     }
+    // the split's CTAs in order of decreasing K, so that the longest ones start first and the
+    // last wave is made of short ones (the split's outputs do not depend on the order)
+    std::stable_sort(L->xtbl.begin(), L->xtbl.end(),
+                     [](const tl::XSplitMat& a, const tl::XSplitMat& b) { return a.K > b.K; });
     memset(&L->bp, 0, sizeof L->bp);
     L->bp.n_mats = n_mats;
     L->bp.M = M;
     L->bp.Mp = round4(M);
     L->bp.mats = nullptr;
     L->grid = (int)std::min<long long>(tiles, num_sms);
-    build_schedule(mats, n_mats, L->grid, &L->sched);
+    build_schedule(mats, n_mats, L->grid, &L->sched, tile_rows);
     if (L->sched.slots > 2 * num_sms || L->sched.splits > num_sms)
         return fail(TL_ERR_DEVICE_FAULT, "internal: schedule needs %d partial slots and %d splits", L->sched.slots,
                     L->sched.splits);
@@ -596,26 +611,30 @@ tl_status build_bs(const tl_nvfp4_matrix* mats, int n_mats, int M, const unsigne
 
 template <int NX>
 tl_status launch_bs_gemm(DevState& d, tl::BsParams& p, int grid, cudaStream_t stream) {
-    using C = tl::BsCfg<NX>;
-    TL_CUDA(cudaFuncSetAttribute(tl::gemm_bs_kernel<NX>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
+    constexpr int WT = bs_wt(NX);
+    using C = tl::BsCfg<NX, WT>;
+    TL_CUDA(cudaFuncSetAttribute(tl::gemm_bs_kernel<NX, WT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::SMEM_BYTES));
     p.partials = d.partials;
     p.counters = d.counters;
     p.err = d.err;
-    tl::gemm_bs_kernel<NX><<<(unsigned)grid, tl::BS_THREADS, C::SMEM_BYTES, stream>>>(p);
+    tl::gemm_bs_kernel<NX, WT><<<(unsigned)grid, tl::BS_THREADS, C::SMEM_BYTES, stream>>>(p);
     TL_CUDA(cudaGetLastError());
     return TL_OK;
 }
 
 // The X split, then the GEMM, on `stream` (bp.segs / bp.seg_begin already on the device).
 tl_status launch_bs(DevState& d, tl::BsParams bp, const tl::XSplitParams& xp, int grid, cudaStream_t stream) {
-    tl::x_split_kernel<<<dim3((unsigned)xp.Mp, (unsigned)xp.n_mats), tl::XS_THREADS, 0, stream>>>(xp);
+    tl::x_split_kernel<<<dim3((unsigned)(xp.Mp / tl::XS_ROWS), (unsigned)xp.n_mats), tl::XS_THREADS, 0, stream>>>(xp);
     TL_CUDA(cudaGetLastError());
-    if (bp.Mp <= 4) return launch_bs_gemm<4>(d, bp, grid, stream);
-    if (bp.Mp <= 8) return launch_bs_gemm<8>(d, bp, grid, stream);
-    if (bp.Mp <= 16) return launch_bs_gemm<16>(d, bp, grid, stream);
-    if (bp.Mp <= 24) return launch_bs_gemm<24>(d, bp, grid, stream);
-    if (bp.Mp <= 32) return launch_bs_gemm<32>(d, bp, grid, stream);
-    return launch_bs_gemm<64>(d, bp, grid, stream);
+    switch (bs_nx(bp.Mp)) {
+        case 4: return launch_bs_gemm<4>(d, bp, grid, stream);
+        case 8: return launch_bs_gemm<8>(d, bp, grid, stream);
+        case 16: return launch_bs_gemm<16>(d, bp, grid, stream);
+        case 24: return launch_bs_gemm<24>(d, bp, grid, stream);
+        case 32: return launch_bs_gemm<32>(d, bp, grid, stream);
+        default: return launch_bs_gemm<64>(d, bp, grid, stream);
+    }
 }
 
 // The schedule as one device blob: segments, then the per-CTA offsets.

@@ -47,8 +47,8 @@ constexpr int TC_PIECES = 4;
 
 struct XSplitMat {
     const __nv_bfloat16* x;   // [M][K]
-    uint8_t* codes;           // [K/256][TC_PIECES][M][128], swizzled rows
-    uint8_t* scales;          // [K/256][TC_PIECES][M][16]
+    uint8_t* codes;           // [K/256][Mp][TC_PIECES][128], swizzled lines
+    uint8_t* scales;          // [K/256][Mp][TC_PIECES][16]
     float* factor;            // [M]
     int K;
 };
@@ -127,100 +127,44 @@ __device__ __forceinline__ uint32_t xs_e2m1x8(const float (&q)[8], uint32_t (&h)
 }
 
 constexpr int XS_THREADS = 256;
+constexpr int XS_ROWS = 4;   // rows per CTA: one group of four rows of the layout
 
-// Grid (Mp, n_mats): one CTA per row of one matrix; rows M .. Mp-1 write zero pieces.
-__global__ void __launch_bounds__(XS_THREADS) x_split_kernel(const __grid_constant__ XSplitParams p) {
-    __shared__ float red[XS_THREADS / 32];
-    __shared__ int bad_sh;
-    const XSplitMat& m = p.mats ? p.mats[blockIdx.y] : p.one;
-    const int row = blockIdx.x;
-    const int K = m.K;
-    const int M = p.M, Mp = p.Mp;
-    const bool pad_row = row >= M;
-    const __nv_bfloat16* x = m.x + (size_t)(pad_row ? 0 : row) * K;
-    uint8_t* const codes = m.codes;
-    uint8_t* const scales = m.scales;
-    float* const factor = m.factor;
-    // 1. the row's largest |x|, and whether any element is NaN or infinite
-    if (threadIdx.x == 0) bad_sh = 0;
-    float mx = 0.0f;
-    bool bad = false;
-#pragma unroll 4
-    for (int k8 = threadIdx.x; !pad_row && k8 < K / 8; k8 += XS_THREADS) {
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(x) + k8);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+// Piece codes and scale of one 16-k block (u: the block's residual in piece-0 units, updated in
+// place). inv_tab: 8 / (8 + m) for m = 0..7, then 0 and 1 / m for m = 1..7 (each correctly
+// rounded), so that 1 / s is exact table value times powers of two, the same bits as a division.
+__device__ __forceinline__ void xs_block_pieces(float (&u)[16], const float* inv_tab, uint8_t* cline, uint8_t* sdst,
+                                                uint32_t chunk, uint32_t ph0) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float a = fabsf(xs_u2f(w[j] << 16)), b = fabsf(xs_u2f(w[j] & 0xFFFF0000u));
-            bad |= !(a <= 3.402823466e38f) || !(b <= 3.402823466e38f);
-            mx = fmaxf(mx, fmaxf(a, b));
+    for (int pc = 0; pc < TC_PIECES; ++pc) {
+        const float unit = (float)(1 << (2 * pc));          // piece pc's units: 4^-pc of piece 0's
+        float a3[6];
+#pragma unroll
+        for (int i = 0; i < 5; ++i) {
+            float r;
+            asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(fabsf(u[3 * i])), "f"(fabsf(u[3 * i + 1])), "f"(fabsf(u[3 * i + 2])));
+            a3[i] = r;
         }
-    }
+        a3[5] = fabsf(u[15]);
+        float b0, b1, amax;
+        asm("max.f32 %0, %1, %2, %3;" : "=f"(b0) : "f"(a3[0]), "f"(a3[1]), "f"(a3[2]));
+        asm("max.f32 %0, %1, %2, %3;" : "=f"(b1) : "f"(a3[3]), "f"(a3[4]), "f"(a3[5]));
+        amax = fmaxf(b0, b1);
+        const uint32_t sc = xs_e4m3_ceil_div6(amax * unit);
+        const float sv = xs_e4m3_value(sc);
+        const float s = sv * (1.0f / unit);                 // the scale in piece-0 units (exact)
+        // 1 / sv: normal codes (1 + m/8) 2^(E-7) -> 2^(7-E) * 8 / (8 + m); subnormal m 2^-9 -> 512 / m
+        const uint32_t E = sc >> 3;
+        const float pw = (E != 0u) ? __uint_as_float((134u - E) << 23) : 512.0f;
+        const float inv = (inv_tab[(E != 0u) ? (sc & 7u) : (8u + sc)] * pw) * unit;   // = 1 / s (0 for sc == 0)
+        uint32_t w[2];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
-    __syncthreads();
-    if (bad) bad_sh = 1;
-    float r = red[0];
+        for (int hlf = 0; hlf < 2; ++hlf) {
+            float q[8];
 #pragma unroll
-    for (int i = 1; i < XS_THREADS / 32; ++i) r = fmaxf(r, red[i]);
-    __syncthreads();
-    const bool bad_row = bad_sh != 0 || pad_row;   // both write zero pieces
-    int e = 0;                                  // r * 2^e in [2^7, 2^8)
-    if (r > 0.0f && !bad_row) {
-        int fe;
-        frexpf(r, &fe);                         // r in [2^(fe-1), 2^fe)
-        e = 8 - fe;
-    }
-    if (threadIdx.x == 0 && !pad_row) factor[row] = bad_row ? __int_as_float(0x7FC00000) : ldexpf(1.0f, -e);
-    // exact scaling by 2^e in two steps (each factor a normal power of two)
-    const float p1 = ldexpf(1.0f, e / 2), p2 = ldexpf(1.0f, e - e / 2);
-    // 2. four pieces per 16-k block, one thread per block
-    for (int b = threadIdx.x; b < K / 16; b += XS_THREADS) {
-        const int kt = b >> 4, bt = b & 15;       // k-tile, block within it
-        const size_t j0 = ((size_t)kt * Mp + (size_t)row) * TC_PIECES;   // line of piece 0
-        // piece p is line j0 + p; its 16-byte chunk bt/2 sits at chunk (bt/2) ^ ((j0 + p) & 7)
-        uint8_t* cline = codes + j0 * 128 + 8 * (bt & 1);
-        uint8_t* sdst = scales + j0 * 16 + bt;
-        const uint32_t chunk = (uint32_t)(bt >> 1), ph0 = (uint32_t)(j0 & 7);
-        if (bad_row) {
-#pragma unroll
-            for (int pc = 0; pc < TC_PIECES; ++pc) {
-                *reinterpret_cast<uint2*>(cline + pc * 128 + ((chunk ^ ((ph0 + pc) & 7u)) << 4)) = make_uint2(0u, 0u);
-                sdst[pc * 16] = 0;
-            }
-            continue;
-        }
-        // u: the block's residual, always in piece-0 units (x * 2^e)
-        float u[16];
-        {
-            const uint4 v0 = __ldg(reinterpret_cast<const uint4*>(x) + 2 * b);
-            const uint4 v1 = __ldg(reinterpret_cast<const uint4*>(x) + 2 * b + 1);
-            const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                u[2 * j] = (xs_u2f(w[j] << 16) * p1) * p2;
-                u[2 * j + 1] = (xs_u2f(w[j] & 0xFFFF0000u) * p1) * p2;
-            }
-        }
-#pragma unroll
-        for (int pc = 0; pc < TC_PIECES; ++pc) {
-            const float unit = (float)(1 << (2 * pc));          // piece pc's units: 4^-pc of piece 0's
-            float amax = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(u[i]));
-            const uint32_t sc = xs_e4m3_ceil_div6(amax * unit);
-            const float sv = xs_e4m3_value(sc);
-            const float s = sv * (1.0f / unit);                 // the scale in piece-0 units (exact)
-            const float inv = (sc != 0u) ? unit / sv : 0.0f;    // = 1 / s
-            uint32_t w[2];
-#pragma unroll
-            for (int hlf = 0; hlf < 2; ++hlf) {
-                float q[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) q[i] = u[8 * hlf + i] * inv;
-                uint32_t h[4];
-                w[hlf] = xs_e2m1x8(q, h);
+            for (int i = 0; i < 8; ++i) q[i] = u[8 * hlf + i] * inv;
+            uint32_t h[4];
+            w[hlf] = xs_e2m1x8(q, h);
+            if (pc + 1 < TC_PIECES) {
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const float2 qv = __half22float2(*reinterpret_cast<const __half2*>(&h[i]));
@@ -228,9 +172,114 @@ __global__ void __launch_bounds__(XS_THREADS) x_split_kernel(const __grid_consta
                     u[8 * hlf + 2 * i + 1] = fmaf(-qv.y, s, u[8 * hlf + 2 * i + 1]);
                 }
             }
-            *reinterpret_cast<uint2*>(cline + pc * 128 + ((chunk ^ ((ph0 + pc) & 7u)) << 4)) = make_uint2(w[0], w[1]);
-            sdst[pc * 16] = (uint8_t)sc;
         }
+        *reinterpret_cast<uint2*>(cline + pc * 128 + ((chunk ^ ((ph0 + pc) & 7u)) << 4)) = make_uint2(w[0], w[1]);
+        sdst[pc * 16] = (uint8_t)sc;
+    }
+}
+
+// Grid (Mp / 4, n_mats): one CTA per group of four rows of one matrix; rows M .. Mp-1 write zero
+// pieces. The four rows' 16-k blocks are shared out evenly over the CTA's threads.
+__global__ void __launch_bounds__(XS_THREADS, 4) x_split_kernel(const __grid_constant__ XSplitParams p) {
+    __shared__ float red[XS_THREADS / 32][XS_ROWS];
+    __shared__ int bad_sh[XS_ROWS];
+    __shared__ float p1_sh[XS_ROWS], p2_sh[XS_ROWS];
+    __shared__ int zero_sh[XS_ROWS];
+    __shared__ float inv_tab[16];
+    const XSplitMat& m = p.mats ? p.mats[blockIdx.y] : p.one;
+    const int row0 = blockIdx.x * XS_ROWS;
+    const int K = m.K;
+    const int M = p.M, Mp = p.Mp;
+    const int KB = K / 16;
+    const __nv_bfloat16* const x = m.x;
+    uint8_t* const codes = m.codes;
+    uint8_t* const scales = m.scales;
+    float* const factor = m.factor;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid < XS_ROWS) bad_sh[tid] = 0;
+    if (tid < 16) inv_tab[tid] = (tid < 8) ? 8.0f / (float)(8 + tid) : (tid == 8) ? 0.0f : 1.0f / (float)(tid - 8);
+    __syncthreads();
+    // 1. each row's largest |x|, and whether any element is NaN or infinite
+#pragma unroll
+    for (int rr = 0; rr < XS_ROWS; ++rr) {
+        float mx = 0.0f;
+        bool bad = false;
+        if (row0 + rr < M) {
+            const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)(row0 + rr) * K);
+#pragma unroll 4
+            for (int k8 = tid; k8 < K / 8; k8 += XS_THREADS) {
+                const uint4 v = __ldg(xr + k8);
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float a = fabsf(xs_u2f(w[j] << 16)), b = fabsf(xs_u2f(w[j] & 0xFFFF0000u));
+                    bad |= !(a <= 3.402823466e38f) || !(b <= 3.402823466e38f);
+                    mx = fmaxf(mx, fmaxf(a, b));
+                }
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+        const bool any_bad = __any_sync(0xFFFFFFFFu, bad);
+        if (lane == 0) {
+            red[warp][rr] = mx;
+            if (any_bad) bad_sh[rr] = 1;
+        }
+    }
+    __syncthreads();
+    if (tid < XS_ROWS) {
+        const int row = row0 + tid;
+        float r = red[0][tid];
+#pragma unroll
+        for (int i = 1; i < XS_THREADS / 32; ++i) r = fmaxf(r, red[i][tid]);
+        const bool pad_row = row >= M;
+        const bool zero = bad_sh[tid] != 0 || pad_row;    // bad and padding rows write zero pieces
+        int e = 0;                                        // r * 2^e in [2^7, 2^8)
+        if (r > 0.0f && !zero) {
+            int fe;
+            frexpf(r, &fe);                               // r in [2^(fe-1), 2^fe)
+            e = 8 - fe;
+        }
+        if (!pad_row) factor[row] = zero ? __int_as_float(0x7FC00000) : ldexpf(1.0f, -e);
+        // exact scaling by 2^e in two steps (each factor a normal power of two)
+        p1_sh[tid] = ldexpf(1.0f, e / 2);
+        p2_sh[tid] = ldexpf(1.0f, e - e / 2);
+        zero_sh[tid] = zero ? 1 : 0;
+    }
+    __syncthreads();
+    // 2. four pieces per 16-k block, one thread per block; block b of row rr is item rr * KB + b
+    int rr = 0, b = tid;
+    while (b >= KB && rr < XS_ROWS) { b -= KB; ++rr; }
+    while (rr < XS_ROWS) {
+        const int row = row0 + rr;
+        const int kt = b >> 4, bt = b & 15;       // k-tile, block within it
+        const size_t j0 = ((size_t)kt * Mp + (size_t)row) * TC_PIECES;   // line of piece 0
+        // piece p is line j0 + p; its 16-byte chunk bt/2 sits at chunk (bt/2) ^ ((j0 + p) & 7)
+        uint8_t* cline = codes + j0 * 128 + 8 * (bt & 1);
+        uint8_t* sdst = scales + j0 * 16 + bt;
+        const uint32_t chunk = (uint32_t)(bt >> 1), ph0 = (uint32_t)(j0 & 7);
+        if (zero_sh[rr]) {
+#pragma unroll
+            for (int pc = 0; pc < TC_PIECES; ++pc) {
+                *reinterpret_cast<uint2*>(cline + pc * 128 + ((chunk ^ ((ph0 + pc) & 7u)) << 4)) = make_uint2(0u, 0u);
+                sdst[pc * 16] = 0;
+            }
+        } else {
+            // u: the block's residual, always in piece-0 units (x * 2^e)
+            const float p1 = p1_sh[rr], p2 = p2_sh[rr];
+            const uint4* xb = reinterpret_cast<const uint4*>(x + (size_t)row * K) + 2 * b;
+            const uint4 v0 = __ldg(xb), v1 = __ldg(xb + 1);
+            const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            float u[16];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                u[2 * j] = (xs_u2f(w[j] << 16) * p1) * p2;
+                u[2 * j + 1] = (xs_u2f(w[j] & 0xFFFF0000u) * p1) * p2;
+            }
+            xs_block_pieces(u, inv_tab, cline, sdst, chunk, ph0);
+        }
+        b += XS_THREADS;
+        while (b >= KB && rr < XS_ROWS) { b -= KB; ++rr; }
     }
 }
 

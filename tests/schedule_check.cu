@@ -11,7 +11,8 @@
 #include <utility>
 #include <vector>
 
-static int check(const std::vector<std::pair<int, int>>& shapes, int grid, double min_eff, bool verbose) {
+static int check(const std::vector<std::pair<int, int>>& shapes, int grid, double min_eff, bool verbose,
+                 int rows = 128) {
     std::vector<tl_nvfp4_matrix> mats;
     for (auto& sh : shapes) {
         tl_nvfp4_matrix m{};
@@ -20,7 +21,7 @@ static int check(const std::vector<std::pair<int, int>>& shapes, int grid, doubl
         mats.push_back(m);
     }
     BsSchedule sc;
-    build_schedule(mats.data(), (int)mats.size(), grid, &sc);
+    build_schedule(mats.data(), (int)mats.size(), grid, &sc, rows);
     int bad = 0;
     if ((int)sc.begin.size() != grid + 1 || sc.begin[0] != 0 || sc.begin[grid] != (int)sc.segs.size()) {
         printf("per-CTA offsets malformed\n");
@@ -41,7 +42,7 @@ static int check(const std::vector<std::pair<int, int>>& shapes, int grid, doubl
     }
     long long total = 0;
     for (size_t i = 0; i < mats.size(); ++i) {
-        const int nt = (mats[i].N + 127) / 128, kt = mats[i].K / 256;
+        const int nt = (mats[i].N + rows - 1) / rows, kt = mats[i].K / 256;
         total += (long long)nt * kt;
         for (int j = 0; j < nt; ++j) {
             auto v = cov[{(int)i, j}];
@@ -74,9 +75,9 @@ static int check(const std::vector<std::pair<int, int>>& shapes, int grid, doubl
     if (mx > ideal) { ++bad; printf("a CTA has %lld k-tiles, more than ceil(total / grid) = %lld\n", mx, ideal); }
     if (eff < min_eff) { ++bad; printf("balance %.4f below %.4f\n", eff, min_eff); }
     if (verbose || bad)
-        printf("%zu matrices, grid %d: %lld k-tiles, largest CTA share %lld (balance %.4f), %zu segments, "
+        printf("%d-row n-tiles, %zu matrices, grid %d: %lld k-tiles, largest CTA share %lld (balance %.4f), %zu segments, "
                "%d splits, %d slots, bad %d\n",
-               mats.size(), grid, total, mx, eff, sc.segs.size(), sc.splits, sc.slots, bad);
+               rows, mats.size(), grid, total, mx, eff, sc.segs.size(), sc.splits, sc.slots, bad);
     return bad;
 }
 
@@ -89,21 +90,24 @@ int main() {
         stack.push_back({34816, 5120});
         stack.push_back({5120, 17408});
     }
-    bad += check(stack, 148, 0.999, true);           // the 64-layer stack
-    bad += check({{5120, 5120}}, 148, 0.0, true);      // single matrices: one k-tile short at most
-    bad += check({{34816, 5120}}, 148, 0.0, true);
-    bad += check({{5120, 17408}}, 148, 0.0, true);
-    bad += check({{677, 2304}}, 54, 0.0, true);
-    bad += check({{256, 512}}, 4, 0.0, true);
-    srand(7);
-    for (int it = 0; it < 300; ++it) {
-        std::vector<std::pair<int, int>> sh;
-        const int n = 1 + rand() % 40;
-        for (int i = 0; i < n; ++i) sh.push_back({1 + rand() % 20000, 256 * (1 + rand() % 80)});
-        long long tiles = 0;
-        for (auto& s2 : sh) tiles += (long long)((s2.first + 127) / 128) * (s2.second / 256);
-        const int grid = (int)std::min<long long>(tiles, 1 + rand() % 160);
-        bad += check(sh, grid, 0.0, false);
+    // n-tiles of 128 weight rows, and of 256 (two weight tiles per stage)
+    for (int rows = 128; rows <= 256; rows *= 2) {
+        bad += check(stack, 148, 0.999, true, rows);           // the 64-layer stack
+        bad += check({{5120, 5120}}, 148, 0.0, true, rows);      // single matrices: one k-tile short at most
+        bad += check({{34816, 5120}}, 148, 0.0, true, rows);
+        bad += check({{5120, 17408}}, 148, 0.0, true, rows);
+        bad += check({{677, 2304}}, 27, 0.0, true, rows);
+        bad += check({{256, 512}}, 2, 0.0, true, rows);
+        srand(7);
+        for (int it = 0; it < 300; ++it) {
+            std::vector<std::pair<int, int>> sh;
+            const int n = 1 + rand() % 40;
+            for (int i = 0; i < n; ++i) sh.push_back({1 + rand() % 20000, 256 * (1 + rand() % 80)});
+            long long tiles = 0;
+            for (auto& s2 : sh) tiles += (long long)((s2.first + rows - 1) / rows) * (s2.second / 256);
+            const int grid = (int)std::min<long long>(tiles, 1 + rand() % 160);
+            bad += check(sh, grid, 0.0, false, rows);
+        }
     }
     printf("bad=%d\n", bad);
     return bad != 0;
