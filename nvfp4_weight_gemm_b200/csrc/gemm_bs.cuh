@@ -13,7 +13,7 @@
 //   Y[m][n]       = bf16( (sum_p 4^-p D[n][4 m + p]) * g * factor[m] )
 //
 //   * Work. A tile is 128 weight rows x 256 k, or two such weight tiles (256 rows) that share
-//     one copy of the X pieces (WT = 2, from 8 X rows up); an n-tile is all k-tiles of its
+//     one copy of the X pieces (WT = 2, for 17 to 32 X rows); an n-tile is all k-tiles of its
 //     weight rows. The host lays out each CTA's work as a list of segments (k-tiles [k0, k1)
 //     of one n-tile), built from the matrices' shapes alone:
 //     - first, whole n-tiles dealt round-robin over the CTAs, so that at any moment the CTAs
