@@ -57,8 +57,8 @@ struct DevState {
     bool ready = false;
     int num_sms = 0;
     int* err = nullptr;            // device status word
-    float* partials = nullptr;     // [2 * num_sms][64][128]
-    unsigned* counters = nullptr;  // [4 * num_sms]
+    float* partials = nullptr;     // [4 * num_sms][64][128]
+    unsigned* counters = nullptr;  // [8 * num_sms]: four per split, up to 2 * num_sms splits
     unsigned* qscratch = nullptr;  // quantiser absmax + non-finite flag
     bool smem_attr_set = false;
     unsigned char* xs_buf = nullptr;   // X pieces of the block-scaled path (calls without a plan)
@@ -106,15 +106,15 @@ tl_status init_locked(int device) {
             break;
         }
         d.num_sms = sms;
-        const size_t pbytes = (size_t)2 * sms * tl::BS_PART_ROWS * tl::TC_BLOCK_N * sizeof(float);
+        const size_t pbytes = (size_t)4 * sms * tl::BS_PART_ROWS * tl::TC_BLOCK_N * sizeof(float);
         if (cudaMalloc(&d.err, 64) != cudaSuccess || cudaMalloc(&d.partials, pbytes) != cudaSuccess ||
-            cudaMalloc(&d.counters, (size_t)4 * sms * sizeof(unsigned)) != cudaSuccess ||
+            cudaMalloc(&d.counters, (size_t)8 * sms * sizeof(unsigned)) != cudaSuccess ||
             cudaMalloc(&d.qscratch, 64) != cudaSuccess) {
             st = fail(TL_ERR_CUDA, "cudaMalloc of the per-device state failed");
             break;
         }
         if (cudaMemset(d.err, 0, 64) != cudaSuccess ||
-            cudaMemset(d.counters, 0, (size_t)4 * sms * sizeof(unsigned)) != cudaSuccess ||
+            cudaMemset(d.counters, 0, (size_t)8 * sms * sizeof(unsigned)) != cudaSuccess ||
             cudaDeviceSynchronize() != cudaSuccess) {
             st = fail(TL_ERR_CUDA, "initialising the per-device state failed");
             break;
@@ -442,11 +442,18 @@ tl_status build_bs_mat(tl::BsMat* m, tl::XSplitMat* xm, const void* x, int M, co
     return TL_OK;
 }
 
-// Each CTA's list of segments (gemm_bs.cuh): whole n-tiles dealt in order, each to the CTA with
-// the fewest k-tiles so far (round-robin when the n-tiles are alike), so that the CTAs move
-// through the matrices side by side and share the X pieces in L2; the last two to three rounds'
-// worth of n-tiles are cut into equal shares of k-tiles (stream-K), so every CTA ends with the
-// same number of k-tiles. Depends only on the shapes and the grid.
+// Each CTA's list of segments (gemm_bs.cuh), built from the shapes and the grid alone. The
+// work is cut in units of 256 weight rows (all k-tiles of them):
+//   - whole units dealt in order, each to the CTA with the fewest k-tiles so far (round-robin
+//     when the units are alike), so that the CTAs move through the matrices side by side and
+//     share the X pieces in L2;
+//   - the last two to three rounds' worth of units cut into equal shares of k-tiles (stream-K),
+//     so every CTA ends with the same number of k-tiles; a cut unit ("split") is summed over
+//     its parts in k order.
+// A launch with 128-row n-tiles runs a unit as its two halves, one after the other, with the
+// same k ranges (each half its own split); a launch with 256-row n-tiles runs it as one. Either
+// way every weight row gets the same cuts in k and the same order of summation, so an output
+// does not depend on M (nor on the launch the size of M selects).
 struct BsSchedule {
     std::vector<tl::BsSeg> segs;
     std::vector<int> begin;   // [grid + 1]
@@ -454,18 +461,29 @@ struct BsSchedule {
     int slots = 0;            // partial slots
 };
 
-// tile_rows: weight rows of an n-tile (128, or 256 when a stage holds two weight tiles).
+constexpr int kBsUnitRows = 256;
+
+// Work units of a stack: 256-row units times k-tiles.
+long long bs_unit_ktiles(const tl_nvfp4_matrix* mats, int n_mats) {
+    long long t = 0;
+    for (int i = 0; i < n_mats; ++i)
+        t += (long long)((mats[i].N + kBsUnitRows - 1) / kBsUnitRows) * (mats[i].K / tl::TC_BLOCK_K);
+    return t;
+}
+
+// tile_rows: weight rows of the launch's n-tiles (128, or 256 when a stage holds two weight tiles).
 void build_schedule(const tl_nvfp4_matrix* mats, int n_mats, int grid, BsSchedule* out,
                     int tile_rows = tl::TC_BLOCK_N) {
-    struct Unit { int mat, ntile, kt; };
+    struct Unit { int mat, unit, kt; };
     std::vector<Unit> units;
     for (int i = 0; i < n_mats; ++i) {
-        const int nt = (mats[i].N + tile_rows - 1) / tile_rows, kt = mats[i].K / tl::TC_BLOCK_K;
-        for (int j = 0; j < nt; ++j) units.push_back({i, j, kt});
+        const int nu = (mats[i].N + kBsUnitRows - 1) / kBsUnitRows, kt = mats[i].K / tl::TC_BLOCK_K;
+        for (int j = 0; j < nu; ++j) units.push_back({i, j, kt});
     }
+    const int halves = kBsUnitRows / tile_rows;   // n-tiles per unit
     const long long U = (long long)units.size(), G = grid;
-    // n-tiles dealt whole: all but a tail of at least two per CTA and at least two of the
-    // largest n-tiles' k-tiles per CTA, enough to even out the dealt part
+    // units dealt whole: all but a tail of at least two per CTA and at least two of the largest
+    // units' k-tiles per CTA, enough to even out the dealt part
     int max_kt = 1;
     for (const Unit& un : units) max_kt = std::max(max_kt, un.kt);
     long long R = std::max(0LL, U - 2 * G), tail = 0;
@@ -473,10 +491,16 @@ void build_schedule(const tl_nvfp4_matrix* mats, int n_mats, int grid, BsSchedul
     while (R > 0 && tail < 2 * G * max_kt) tail += units[--R].kt;
     std::vector<std::vector<tl::BsSeg>> per(grid);
     std::vector<long long> load(grid, 0);
-    auto seg = [](const Unit& u, int k0, int k1) {
+    // the n-tiles of unit u (those that hold rows < N)
+    auto ntiles_of = [&](const Unit& u, int* first) {
+        *first = u.unit * halves;
+        const int nt_mat = (mats[u.mat].N + tile_rows - 1) / tile_rows;
+        return std::min(halves, nt_mat - *first);
+    };
+    auto seg = [](const Unit& u, int ntile, int k0, int k1) {
         tl::BsSeg sg;
         sg.mat = u.mat;
-        sg.ntile = u.ntile;
+        sg.ntile = ntile;
         sg.k0 = (uint16_t)k0;
         sg.k1 = (uint16_t)k1;
         sg.split = -1;
@@ -485,15 +509,17 @@ void build_schedule(const tl_nvfp4_matrix* mats, int n_mats, int grid, BsSchedul
         sg.parts = 1;
         return sg;
     };
-    // deal each whole n-tile, in order, to the CTA with the fewest k-tiles so far (the one that
-    // will be free first; ties to the lowest index): round-robin when the n-tiles are alike
+    // deal each whole unit, in order, to the CTA with the fewest k-tiles so far (the one that
+    // will be free first; ties to the lowest index): round-robin when the units are alike
     std::priority_queue<std::pair<long long, int>, std::vector<std::pair<long long, int>>,
                         std::greater<std::pair<long long, int>>> freeq;
     for (int c = 0; c < grid; ++c) freeq.push({0LL, c});
     for (long long u = 0; u < R; ++u) {
         const int c = freeq.top().second;
         freeq.pop();
-        per[c].push_back(seg(units[u], 0, units[u].kt));
+        int t0 = 0;
+        const int nt = ntiles_of(units[u], &t0);
+        for (int h = 0; h < nt; ++h) per[c].push_back(seg(units[u], t0 + h, 0, units[u].kt));
         load[c] += units[u].kt;
         freeq.push({load[c], c});
     }
@@ -523,18 +549,25 @@ void build_schedule(const tl_nvfp4_matrix* mats, int n_mats, int grid, BsSchedul
         size_t j = i;
         while (j < parts.size() && parts[j].unit == parts[i].unit) ++j;
         const Unit& un = units[parts[i].unit];
+        int t0 = 0;
+        const int nt = ntiles_of(un, &t0);
         if (j - i == 1) {
-            per[parts[i].cta].push_back(seg(un, parts[i].k0, parts[i].k1));
+            for (int h = 0; h < nt; ++h) per[parts[i].cta].push_back(seg(un, t0 + h, parts[i].k0, parts[i].k1));
         } else {
-            const int split = out->splits++;
-            for (size_t r = i; r < j; ++r) {
-                tl::BsSeg sg = seg(un, parts[r].k0, parts[r].k1);
-                sg.split = split;
-                sg.slot = out->slots++;
-                sg.rank = (uint16_t)(r - i);
-                sg.parts = (uint16_t)(j - i);
-                per[parts[r].cta].push_back(sg);
-            }
+            // each n-tile of the unit is a split of its own, its parts in consecutive slots; a
+            // CTA's parts of the unit's n-tiles follow one another
+            int split0 = out->splits, slot0 = out->slots;
+            out->splits += nt;
+            out->slots += nt * (int)(j - i);
+            for (size_t r = i; r < j; ++r)
+                for (int h = 0; h < nt; ++h) {
+                    tl::BsSeg sg = seg(un, t0 + h, parts[r].k0, parts[r].k1);
+                    sg.split = split0 + h;
+                    sg.rank = (uint16_t)(r - i);
+                    sg.parts = (uint16_t)(j - i);
+                    sg.slot = slot0 + h * (int)(j - i) + (int)(r - i);
+                    per[parts[r].cta].push_back(sg);
+                }
         }
         i = j;
     }
@@ -570,7 +603,6 @@ tl_status build_bs(const tl_nvfp4_matrix* mats, int n_mats, int M, const unsigne
                    unsigned char* xs, int num_sms, BsLaunch* L) {
     L->tbl.assign(n_mats, tl::BsMat());
     L->xtbl.assign(n_mats, tl::XSplitMat());
-    long long tiles = 0;
     size_t xoff = 0, yoff = 0, soff = 0;
     const int tile_rows = tl::TC_BLOCK_N * bs_wt(bs_nx(round4(M)));
     for (int i = 0; i < n_mats; ++i) {
@@ -580,7 +612,6 @@ tl_status build_bs(const tl_nvfp4_matrix* mats, int n_mats, int M, const unsigne
         tl_status st = build_bs_mat(&L->tbl[i], &L->xtbl[i], x, M, m.w_codes, m.w_scales, m.global_scale, y,
                                     m.N, m.K, xs + soff);
         if (st != TL_OK) return st;
-        tiles += (long long)((m.N + tile_rows - 1) / tile_rows) * (m.K / tl::TC_BLOCK_K);
         xoff += (size_t)2 * M * m.K;
         yoff += (size_t)2 * M * m.N;
         soff += xs_bytes_of(M, m.K);
@@ -594,9 +625,9 @@ tl_status build_bs(const tl_nvfp4_matrix* mats, int n_mats, int M, const unsigne
     L->bp.M = M;
     L->bp.Mp = round4(M);
     L->bp.mats = nullptr;
-    L->grid = (int)std::min<long long>(tiles, num_sms);
+    L->grid = (int)std::min<long long>(bs_unit_ktiles(mats, n_mats), num_sms);
     build_schedule(mats, n_mats, L->grid, &L->sched, tile_rows);
-    if (L->sched.slots > 2 * num_sms || L->sched.splits > num_sms)
+    if (L->sched.slots > 4 * num_sms || L->sched.splits > 2 * num_sms)
         return fail(TL_ERR_DEVICE_FAULT, "internal: schedule needs %d partial slots and %d splits", L->sched.slots,
                     L->sched.splits);
     if (n_mats == 1) L->bp.one = L->tbl[0];
