@@ -13,7 +13,7 @@
 //   Y[m][n]       = bf16( (sum_p 4^-p D[n][4 m + p]) * g * factor[m] )
 //
 //   * Work. A tile is 128 weight rows x 256 k, or two such weight tiles (256 rows) that share
-//     one copy of the X pieces (WT = 2, for 17 to 32 X rows); an n-tile is all k-tiles of its
+//     one copy of the X pieces (WT = 2, for 9 to 32 X rows); an n-tile is all k-tiles of its
 //     weight rows. The host lays out each CTA's work as a list of segments (k-tiles [k0, k1)
 //     of one n-tile), built from the matrices' shapes alone:
 //     - first, whole n-tiles dealt round-robin over the CTAs, so that at any moment the CTAs
@@ -223,8 +223,8 @@ gemm_bs_kernel(const __grid_constant__ BsParams p) {
         const int wt = lane >> 2;                               // weight tile of a W lane
         // L2 policies: X pieces evict-last (every CTA on the matrix reads them); weights evict-first
         // with one weight tile per stage, evict-normal with two, which in paired timings keeps
-        // the X pieces from being re-read from DRAM at 17 to 32 X rows (3-4% less time there)
-        // while costing about 1% below
+        // the X pieces from being re-read from DRAM with two tiles (3-4% less time there) while
+        // costing about 1% with one
         const uint64_t pol = w_lane ? ((WT == 2) ? policy_evict_normal() : policy_evict_first()) : policy_evict_last();
         // lane 2: X piece codes (4 Mp rows x 128 B), lane 3: X piece scales (4 Mp rows x 16 B)
         const uint32_t xbytes = (uint32_t)(TC_PIECES * p.Mp) * ((lane == 2) ? 128u : 16u);

@@ -583,7 +583,7 @@ void build_schedule(const tl_nvfp4_matrix* mats, int n_mats, int grid, BsSchedul
 // The X rows of the launch that serves Mp rows, and its weight tiles per stage: two (one X
 // stage for 256 weight rows) from TL_BS_WT2_MIN_NX rows up to 32.
 #ifndef TL_BS_WT2_MIN_NX
-#define TL_BS_WT2_MIN_NX 24
+#define TL_BS_WT2_MIN_NX 16
 #endif
 constexpr int bs_nx(int Mp) { return Mp <= 4 ? 4 : Mp <= 8 ? 8 : Mp <= 16 ? 16 : Mp <= 24 ? 24 : Mp <= 32 ? 32 : 64; }
 constexpr int bs_wt(int nx) { return (nx >= TL_BS_WT2_MIN_NX && nx <= 32) ? 2 : 1; }
