@@ -1,13 +1,13 @@
 // gemm_bs.cuh -- block-scaled tensor-core NVFP4 verify GEMM for sm_100a (no CUDA-core dequant).
 //
-// Y[M,N] = X[M,K] . dequant(W)[N,K]^T for M <= 32 (TandemLLM docs v0.12.0, "What TandemLLM is",
-// section 1.2). W is already E2M1 with one E4M3 scale per 16 k, which is what
-// tcgen05.mma.kind::mxf4nvf4.block_scale consumes: the weight tile goes from HBM (TMA) into
-// shared memory and from there straight into the tensor core, with no decode on the CUDA
-// cores. X is brought into the same form beforehand (xsplit.cuh): per row a power of two and
-// TC_PIECES FP4 pieces with E4M3 scales. The rows' pieces are stacked along the MMA's N
-// dimension (row m's pieces adjacent; Mp = M rounded up to a multiple of 4, padding rows
-// zero), so one MMA per 64-k chunk serves every X row and every piece:
+// Y[M,N] = X[M,K] . dequant(W)[N,K]^T for M <= 64 per launch (TandemLLM docs v0.12.0, "What
+// TandemLLM is", section 1.2: the draft tree's rows, 1 to 32). W is already E2M1 with one E4M3
+// scale per 16 k, which is what tcgen05.mma.kind::mxf4nvf4.block_scale consumes: the weight
+// tile goes from HBM (TMA) into shared memory and from there straight into the tensor core,
+// with no decode on the CUDA cores. X is brought into the same form beforehand (xsplit.cuh):
+// per row a power of two and TC_PIECES FP4 pieces with E4M3 scales. The rows' pieces are
+// stacked along the MMA's N dimension (row m's pieces adjacent; Mp = M rounded up to a multiple
+// of 4, padding rows zero), so one MMA per 64-k chunk serves every X row and every piece:
 //
 //   D[n][4 m + p] = sum_k  w[n][k] * piece_p[m][k]        (fp32, in tensor memory; N = 4 Mp)
 //   Y[m][n]       = bf16( (sum_p 4^-p D[n][4 m + p]) * g * factor[m] )
@@ -15,14 +15,15 @@
 //   * Work. A tile is 128 weight rows x 256 k, or two such weight tiles (256 rows) that share
 //     one copy of the X pieces (WT = 2, for 9 to 32 X rows); an n-tile is all k-tiles of its
 //     weight rows. The host lays out each CTA's work as a list of segments (k-tiles [k0, k1)
-//     of one n-tile), built from the matrices' shapes alone:
-//     - first, whole n-tiles dealt round-robin over the CTAs, so that at any moment the CTAs
-//       work on neighbouring n-tiles of one or two matrices and the X pieces they all read
-//       stay in L2;
-//     - then the remaining n-tiles as one list of k-tiles cut so that every CTA ends with the
+//     of one n-tile), built from the matrices' shapes alone, in units of 256 weight rows:
+//     - first, whole units dealt round-robin over the CTAs, so that at any moment the CTAs
+//       work on neighbouring rows of one or two matrices and the X pieces they all read stay
+//       in L2;
+//     - then the remaining units as one list of k-tiles cut so that every CTA ends with the
 //       same number of k-tiles (stream-K). A cut n-tile ("split") is reduced by its last
-//       contributor, adding the parts in k order, so every output has one fixed reduction
-//       order that does not depend on M.
+//       contributor, adding the parts in k order. With 128-row n-tiles a unit runs as its two
+//       halves with the same cuts, so every output has one fixed reduction order that does
+//       not depend on M.
 //   * Roles, 12 warps.
 //     - Warp 0: copies into a ring of stages, four (six with WT = 2) per tile from as many
 //       lanes at once. Lanes 0 and 1 (4 and 5 for the second weight tile): a TMA tensor copy
@@ -84,8 +85,8 @@ struct BsParams {
     int Mp;                 // M rounded up to a multiple of 4: X rows per piece group in the layout
     const BsSeg* segs;      // every CTA's segments, CTA by CTA
     const int* seg_begin;   // [gridDim.x + 1]: CTA c runs segs[seg_begin[c] .. seg_begin[c+1])
-    float* partials;        // [slots][32][128] fp32
-    unsigned* counters;     // [4 * splits], zero between launches
+    float* partials;        // [slots][64 x 128] fp32: [X row][128] or, with two weight tiles, [X row][256]
+    unsigned* counters;     // [4 * splits] (one per 32-row quarter), zero between launches
     int* err;
     BsMat one;
 };
