@@ -200,9 +200,19 @@ tl_status tl_nvfp4_verify_stack_host(const tl_nvfp4_matrix* mats, int n_mats, in
  * work, asynchronous on `stream`, and capturable into a CUDA graph.
  * tl_nvfp4_plan_run_host() is the end-to-end form: it requires that the plan's X_i
  * are packed back to back in one device buffer (X_{i+1} starts right after X_i) and
- * likewise the Y_i, then copies all X from `x_host`, runs, and copies all Y to
- * `y_host` (pinned host memory keeps the copies asynchronous); TL_ERR_INVALID_VALUE
- * if the plan's buffers are not packed. Destroy synchronises the device before freeing.
+ * likewise the Y_i, then copies X from `x_host`, runs, and copies Y to `y_host`
+ * (pinned host memory keeps the copies asynchronous); TL_ERR_INVALID_VALUE if the
+ * plan's buffers are not packed. With two or more matrices the stack is cut into up to
+ * 8 chunks of consecutive matrices (about equal weight bytes), each launched on its
+ * own, so that the copy of X into chunk c + 1, the computation of chunk c and the copy
+ * of Y out of chunk c - 1 overlap (two internal streams, ordered with `stream` by
+ * events: the call is ordered after earlier work on `stream`, and later work on `stream`
+ * sees all of Y copied out). The first such call builds the chunks (synchronous: it
+ * allocates their descriptor tables and X-piece scratch, so not during stream capture).
+ * Each chunk is scheduled on its own, so where the whole-stack run cuts an n-tile across
+ * CTAs the chunked run may cut it elsewhere: its results are deterministic and within the
+ * same tolerance, not always the same bits as tl_nvfp4_plan_run(). Destroy synchronises the
+ * device before freeing.
  * One plan must not run on two streams at once (the runs share the split-K workspace
  * of the device; runs on one stream are ordered). */
 typedef struct tl_nvfp4_plan_st* tl_nvfp4_plan;

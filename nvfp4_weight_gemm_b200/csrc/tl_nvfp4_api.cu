@@ -70,6 +70,12 @@ struct DevState {
 std::mutex g_mu;
 DevState g_dev[kMaxDevices];
 int g_path = TL_PATH_BLOCK_SCALED;   // which tensor-core path the GEMM entry points take
+
+// The path setting, read once per call or plan (never while g_mu is held).
+int current_path() {
+    std::lock_guard<std::mutex> lk(g_mu);
+    return g_path;
+}
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 tl_status load_encode_fn() {
@@ -278,9 +284,12 @@ tl_status stack_table(DevState& d, const std::vector<tl::TcMat>& mats, cudaStrea
 
 // Validate a stack and build its launch parameters (host side only, plus the
 // state lookup). `table_out` receives the TcMat array when n_mats > 1.
+// path: the GEMM path the parameters are for (the caller's copy of the setting, so that one
+// call or plan never mixes two paths).
 tl_status build_params(const tl_nvfp4_matrix* mats, int n_mats, int M, const unsigned char* x_dev,
-                       unsigned char* y_dev, DevState** dstate, tl::TcParams* p, std::vector<tl::TcMat>* table_out) {
-    tl_status st = check_M(M, g_path == TL_PATH_BLOCK_SCALED ? kBsMaxRows : kExactMaxRows);
+                       unsigned char* y_dev, int path, DevState** dstate, tl::TcParams* p,
+                       std::vector<tl::TcMat>* table_out) {
+    tl_status st = check_M(M, path == TL_PATH_BLOCK_SCALED ? kBsMaxRows : kExactMaxRows);
     if (st != TL_OK) return st;
     if (!mats) return fail(TL_ERR_INVALID_VALUE, "mats is null");
     if (n_mats < 1 || n_mats > TL_NVFP4_MAX_STACK)
@@ -303,7 +312,7 @@ tl_status build_params(const tl_nvfp4_matrix* mats, int n_mats, int M, const uns
     if (M == 0) return TL_OK;
     st = current_state(dstate);
     if (st != TL_OK) return st;
-    if (g_path == TL_PATH_BLOCK_SCALED) return TL_OK;   // the block-scaled launch builds its own tables
+    if (path == TL_PATH_BLOCK_SCALED) return TL_OK;     // the block-scaled launch builds its own tables
     const int NX = M <= 16 ? 16 : 32;
     std::vector<tl::TcMat>& tbl = *table_out;
     tbl.assign(n_mats, tl::TcMat());
@@ -339,7 +348,7 @@ tl_status run_stack_rows(const tl_nvfp4_matrix* mats, int n_mats, int M, const u
 // rows (rows r0 .. r0 + Mg - 1 of every X_i and Y_i), each group one launch.
 tl_status run_stack(const tl_nvfp4_matrix* mats, int n_mats, int M, const unsigned char* x_dev,
                     unsigned char* y_dev, void* stream_) {
-    const int lim = (g_path == TL_PATH_BLOCK_SCALED) ? kBsMaxRows : kExactMaxRows;
+    const int lim = (current_path() == TL_PATH_BLOCK_SCALED) ? kBsMaxRows : kExactMaxRows;
     if (M <= lim) return run_stack_rows(mats, n_mats, M, x_dev, y_dev, stream_);
     tl_status st = check_M(M);
     if (st != TL_OK) return st;
@@ -379,9 +388,10 @@ tl_status run_stack_rows(const tl_nvfp4_matrix* mats, int n_mats, int M, const u
     DevState* d = nullptr;
     tl::TcParams p;
     std::vector<tl::TcMat> tbl;
-    tl_status st = build_params(mats, n_mats, M, x_dev, y_dev, &d, &p, &tbl);
+    const int path = current_path();
+    tl_status st = build_params(mats, n_mats, M, x_dev, y_dev, path, &d, &p, &tbl);
     if (st != TL_OK || M == 0) return st;
-    if (g_path == TL_PATH_BLOCK_SCALED) return run_stack_bs(mats, n_mats, M, x_dev, y_dev, stream_, d);
+    if (path == TL_PATH_BLOCK_SCALED) return run_stack_bs(mats, n_mats, M, x_dev, y_dev, stream_, d);
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
     if (n_mats > 1) {
         st = stack_table(*d, tbl, stream, &p.mats);
@@ -844,6 +854,16 @@ struct tl_nvfp4_plan_st {
     const void* x_base = nullptr;     // packed X_i buffer (or nullptr if not packed)
     void* y_base = nullptr;           // packed Y_i buffer (or nullptr if not packed)
     size_t x_bytes = 0, y_bytes = 0;
+    // Host-buffer runs, pipelined: the stack cut into chunks of consecutive matrices, each a
+    // plan of its own, so that copying X of chunk c + 1 in, computing chunk c and copying Y of
+    // chunk c - 1 out overlap (built at the first tl_nvfp4_plan_run_host).
+    int M = 0;
+    std::vector<tl_nvfp4_matrix> mats;          // copy of the descriptors (device pointers)
+    bool chunks_built = false;
+    std::vector<tl_nvfp4_plan_st*> chunks;
+    std::vector<size_t> cx_off, cx_len, cy_off, cy_len;
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    std::vector<cudaEvent_t> ev;               // start, done, then per chunk: X in, computed
 };
 
 namespace {
@@ -878,29 +898,78 @@ tl_status plan_build_bs(tl_nvfp4_plan plan, const tl_nvfp4_matrix* mats, int n_m
 }
 
 tl_status plan_launch(tl_nvfp4_plan plan, cudaStream_t s) {
-    if (plan->path == TL_PATH_BLOCK_SCALED) return launch_bs(*plan->d, plan->bparams, plan->xparams, plan->grid, s);
+    if (plan->path == TL_PATH_BLOCK_SCALED) {
+        if (plan->grid < 1 || !plan->bparams.segs) return fail(TL_ERR_DEVICE_FAULT, "internal: plan without a schedule");
+        return launch_bs(*plan->d, plan->bparams, plan->xparams, plan->grid, s);
+    }
+    if (plan->params.n_mats < 1 || plan->params.total_tiles < 1 || (plan->params.n_mats > 1 && !plan->params.mats))
+        return fail(TL_ERR_DEVICE_FAULT, "internal: plan without descriptors");
     tl::TcParams p = plan->params;
     return launch_tc_any(*plan->d, p, s);
 }
 
-}  // namespace
+tl_status plan_create_path(const tl_nvfp4_matrix* mats, int n_mats, int M, int path, tl_nvfp4_plan* plan_out);
 
-extern "C" {
+// Chunks of a host-buffer run: up to kHostChunks groups of consecutive matrices with about
+// equal weight bytes, each its own plan (same path), plus two copy streams and their events.
+constexpr int kHostChunks = 8;
 
-tl_status tl_nvfp4_plan_create(const tl_nvfp4_matrix* mats, int n_mats, int M, tl_nvfp4_plan* plan_out) {
+tl_status plan_build_chunks(tl_nvfp4_plan plan) {
+    plan->chunks_built = true;
+    const int n = (int)plan->mats.size();
+    const int C = std::min(kHostChunks, n);
+    if (C < 2) return TL_OK;
+    double total = 0.0;
+    for (const tl_nvfp4_matrix& m : plan->mats) total += (double)m.N * m.K;
+    std::vector<int> cut{0};
+    double acc = 0.0;
+    for (int i = 0; i + 1 < n && (int)cut.size() < C; ++i) {
+        acc += (double)plan->mats[i].N * plan->mats[i].K;
+        if (acc >= total * (double)cut.size() / C) cut.push_back(i + 1);
+    }
+    cut.push_back(n);
+    size_t xo = 0, yo = 0;
+    for (size_t c = 0; c + 1 < cut.size(); ++c) {
+        const int a = cut[c], b = cut[c + 1];
+        size_t xl = 0, yl = 0;
+        for (int i = a; i < b; ++i) {
+            xl += (size_t)2 * plan->M * plan->mats[i].K;
+            yl += (size_t)2 * plan->M * plan->mats[i].N;
+        }
+        tl_nvfp4_plan cp = nullptr;
+        tl_status st = plan_create_path(plan->mats.data() + a, b - a, plan->M, plan->path, &cp);
+        if (st != TL_OK) return st;
+        plan->chunks.push_back(cp);
+        plan->cx_off.push_back(xo);
+        plan->cx_len.push_back(xl);
+        plan->cy_off.push_back(yo);
+        plan->cy_len.push_back(yl);
+        xo += xl;
+        yo += yl;
+    }
+    TL_CUDA(cudaStreamCreateWithFlags(&plan->s_in, cudaStreamNonBlocking));
+    TL_CUDA(cudaStreamCreateWithFlags(&plan->s_out, cudaStreamNonBlocking));
+    plan->ev.assign(2 + 2 * plan->chunks.size(), nullptr);
+    for (cudaEvent_t& e : plan->ev) TL_CUDA(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+    return TL_OK;
+}
+
+tl_status plan_create_path(const tl_nvfp4_matrix* mats, int n_mats, int M, int path, tl_nvfp4_plan* plan_out) {
     if (!plan_out) return fail(TL_ERR_INVALID_VALUE, "plan_out is null");
     *plan_out = nullptr;
     if (M == 0) return fail(TL_ERR_INVALID_VALUE, "a plan needs M >= 1");
     DevState* d = nullptr;
     tl::TcParams p;
     std::vector<tl::TcMat> tbl;
-    tl_status st = build_params(mats, n_mats, M, nullptr, nullptr, &d, &p, &tbl);
+    tl_status st = build_params(mats, n_mats, M, nullptr, nullptr, path, &d, &p, &tbl);
     if (st != TL_OK) return st;
     tl_nvfp4_plan plan = new tl_nvfp4_plan_st();
     TL_CUDA(cudaGetDevice(&plan->device));
     plan->d = d;
     plan->params = p;
-    plan->path = g_path;
+    plan->path = path;
+    plan->M = M;
+    plan->mats.assign(mats, mats + n_mats);
     if (plan->path == TL_PATH_BLOCK_SCALED) {
         st = plan_build_bs(plan, mats, n_mats, M);
         if (st != TL_OK) {
@@ -933,6 +1002,16 @@ tl_status tl_nvfp4_plan_create(const tl_nvfp4_matrix* mats, int n_mats, int M, t
     return TL_OK;
 }
 
+}  // namespace
+
+extern "C" {
+
+tl_status tl_nvfp4_plan_create(const tl_nvfp4_matrix* mats, int n_mats, int M, tl_nvfp4_plan* plan_out) {
+    if (!plan_out) return fail(TL_ERR_INVALID_VALUE, "plan_out is null");
+    *plan_out = nullptr;
+    return plan_create_path(mats, n_mats, M, current_path(), plan_out);
+}
+
 tl_status tl_nvfp4_plan_run(tl_nvfp4_plan plan, void* stream) {
     if (!plan) return fail(TL_ERR_INVALID_VALUE, "plan is null");
     return plan_launch(plan, static_cast<cudaStream_t>(stream));
@@ -944,15 +1023,61 @@ tl_status tl_nvfp4_plan_run_host(tl_nvfp4_plan plan, const void* x_host, void* y
     if (!plan->x_base || !plan->y_base)
         return fail(TL_ERR_INVALID_VALUE, "the plan's X and Y buffers are not packed back to back");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    TL_CUDA(cudaMemcpyAsync(const_cast<void*>(plan->x_base), x_host, plan->x_bytes, cudaMemcpyHostToDevice, s));
-    tl_status st = plan_launch(plan, s);
-    if (st != TL_OK) return st;
-    TL_CUDA(cudaMemcpyAsync(y_host, plan->y_base, plan->y_bytes, cudaMemcpyDeviceToHost, s));
+    if (!plan->chunks_built) {
+        tl_status st = plan_build_chunks(plan);
+        if (st != TL_OK) return st;
+    }
+    if (plan->chunks.empty()) {
+        TL_CUDA(cudaMemcpyAsync(const_cast<void*>(plan->x_base), x_host, plan->x_bytes, cudaMemcpyHostToDevice, s));
+        tl_status st = plan_launch(plan, s);
+        if (st != TL_OK) return st;
+        TL_CUDA(cudaMemcpyAsync(y_host, plan->y_base, plan->y_bytes, cudaMemcpyDeviceToHost, s));
+        return TL_OK;
+    }
+    // X of every chunk in on s_in; chunk c computed on `stream` once its X is in; its Y out on
+    // s_out once computed; `stream` resumes after the last Y is out.
+    const unsigned char* xh = static_cast<const unsigned char*>(x_host);
+    unsigned char* yh = static_cast<unsigned char*>(y_host);
+    unsigned char* xd = static_cast<unsigned char*>(const_cast<void*>(plan->x_base));
+    unsigned char* yd = static_cast<unsigned char*>(plan->y_base);
+    const size_t C = plan->chunks.size();
+    cudaEvent_t e_start = plan->ev[0], e_done = plan->ev[1];
+    TL_CUDA(cudaEventRecord(e_start, s));
+    TL_CUDA(cudaStreamWaitEvent(plan->s_in, e_start, 0));
+    TL_CUDA(cudaStreamWaitEvent(plan->s_out, e_start, 0));
+    for (size_t c = 0; c < C; ++c) {
+        TL_CUDA(cudaMemcpyAsync(xd + plan->cx_off[c], xh + plan->cx_off[c], plan->cx_len[c], cudaMemcpyHostToDevice,
+                                plan->s_in));
+        TL_CUDA(cudaEventRecord(plan->ev[2 + 2 * c], plan->s_in));
+    }
+    for (size_t c = 0; c < C; ++c) {
+        TL_CUDA(cudaStreamWaitEvent(s, plan->ev[2 + 2 * c], 0));
+        tl_status st = plan_launch(plan->chunks[c], s);
+        if (st != TL_OK) return st;
+        TL_CUDA(cudaEventRecord(plan->ev[3 + 2 * c], s));
+        TL_CUDA(cudaStreamWaitEvent(plan->s_out, plan->ev[3 + 2 * c], 0));
+        TL_CUDA(cudaMemcpyAsync(yh + plan->cy_off[c], yd + plan->cy_off[c], plan->cy_len[c], cudaMemcpyDeviceToHost,
+                                plan->s_out));
+    }
+    TL_CUDA(cudaEventRecord(e_done, plan->s_out));
+    TL_CUDA(cudaStreamWaitEvent(s, e_done, 0));
     return TL_OK;
 }
 
 tl_status tl_nvfp4_plan_destroy(tl_nvfp4_plan plan) {
     if (!plan) return TL_OK;
+    for (tl_nvfp4_plan cp : plan->chunks) tl_nvfp4_plan_destroy(cp);
+    if (plan->s_in || plan->s_out || !plan->ev.empty()) {
+        int prev = 0;
+        cudaGetDevice(&prev);
+        cudaSetDevice(plan->device);
+        cudaDeviceSynchronize();
+        for (cudaEvent_t e : plan->ev)
+            if (e) cudaEventDestroy(e);
+        if (plan->s_in) cudaStreamDestroy(plan->s_in);
+        if (plan->s_out) cudaStreamDestroy(plan->s_out);
+        cudaSetDevice(prev);
+    }
     if (plan->table || plan->bs_tables || plan->xs) {
         int prev = 0;
         cudaGetDevice(&prev);

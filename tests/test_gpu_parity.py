@@ -519,6 +519,54 @@ def test_stack_host_buffers_end_to_end(path):
         off += n
 
 
+@pytest.mark.parametrize("path", list(TC_PATHS))
+@pytest.mark.parametrize("M", [3, 17])
+def test_plan_host_buffers_pipelined(M, path):
+    # a plan's host-buffer run copies X in, computes and copies Y out in overlapping chunks of
+    # matrices (each chunk its own launch, scheduled on its own): within tolerance of the oracle,
+    # like the plan's device run, and the same bits on every run
+    ents, refs = _small_stack(M, n_layers=3)
+    xtot = sum(e[3].numel() for e in ents)
+    ytot = sum(e[4].numel() for e in ents)
+    x_dev = torch.empty(xtot, dtype=torch.bfloat16, device=DEV)
+    y_dev = torch.empty(ytot, dtype=torch.bfloat16, device=DEV)
+    packed, xo, yo = [], 0, 0
+    for (c, s, g, x, y) in ents:
+        xv = x_dev[xo:xo + x.numel()].view(x.shape)
+        xv.copy_(x)
+        packed.append((c, s, g, xv, y_dev[yo:yo + y.numel()].view(y.shape)))
+        xo += x.numel()
+        yo += y.numel()
+    x_host = x_dev.cpu().pin_memory()
+    y_host = torch.empty(ytot, dtype=torch.bfloat16).pin_memory()
+    with tl.gemm_path(TC_PATHS[path]):
+        plan = tl.Plan(packed, M)
+    try:
+        plan.run()
+        torch.cuda.synchronize()
+        y_dev_run = y_dev.cpu()
+        y_dev.zero_()
+        x_dev.zero_()
+        first = None
+        for _ in range(2):
+            y_host.zero_()
+            plan.run_host(x_host, y_host)
+            torch.cuda.synchronize()
+            tl.check_device_error()
+            if first is None:
+                first = y_host.clone()
+            assert torch.equal(y_host, first), "host-buffer runs differ"
+        off = 0
+        for (c, s, g, x, y), (y_ref, a_ref, _) in zip(ents, refs):
+            n = y.numel()
+            for name, buf in (("host", y_host), ("device", y_dev_run)):
+                got = buf[off:off + n].view(y.shape).float().numpy().astype(np.float64)
+                assert_within_tol(got, y_ref, a_ref, f"plan {name} M={M} [{path}]")
+            off += n
+    finally:
+        plan.close()
+
+
 # ------------------------------------------------------------------ failure path
 
 def test_bounded_wait_reports_timeout_and_context_survives():
