@@ -914,20 +914,28 @@ tl_status plan_create_path(const tl_nvfp4_matrix* mats, int n_mats, int M, int p
 // equal weight bytes, each its own plan (same path), plus two copy streams and their events.
 constexpr int kHostChunks = 8;
 
-tl_status plan_build_chunks(tl_nvfp4_plan plan) {
-    plan->chunks_built = true;
-    const int n = (int)plan->mats.size();
-    const int C = std::min(kHostChunks, n);
-    if (C < 2) return TL_OK;
+// Chunk boundaries of a host-buffer run over n matrices: 0 = cut[0] < cut[1] < ... < cut[C] = n,
+// C = min(chunks, n) groups of consecutive matrices, a group ending where the running weight
+// count (N x K) first reaches its share of the total.
+std::vector<int> host_chunk_cuts(const tl_nvfp4_matrix* mats, int n, int chunks) {
+    const int C = std::min(chunks, n);
     double total = 0.0;
-    for (const tl_nvfp4_matrix& m : plan->mats) total += (double)m.N * m.K;
+    for (int i = 0; i < n; ++i) total += (double)mats[i].N * mats[i].K;
     std::vector<int> cut{0};
     double acc = 0.0;
     for (int i = 0; i + 1 < n && (int)cut.size() < C; ++i) {
-        acc += (double)plan->mats[i].N * plan->mats[i].K;
+        acc += (double)mats[i].N * mats[i].K;
         if (acc >= total * (double)cut.size() / C) cut.push_back(i + 1);
     }
     cut.push_back(n);
+    return cut;
+}
+
+tl_status plan_build_chunks(tl_nvfp4_plan plan) {
+    plan->chunks_built = true;
+    const int n = (int)plan->mats.size();
+    if (std::min(kHostChunks, n) < 2) return TL_OK;
+    const std::vector<int> cut = host_chunk_cuts(plan->mats.data(), n, kHostChunks);
     size_t xo = 0, yo = 0;
     for (size_t c = 0; c + 1 < cut.size(); ++c) {
         const int a = cut[c], b = cut[c + 1];

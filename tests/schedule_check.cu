@@ -2,8 +2,9 @@
 // every k-tile of every n-tile is covered exactly once, split n-tiles carry consistent ranks,
 // part counts, consecutive partial slots and k order, the workspace limits hold, the work per
 // CTA (in 256-row units times k-tiles) is balanced, and the k ranges of every weight row are the
-// same with 128-row and with 256-row n-tiles (so outputs do not depend on the launch). Built and
-// run by tests/test_schedule.py; no GPU is touched.
+// same with 128-row and with 256-row n-tiles (so outputs do not depend on the launch); and the
+// chunks a host-buffer run cuts the stack into. Built and run by tests/test_schedule.py; no GPU
+// is touched.
 #include "../nvfp4_weight_gemm_b200/csrc/tl_nvfp4_api.cu"
 
 #include <algorithm>
@@ -114,6 +115,28 @@ static int same_cuts(const std::vector<std::pair<int, int>>& shapes, int grid) {
     return bad;
 }
 
+// Chunks of a host-buffer run: boundaries strictly increasing from 0 to n, at most
+// min(8, n) chunks; the 64-layer stack splits at every eighth of its layers.
+static int check_chunks(const std::vector<std::pair<int, int>>& shapes, const std::vector<int>* expect) {
+    std::vector<tl_nvfp4_matrix> mats;
+    for (auto& sh : shapes) {
+        tl_nvfp4_matrix m{};
+        m.N = sh.first;
+        m.K = sh.second;
+        mats.push_back(m);
+    }
+    const int n = (int)mats.size();
+    const std::vector<int> cut = host_chunk_cuts(mats.data(), n, kHostChunks);
+    int bad = 0;
+    if (cut.empty() || cut.front() != 0 || cut.back() != n) ++bad;
+    for (size_t i = 1; i < cut.size(); ++i)
+        if (cut[i] <= cut[i - 1]) ++bad;
+    if ((int)cut.size() - 1 > std::min(kHostChunks, n)) ++bad;
+    if (expect && cut != *expect) ++bad;
+    if (bad) printf("host-buffer chunks malformed for %d matrices\n", n);
+    return bad;
+}
+
 int main() {
     int bad = 0;
     std::vector<std::pair<int, int>> stack;
@@ -160,6 +183,26 @@ int main() {
             long long units = 0;
             for (auto& s2 : sh) units += (long long)((s2.first + 255) / 256) * (s2.second / 256);
             bad += same_cuts(sh, (int)std::min<long long>(units, 1 + rand() % 160));
+        }
+    }
+    {
+        std::vector<std::pair<int, int>> stack;
+        for (int l = 0; l < 64; ++l) {
+            stack.push_back({7168, 5120});
+            stack.push_back({5120, 5120});
+            stack.push_back({34816, 5120});
+            stack.push_back({5120, 17408});
+        }
+        std::vector<int> every8{0, 32, 64, 96, 128, 160, 192, 224, 256};
+        bad += check_chunks(stack, &every8);
+        bad += check_chunks({{677, 2304}}, nullptr);
+        bad += check_chunks({{256, 512}, {100000, 25600}, {128, 256}}, nullptr);
+        srand(13);
+        for (int it = 0; it < 300; ++it) {
+            std::vector<std::pair<int, int>> sh;
+            const int n = 1 + rand() % 300;
+            for (int i = 0; i < n; ++i) sh.push_back({1 + rand() % 40000, 256 * (1 + rand() % 100)});
+            bad += check_chunks(sh, nullptr);
         }
     }
     printf("bad=%d\n", bad);
