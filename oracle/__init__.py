@@ -4,6 +4,9 @@ TEST INFRASTRUCTURE ONLY. Only the tests, ``__graft_entry__.smoke()`` and the
 benchmark's CPU-baseline leg may import this package. The GPU library never
 imports it and shares no code with it.
 
+It also holds, in numpy fp64, the oracle of the next row: the FP8 output head's logits and the
+greedy top-2 / near-tie statistic (end of this file).
+
 The C source computes everything in fp64 from the format definitions:
 E2M1 codes (two per byte, low nibble = even k), one E4M3 scale per 16-element
 K block, one FP32 tensor scale; Y = X . dequant(W)^T. See the header of
@@ -157,3 +160,76 @@ def num_threads() -> int:
 
 def set_num_threads(n: int) -> None:
     lib().or_set_num_threads(int(n))
+
+
+# ---------------------------------------------------------------- FP8 output head (next row)
+#
+# The served weights keep the output head in FP8 (TandemLLM docs v0.12.0, "What TandemLLM is",
+# the paragraph on cutting the bytes a step reads), and the greedy output is exact up to near
+# ties, where the two best tokens are within one unit in the last place (same page, "the first
+# rule is agreement with greedy decoding"). Parity pinned by tests/test_oracle_pins.py.
+
+def fp8_head_logits(x_bits: np.ndarray, w_fp8: np.ndarray, scale) -> np.ndarray:
+    """Logits of an FP8 output head in fp64: L[m, n] = (sum_k x[m, k] * e4m3(w[n, k])) * s_n.
+
+    x_bits: bf16 bits uint16[M, K]; w_fp8: uint8[N, K] E4M3 bytes (0x7F / 0xFF decode to NaN,
+    which gives NaN logits); scale: one float (per tensor) or N floats (per output row): the
+    pages do not say which, so both are accepted. The sum is a library fp64 matrix product."""
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    w_fp8 = np.ascontiguousarray(w_fp8, dtype=np.uint8)
+    if x_bits.ndim != 2 or w_fp8.ndim != 2 or x_bits.shape[1] != w_fp8.shape[1]:
+        raise ValueError("x is [M, K] and w is [N, K]")
+    table = np.array([e4m3_decode(b) for b in range(256)], dtype=np.float64)
+    w = table[w_fp8]
+    x = (x_bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    logits = x @ w.T
+    s = np.asarray(scale, dtype=np.float64)
+    if s.ndim == 0:
+        return logits * s
+    if s.shape != (w_fp8.shape[0],):
+        raise ValueError("a per-row scale has one value per output row")
+    return logits * s[None, :]
+
+
+def bf16_ulp(v: float) -> float:
+    """Spacing of bf16 values at |v|: 2^(e - 7) for 2^e <= |v| < 2^(e + 1) with e >= -126 (eight
+    significand bits), the subnormal spacing 2^-133 below 2^-126; NaN for a non-finite v."""
+    a = abs(float(v))
+    if not np.isfinite(a):
+        return float("nan")
+    if a < 2.0 ** -126:
+        return 2.0 ** -133
+    e = int(np.floor(np.log2(a)))
+    # guard the floor of log2 at exact powers of two and just below them
+    if 2.0 ** e > a:
+        e -= 1
+    elif 2.0 ** (e + 1) <= a:
+        e += 1
+    return 2.0 ** (e - 7)
+
+
+def greedy_top2(logits: np.ndarray):
+    """Per row of logits[M, N] (N >= 2): the greedy token (largest logit, lowest index among
+    equal ones), the largest and second largest values, and their gap in bf16 units in the last
+    place at the largest value. The pages report near ties as gaps below one ulp (0.04 to 0.76
+    ulp measured), so the gap is read on logits finer than the ulp's format: here fp64 logits
+    against the bf16 spacing. A row with a NaN gives index -1 and NaN values."""
+    L = np.asarray(logits, dtype=np.float64)
+    if L.ndim != 2 or L.shape[1] < 2:
+        raise ValueError("logits is [M, N] with N >= 2")
+    M = L.shape[0]
+    idx = np.full(M, -1, dtype=np.int64)
+    top1 = np.full(M, np.nan)
+    top2 = np.full(M, np.nan)
+    gap = np.full(M, np.nan)
+    for m in range(M):
+        row = L[m]
+        if np.isnan(row).any():
+            continue
+        i = int(np.argmax(row))            # the first of equal maxima
+        rest = np.delete(row, i)
+        idx[m] = i
+        top1[m] = row[i]
+        top2[m] = rest.max()
+        gap[m] = (top1[m] - top2[m]) / bf16_ulp(top1[m])
+    return idx, top1, top2, gap

@@ -337,3 +337,81 @@ def test_gemm_sampled_equals_full(orc):
     mi, ni = rng.integers(0, 6, 50), rng.integers(0, 64, 50)
     ys, as_ = orc.gemm_sampled(x, codes, scales, g, mi, ni)
     assert np.array_equal(ys, y[mi, ni]) and np.array_equal(as_, a[mi, ni])
+
+
+# ---------------------------------------------------------------- FP8 output head (next row)
+
+def _bf16_bits(vals):
+    return torch.tensor(vals, dtype=torch.float32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def test_head_one_hot_rows_pick_x_columns(orc):
+    # W row n holds the E4M3 code of +1 (0x38) or -1 (0xB8) at column k_n, zeros elsewhere:
+    # logits[m, n] = +-x[m, k_n] * s_n exactly; catches a transposed W or a scale on the wrong axis
+    M, N, K = 3, 5, 7
+    rng = np.random.default_rng(3)
+    x = rng.integers(-8, 9, size=(M, K)).astype(np.float32) / 4.0
+    cols = [6, 0, 3, 3, 1]
+    signs = [1, -1, 1, -1, 1]
+    w = np.zeros((N, K), dtype=np.uint8)
+    for n, (k, sg) in enumerate(zip(cols, signs)):
+        w[n, k] = 0x38 if sg > 0 else 0xB8
+    s = np.array([1.0, 0.5, 2.0, 0.25, 8.0])
+    got = orc.fp8_head_logits(_bf16_bits(x), w, s)
+    for m in range(M):
+        for n in range(N):
+            assert got[m, n] == signs[n] * x[m, cols[n]] * s[n]
+    got1 = orc.fp8_head_logits(_bf16_bits(x), w, 0.5)
+    assert np.array_equal(got1, orc.fp8_head_logits(_bf16_bits(x), w, np.full(N, 0.5)))
+
+
+def test_head_brute_force_exact_rationals(orc):
+    # tiny random case against exact rational sums, E4M3 decoded by torch's float8_e4m3fn
+    M, N, K = 2, 3, 5
+    rng = np.random.default_rng(11)
+    x = (rng.standard_normal((M, K)) * 3).astype(np.float32)
+    xb = _bf16_bits(x)
+    w = rng.integers(0, 256, size=(N, K)).astype(np.uint8)
+    w[(w & 0x7F) == 0x7F] = 0x3A                      # no NaN codes here
+    wv = torch.from_numpy(w).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    xv = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    s = np.array([0.75, 1.0 / 3.0, 5.0])
+    got = orc.fp8_head_logits(xb, w, s)
+    for m in range(M):
+        for n in range(N):
+            exact = sum(Fraction(float(xv[m, k])) * Fraction(float(wv[n, k])) for k in range(K)) * Fraction(float(s[n]))
+            assert abs(Fraction(float(got[m, n])) - exact) <= abs(exact) * Fraction(1, 2 ** 50) + Fraction(1, 2 ** 200)
+
+
+def test_head_nan_codes_give_nan_logits(orc):
+    w = np.array([[0x38, 0x7F], [0x38, 0x38]], dtype=np.uint8)
+    got = orc.fp8_head_logits(_bf16_bits(np.array([[1.0, 1.0]])), w, 1.0)
+    assert math.isnan(got[0, 0]) and got[0, 1] == 2.0
+
+
+def test_bf16_ulp_matches_torch_nextafter(orc):
+    vals = [1.0, 1.5, 2.0, 3.0, -3.0, 0.1, 1e-3, 448.0, 65504.0, 3.0e38, 2.0 ** -126, 2.0 ** -130]
+    for v in vals:
+        b = torch.tensor(v, dtype=torch.bfloat16)
+        up = torch.nextafter(b.abs(), torch.tensor(float("inf"), dtype=torch.bfloat16))
+        assert orc.bf16_ulp(float(b)) == float(up.double() - b.abs().double()), v
+    assert orc.bf16_ulp(0.0) == 2.0 ** -133
+    assert math.isnan(orc.bf16_ulp(float("inf")))
+
+
+def test_greedy_top2_hand_worked(orc):
+    logits = np.array([
+        [1.0, 1.0 + 2.0 ** -9, 0.5],      # best is index 1; gap 2^-9 in ulps of 2^-7: 0.25
+        [2.0, 2.0, 1.0],                  # equal maxima: the lower index, gap 0
+        [-1.0, -2.0, -5.0],               # gap 1 in ulps of 2^-7 at -1: 128
+        [0.0, 3.0, 2.9375],               # gap 0.0625 in ulps of 2^-6 at 3: 4
+        [1.0, float("nan"), 0.0],         # a NaN row
+    ])
+    idx, t1, t2, gap = orc.greedy_top2(logits)
+    assert list(idx) == [1, 0, 0, 1, -1]
+    assert list(t1[:4]) == [1.0 + 2.0 ** -9, 2.0, -1.0, 3.0]
+    assert list(t2[:4]) == [1.0, 2.0, -2.0, 2.9375]
+    assert list(gap[:4]) == [0.25, 0.0, 128.0, 4.0]
+    assert math.isnan(gap[4]) and math.isnan(t1[4])
+    with pytest.raises(ValueError):
+        orc.greedy_top2(np.zeros((2, 1)))
