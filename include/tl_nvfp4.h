@@ -55,7 +55,7 @@ typedef enum {
     TL_OK = 0,
     TL_ERR_INVALID_VALUE = 1,   /* a size or pointer argument is out of range */
     TL_ERR_MISALIGNED = 2,      /* a pointer is not 16-byte aligned */
-    TL_ERR_UNSUPPORTED = 3,     /* valid request this build does not serve (e.g. M > 128) */
+    TL_ERR_UNSUPPORTED = 3,     /* valid request this library does not serve (e.g. M > 128) */
     TL_ERR_CUDA = 4,            /* a CUDA runtime/driver call failed */
     TL_ERR_TIMEOUT = 5,         /* a device-side wait ran past its iteration limit */
     TL_ERR_NOT_INITIALIZED = 6, /* no usable device / state */
