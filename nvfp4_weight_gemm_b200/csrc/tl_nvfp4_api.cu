@@ -931,11 +931,27 @@ std::vector<int> host_chunk_cuts(const tl_nvfp4_matrix* mats, int n, int chunks)
     return cut;
 }
 
+// Builds the chunks, their streams and events all at once: on any failure nothing is kept (the
+// next host-buffer run tries again).
 tl_status plan_build_chunks(tl_nvfp4_plan plan) {
-    plan->chunks_built = true;
     const int n = (int)plan->mats.size();
-    if (std::min(kHostChunks, n) < 2) return TL_OK;
+    if (std::min(kHostChunks, n) < 2) {
+        plan->chunks_built = true;
+        return TL_OK;
+    }
     const std::vector<int> cut = host_chunk_cuts(plan->mats.data(), n, kHostChunks);
+    std::vector<tl_nvfp4_plan> chunks;
+    std::vector<size_t> cx_off, cx_len, cy_off, cy_len;
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    std::vector<cudaEvent_t> ev(2 + 2 * (cut.size() - 1), nullptr);
+    auto undo = [&](tl_status st) {
+        for (tl_nvfp4_plan cp : chunks) tl_nvfp4_plan_destroy(cp);
+        for (cudaEvent_t e : ev)
+            if (e) cudaEventDestroy(e);
+        if (s_in) cudaStreamDestroy(s_in);
+        if (s_out) cudaStreamDestroy(s_out);
+        return st;
+    };
     size_t xo = 0, yo = 0;
     for (size_t c = 0; c + 1 < cut.size(); ++c) {
         const int a = cut[c], b = cut[c + 1];
@@ -946,19 +962,30 @@ tl_status plan_build_chunks(tl_nvfp4_plan plan) {
         }
         tl_nvfp4_plan cp = nullptr;
         tl_status st = plan_create_path(plan->mats.data() + a, b - a, plan->M, plan->path, &cp);
-        if (st != TL_OK) return st;
-        plan->chunks.push_back(cp);
-        plan->cx_off.push_back(xo);
-        plan->cx_len.push_back(xl);
-        plan->cy_off.push_back(yo);
-        plan->cy_len.push_back(yl);
+        if (st != TL_OK) return undo(st);
+        chunks.push_back(cp);
+        cx_off.push_back(xo);
+        cx_len.push_back(xl);
+        cy_off.push_back(yo);
+        cy_len.push_back(yl);
         xo += xl;
         yo += yl;
     }
-    TL_CUDA(cudaStreamCreateWithFlags(&plan->s_in, cudaStreamNonBlocking));
-    TL_CUDA(cudaStreamCreateWithFlags(&plan->s_out, cudaStreamNonBlocking));
-    plan->ev.assign(2 + 2 * plan->chunks.size(), nullptr);
-    for (cudaEvent_t& e : plan->ev) TL_CUDA(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+    if (cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking) != cudaSuccess)
+        return undo(fail(TL_ERR_CUDA, "creating the host-buffer run's streams failed"));
+    for (cudaEvent_t& e : ev)
+        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess)
+            return undo(fail(TL_ERR_CUDA, "creating the host-buffer run's events failed"));
+    plan->chunks = std::move(chunks);
+    plan->cx_off = std::move(cx_off);
+    plan->cx_len = std::move(cx_len);
+    plan->cy_off = std::move(cy_off);
+    plan->cy_len = std::move(cy_len);
+    plan->s_in = s_in;
+    plan->s_out = s_out;
+    plan->ev = std::move(ev);
+    plan->chunks_built = true;
     return TL_OK;
 }
 
