@@ -389,6 +389,12 @@ def main_gpu(args):
                              "gbs": round(gbs, 1), "frac": round(gbs / peak, 4),
                              "w_only_gbs": round(w_bytes(shapes) / (per_M[M] * 1e-3) / 1e9, 1)}
         cb, cs, cthreads = cpu_sample(CPU_ROWS, 32)
+        # what this staircase implies for the draft-tree size (host-side summary, after timing)
+        try:
+            from nvfp4_weight_gemm_b200 import staircut
+            cut = staircut.report(staircut.Staircase({M: per_M[M] for M in M_SWEEP}))
+        except Exception as exc:  # a summary only: it never fails the run
+            cut = {"error": str(exc)[:200]}
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 3), "higher_is_better": True,
@@ -402,6 +408,7 @@ def main_gpu(args):
             "staircase": stair,
             "min_frac_over_M": round(min(v["frac"] for v in stair.values()), 4),
             "m_invariance_row_fraction": inv,
+            "staircut": cut,
             "cpu_baseline": {"value": round(cb / cs / 1e9, 4), "unit": "GB/s", "cores": cthreads, "kind": "oracle",
                              "sample": CPU_SAMPLE_DESC},
             "e2e": {"value": round(job_gbs(world, bytes_step, e2e_ms), 1), "unit": "GB/s",

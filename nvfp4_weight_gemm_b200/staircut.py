@@ -111,3 +111,16 @@ def choose(parents: Sequence[int], accept: Sequence[float], stair: Staircase, ov
             best = c
     assert best is not None
     return best
+
+
+def report(stair: Staircase, overhead_ms: float = 0.0, accept: Sequence[float] = (0.3, 0.5, 0.7, 0.9),
+           n_nodes: int = 40) -> Dict[str, Dict[str, float]]:
+    """The cut chosen on `stair` for chains of `n_nodes` drafts each accepted with probability p
+    given its parent, for each p: a summary of what the staircase implies for the tree size."""
+    out: Dict[str, Dict[str, float]] = {}
+    parents = [-1] + list(range(n_nodes - 1))
+    for p in accept:
+        c = choose(parents, [p] * n_nodes, stair, overhead_ms)
+        out[f"p={p:g}"] = {"nodes": c.size, "rows": c.rows, "tokens": round(c.tokens, 4),
+                           "ms": round(c.ms, 4), "tokens_per_ms": round(c.tokens_per_ms, 4)}
+    return out

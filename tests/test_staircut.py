@@ -105,3 +105,12 @@ def test_invalid_trees_are_refused():
         sc.path_probs([-1], [1.5])                   # acceptance outside [0, 1]
     with pytest.raises(ValueError):
         sc.path_probs([-1, 0], [0.5])                # lengths differ
+
+
+def test_report_on_a_staircase():
+    flat = sc.Staircase({m: 2.0 for m in range(1, 33)})
+    r = sc.report(flat)
+    assert set(r) == {"p=0.3", "p=0.5", "p=0.7", "p=0.9"}
+    assert all(v["nodes"] == 31 and v["rows"] == 32 for v in r.values())   # flat price: the largest tree
+    r2 = sc.report(GB10)
+    assert all(v["nodes"] in sc.SNAP_NODES and v["nodes"] != 7 for v in r2.values())
