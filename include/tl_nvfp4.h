@@ -30,9 +30,10 @@
  * stream) and do not synchronise, unless stated. The library keeps one small
  * per-device state (split-K workspace, error word, descriptor cache) created
  * by tl_init() or lazily by the first call on a device; call tl_init() before
- * capturing a stream into a CUDA graph. The host side of every entry point is
+ * capturing a stream into a CUDA graph (see "Allocation" below for when else a call
+ * without a plan allocates). The host side of every entry point is
  * thread-safe. On the GPU, launches of one device share its workspace (split-K
- * partials and counters, the X pieces of calls made without a plan): calls whose
+ * partials and counters, the prepared X or X pieces of calls made without a plan): calls whose
  * kernels could overlap (different streams, or host threads without ordering)
  * must be serialised by the caller, e.g. by issuing them on one stream.
  *
@@ -77,33 +78,56 @@ typedef enum {
  * tl_nvfp4_verify_stack_host() and of plans (a plan keeps the path that was selected
  * when it was created). tl_nvfp4_verify_gemm_noalloc() always takes TL_PATH_BF16_EXACT.
  *
- * TL_PATH_BLOCK_SCALED (the default). Before the GEMM, a small kernel writes each row of
- * X as a power of two times a sum of four NVFP4-shaped pieces (E2M1 codes with one E4M3
- * scale per 16 k; each piece codes what the pieces before it left over). The GEMM then
- * feeds the weights' codes and scales and those pieces straight into the FP4
- * block-scaled tensor-core MMA, which decodes on the fly: no CUDA-core work per weight.
- * Accuracy: each X element is represented to within (1.125/6)^4 (about 1.24e-3) of the
- * largest |x| of its 16-element block, plus a floor about 2^-20 below the row's largest
- * |x|. Spread over a dense row of W, as in real weights, that keeps Y within
- * |y - y_ref| <= 1e-3 * sum_k |x w| + 2^-8 |y_ref| of the exact product (the pages'
- * workload shapes and distributions are tested). A row of W with very few nonzero
- * weights (an identity or one-hot matrix) can exceed that bound on an X element that is
- * much smaller than its block's largest: use TL_PATH_BF16_EXACT for such weights. Reduction
- * order is fixed, so runs are bit-identical, and a row's result does not depend on M. A
- * row of X holding a NaN or an infinity gives NaN outputs for the whole row. The path
- * needs scratch for the pieces, (4 * K/2 + 4 * K/16) * M + 4 * M bytes per matrix (256-byte
- * aligned parts), allocated by the first call of a size (outside stream capture) and
- * kept, or owned by a plan.
+ * TL_PATH_EXACT (the default). Exact operands on the f16 tensor-core MMA, fp32 accumulate:
+ *   - W: CUDA cores turn each byte of codes into two f16 E2M1 values (hardware convert) and
+ *     multiply by the block's E4M3 scale in f16. W' = e2m1 * e4m3 has at most 6 significant
+ *     bits and lies in [2^-10, 2688], so it is exact in f16.
+ *   - X: a small kernel first writes each row of X as f16(x * 2^-e_m), with e_m chosen so the
+ *     row's largest |x| lands in [2^15, 2^16); every bf16 value within about 32 binades of
+ *     the row's largest is then exact in f16. The epilogue multiplies row m by
+ *     global_scale * 2^e_m. A row the kernel cannot reproduce exactly (a wider range, a NaN or
+ *     infinity, or a largest |x| outside 2^-45 .. 2^75) is recomputed after the GEMM by an
+ *     fp64 CUDA-core kernel from the bf16 X as given (slow, but such rows do not occur in
+ *     activations). So every product is exact and only the fp32 sums round:
+ *     |y - y_ref| <= 1e-3 * sum_k |x w| + 2^-8 |y_ref| holds for every input, and results
+ *     are bit-exact wherever the exact result and its partial sums are representable.
+ *   Needs scratch for the prepared X: 2*M*K bytes + 4*M + 256 bytes per matrix (each part
+ *   rounded up to 256 bytes), owned by a plan, or (calls without a plan) one per-device
+ *   buffer that grows to the largest size used (see "Allocation" below).
  *
- * TL_PATH_BF16_EXACT. CUDA cores decode each weight to bf16 (exact: an E2M1 value times
- * an E4M3 scale has at most 6 significant bits) and the bf16 tensor-core MMA takes it
- * with X as given, so products are exact and only the fp32 sums round. Slower: the
- * decode is CUDA-core bound.
+ * TL_PATH_BF16_EXACT. The same exact arithmetic with the bf16 MMA: CUDA cores decode each
+ * weight to bf16 with integer bit operations and X is used as given (no preparation, no
+ * scratch). About half as fast: its decode is bound by the integer pipe.
  *
+ * TL_PATH_BLOCK_SCALED (approximate; not the default). Before the GEMM, a small kernel
+ * writes each row of X as a power of two times a sum of four NVFP4-shaped pieces (E2M1
+ * codes with one E4M3 scale per 16 k; each piece codes what the pieces before it left
+ * over), and the GEMM feeds the weights' codes and scales and those pieces straight into
+ * the FP4 block-scaled MMA. It does NOT reproduce X exactly: each X element carries an
+ * error of up to about 1.24e-3 of the largest |x| of its 16-element block, so the
+ * per-element bound above is not guaranteed (a weight row with few nonzero weights, such as
+ * an identity or one-hot matrix, can exceed it on an X element much smaller than its block's
+ * largest). A row of X holding a NaN or an infinity gives NaN outputs for the whole row.
+ * Scratch for the pieces: (4 * K/2 + 4 * K/16) * M + 4 * M bytes per matrix.
+ *
+ * All three paths have a fixed reduction order (runs are bit-identical) and compute each
+ * row of Y independently of the other rows, so a row's result does not depend on M.
  * tl_set_gemm_path() returns TL_ERR_INVALID_VALUE for any other value. The setting is
- * process-wide; change it only while no call is in flight. */
+ * process-wide; change it only while no call is in flight.
+ *
+ * Allocation. Plans allocate everything they need when they are created. Calls without a
+ * plan (tl_nvfp4_verify_gemm, tl_nvfp4_verify_stack, tl_nvfp4_verify_stack_host) may allocate
+ * device memory, and then synchronise the device first, only (a) at the first call on a
+ * device (its per-device state), (b) when a call needs more path scratch than any earlier call
+ * (the buffer grows and is kept), and (c) when a stack's descriptor table is larger than the
+ * cache slot it lands in (eight slots; each grows to the largest table it has held, with a
+ * pinned host staging buffer of the same size). Once those sizes have been reached, calls
+ * neither allocate nor synchronise: a stack whose descriptors are not cached is uploaded with
+ * an asynchronous copy on the call's stream. None of (a)-(c) may happen during stream capture
+ * (the call returns TL_ERR_UNSUPPORTED): run each size once before capturing. */
 #define TL_PATH_BLOCK_SCALED 0
 #define TL_PATH_BF16_EXACT 1
+#define TL_PATH_EXACT 2
 tl_status tl_set_gemm_path(int path);
 int tl_get_gemm_path(void);
 
@@ -142,19 +166,27 @@ tl_status tl_nvfp4_verify_gemm_simt(const void* x, int M, const void* w_codes, c
  * device memory through their own pool and do not let a library call cudaMalloc. This
  * call allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
  *
- * Same arguments, rules, kernel and results as tl_nvfp4_verify_gemm(). Its split-K
- * scratch is one static device array inside this library, 5 MiB (partials for up to
- * 160 CTAs, their counters, a status word), which every GPU that loads the library holds
- * until the process exits. Limits: M <= 32 (larger M returns TL_ERR_UNSUPPORTED with a
+ * Same arguments and rules as tl_nvfp4_verify_gemm(); it always runs the TL_PATH_BF16_EXACT
+ * kernel (whatever tl_set_gemm_path() selected), with the same grid on GPUs of at most 160
+ * SMs, so its results are bit-identical to tl_nvfp4_verify_gemm() under TL_PATH_BF16_EXACT.
+ * Its split-K scratch is one static device array inside this library, 5 MiB (partials for
+ * up to 160 CTAs, their counters, a status word), which every GPU that loads the library
+ * holds until the process exits. Limits: M <= 32 (larger M returns TL_ERR_UNSUPPORTED with a
  * message); the grid is capped at 160 CTAs.
  *
- * The first call on a device does a one-time set-up with that device current (it looks up
- * the array's device address and the SM count); make that first call before capturing a
- * stream into a graph. Every call shares the one array and each launch clears its counters
- * first, so calls whose kernels overlap on the GPU (different streams, or several host
- * threads without ordering) race and give undefined results: keep them on one stream.
- * A device-side wait that runs out is recorded only in the array's own status word, not
- * reported by tl_check_device_error(). */
+ * When the memory is taken. The array belongs to the library's CUDA module, which the CUDA
+ * runtime loads onto a device the first time the library touches that device (lazily, the
+ * default since CUDA 12.2). For a caller that uses only this entry point that is the first
+ * call, whose one-time set-up (with the device current: the array's device address and the
+ * SM count) loads the module: the array and the module's code are allocated then, by the
+ * runtime. Make that first call at start-up, before handing free memory to a pool, and
+ * before capturing a stream into a graph. Later calls take no device memory.
+ *
+ * Every call shares the one array and each launch clears its counters first, so calls whose
+ * kernels overlap on the GPU (different streams, or several host threads without ordering)
+ * race and give undefined results: keep them on one stream. A device-side wait that runs out
+ * is recorded in the array's status word, which tl_noalloc_check_error() (allocation-free)
+ * and tl_check_device_error() read and clear. */
 tl_status tl_nvfp4_verify_gemm_noalloc(const void* x, int M, const void* w_codes, const void* w_scales,
                                        float global_scale, void* y, int N, int K, void* stream);
 
@@ -237,8 +269,16 @@ tl_status tl_nvfp4_quantize(const float* w, int N, int K, void* w_codes, void* w
                             float* global_scale_out, void* stream);
 
 /* Synchronise `stream`, then report and clear the device status word:
- * TL_OK, TL_ERR_TIMEOUT (a bounded wait ran out) or TL_ERR_DEVICE_FAULT. */
+ * TL_OK, TL_ERR_TIMEOUT (a bounded wait ran out) or TL_ERR_DEVICE_FAULT. Also reads and
+ * clears the status word of tl_nvfp4_verify_gemm_noalloc()'s static scratch on the current
+ * device. After a timeout it clears every split-K counter of the device. Creates the
+ * per-device state if the device has none (allocates). */
 tl_status tl_check_device_error(void* stream);
+
+/* The allocation-free check for callers of tl_nvfp4_verify_gemm_noalloc(): synchronise
+ * `stream`, then report and clear the status word of the static scratch on the current
+ * device (TL_OK if the entry point never ran there). Touches no other state. */
+tl_status tl_noalloc_check_error(void* stream);
 
 /* Self-test of the device-side failure path: launches one thread that waits, with the
  * library's bounded wait, on an mbarrier that nothing completes, for at most

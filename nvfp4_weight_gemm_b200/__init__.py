@@ -13,8 +13,8 @@ from . import _lib
 from ._lib import Matrix, TlError, check
 
 __all__ = ["verify_gemm", "verify_gemm_simt", "set_gemm_path", "get_gemm_path", "gemm_path", "PATH_BLOCK_SCALED",
-           "PATH_BF16_EXACT", "verify_stack", "verify_stack_host", "Plan", "dequant",
-           "quantize", "check_device_error", "init", "num_sms", "Matrix", "TlError"]
+           "PATH_BF16_EXACT", "PATH_EXACT", "verify_stack", "verify_stack_host", "Plan", "dequant",
+           "quantize", "check_device_error", "noalloc_check_error", "init", "num_sms", "Matrix", "TlError"]
 
 
 def _stream(stream):
@@ -37,12 +37,14 @@ def num_sms(device: int = 0) -> int:
 
 PATH_BLOCK_SCALED = _lib.TL_PATH_BLOCK_SCALED
 PATH_BF16_EXACT = _lib.TL_PATH_BF16_EXACT
+PATH_EXACT = _lib.TL_PATH_EXACT
 
 
 def set_gemm_path(path: int) -> None:
     """Select the tensor-core path of verify_gemm, verify_stack(_host) and new plans:
-    PATH_BLOCK_SCALED (default; FP4 block-scaled MMA, within the stated tolerance) or
-    PATH_BF16_EXACT (CUDA-core decode to bf16, exact products)."""
+    PATH_EXACT (default; exact f16 operands: hardware E2M1 decode, X prepared per row),
+    PATH_BF16_EXACT (exact bf16 operands, integer decode; slower) or PATH_BLOCK_SCALED
+    (approximate: X split into FP4 pieces for the block-scaled MMA)."""
     check(_lib.lib().tl_set_gemm_path(path))
 
 
@@ -163,3 +165,8 @@ def quantize(w, stream=None):
 
 def check_device_error(stream=None) -> None:
     check(_lib.lib().tl_check_device_error(_stream(stream)))
+
+
+def noalloc_check_error(stream=None) -> None:
+    """Status word of the no-allocation entry point's static scratch (allocation-free)."""
+    check(_lib.lib().tl_noalloc_check_error(_stream(stream)))

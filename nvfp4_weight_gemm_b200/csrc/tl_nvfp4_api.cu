@@ -21,6 +21,7 @@
 
 #include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
+#include "xprep.cuh"
 #include "gemm_bs.cuh"
 #include "kernels_aux.cuh"
 
@@ -45,11 +46,24 @@ tl_status fail(tl_status st, const char* fmt, ...) {
     } while (0)
 
 constexpr int kMaxDevices = 64;
+
+// Split-K counters of one device: four per split n-tile (one per 32-row quarter), at most
+// 2 * SMs splits (the block-scaled schedule's bound, checked in build_bs; the exact kernel
+// uses 4 per CTA). Allocated, and cleared after a device-side timeout, in full.
+constexpr int kSplitsPerSm = 2, kCountersPerSplit = 4;
+size_t counter_words(int sms) { return (size_t)kCountersPerSplit * kSplitsPerSm * sms; }
 constexpr int kStackCacheSlots = 8;
 
+// One slot of the descriptor-table cache. A slot's device buffer only grows (to the largest
+// table it has held); refilling it is an asynchronous copy from the slot's pinned staging
+// buffer on the caller's stream, so after the slots have grown no call allocates or
+// synchronises the device.
 struct StackCacheEntry {
-    std::vector<unsigned char> key;   // host bytes of a descriptor table
+    std::vector<unsigned char> key;   // host bytes of the table the slot holds
     void* table = nullptr;            // device copy
+    void* staging = nullptr;          // pinned host copy the refill reads
+    size_t cap = 0;                   // bytes of `table` and `staging`
+    cudaEvent_t copied = nullptr;     // recorded after the last refill copy
     unsigned long long last_use = 0;
 };
 
@@ -63,13 +77,15 @@ struct DevState {
     bool smem_attr_set = false;
     unsigned char* xs_buf = nullptr;   // X pieces of the block-scaled path (calls without a plan)
     size_t xs_cap = 0;
+    unsigned char* xh_buf = nullptr;   // prepared X of the exact path (calls without a plan)
+    size_t xh_cap = 0;
     StackCacheEntry cache[kStackCacheSlots];
     unsigned long long use_clock = 0;
 };
 
 std::mutex g_mu;
 DevState g_dev[kMaxDevices];
-int g_path = TL_PATH_BLOCK_SCALED;   // which tensor-core path the GEMM entry points take
+int g_path = TL_PATH_EXACT;   // which tensor-core path the GEMM entry points take
 
 // The path setting, read once per call or plan (never while g_mu is held).
 int current_path() {
@@ -114,13 +130,13 @@ tl_status init_locked(int device) {
         d.num_sms = sms;
         const size_t pbytes = (size_t)4 * sms * tl::BS_PART_ROWS * tl::TC_BLOCK_N * sizeof(float);
         if (cudaMalloc(&d.err, 64) != cudaSuccess || cudaMalloc(&d.partials, pbytes) != cudaSuccess ||
-            cudaMalloc(&d.counters, (size_t)8 * sms * sizeof(unsigned)) != cudaSuccess ||
+            cudaMalloc(&d.counters, counter_words(sms) * sizeof(unsigned)) != cudaSuccess ||
             cudaMalloc(&d.qscratch, 64) != cudaSuccess) {
             st = fail(TL_ERR_CUDA, "cudaMalloc of the per-device state failed");
             break;
         }
         if (cudaMemset(d.err, 0, 64) != cudaSuccess ||
-            cudaMemset(d.counters, 0, (size_t)8 * sms * sizeof(unsigned)) != cudaSuccess ||
+            cudaMemset(d.counters, 0, counter_words(sms) * sizeof(unsigned)) != cudaSuccess ||
             cudaDeviceSynchronize() != cudaSuccess) {
             st = fail(TL_ERR_CUDA, "initialising the per-device state failed");
             break;
@@ -184,8 +200,16 @@ tl_status encode_3d(CUtensorMap* tm, CUtensorMapDataType dt, const void* base, c
     return TL_OK;
 }
 
+// Scratch of the exact path for one matrix with M rows: the prepared X (f16 [M][K]), the row
+// factors (float [M]) and the row mask (one word), each part 256-byte aligned.
+size_t xh_bytes_of(int M, int K) {
+    return (((size_t)2 * M * K + 255) & ~size_t(255)) + (((size_t)4 * M + 255) & ~size_t(255)) + 256;
+}
+
+// xh: the matrix's exact-path scratch (xh_bytes_of bytes) for the f16 operands, or nullptr for
+// the bf16 decode (X used as given).
 tl_status build_mat(tl::TcMat* m, const void* x, int M, int NX, const void* codes, const void* scales, float g,
-                    void* y, int N, int K, long long tile_begin) {
+                    void* y, int N, int K, long long tile_begin, unsigned char* xh = nullptr) {
     memset(m, 0, sizeof *m);
     // All three maps are rank 3 so that one converged load instruction can issue them.
     // Codes and scales: {bytes per row, N rows, 1}; a tile box is 128 rows of one k-tile.
@@ -199,7 +223,19 @@ tl_status build_mat(tl::TcMat* m, const void* x, int M, int NX, const void* code
     // X viewed as {64 elements, M rows, K/64 slices}: one box {64, NX, 4} lands the four 64-k
     // slices of a tile one after another in shared memory, each NX rows x 128 B, swizzled;
     // rows >= M read zero.
-    st = encode_3d(&m->tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, {64, (cuuint64_t)M, k / 64}, {k * 2, 128},
+    if (xh) {
+        m->x = static_cast<const __nv_bfloat16*>(x);
+        m->xh = reinterpret_cast<__half*>(xh);
+        m->rowfac = reinterpret_cast<float*>(xh + (((size_t)2 * M * K + 255) & ~size_t(255)));
+        m->rowmask = reinterpret_cast<unsigned*>(reinterpret_cast<unsigned char*>(m->rowfac) +
+                                                 (((size_t)4 * M + 255) & ~size_t(255)));
+        m->codes = static_cast<const uint8_t*>(codes);
+        m->scales = static_cast<const uint8_t*>(scales);
+        m->g = g;
+        m->K = K;
+    }
+    st = encode_3d(&m->tm_x, xh ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                   xh ? static_cast<const void*>(xh) : x, {64, (cuuint64_t)M, k / 64}, {k * 2, 128},
                    {64, (cuuint32_t)NX, 4}, CU_TENSOR_MAP_SWIZZLE_128B, "X");
     if (st != TL_OK) return st;
     m->y = static_cast<__nv_bfloat16*>(y);
@@ -211,24 +247,35 @@ tl_status build_mat(tl::TcMat* m, const void* x, int M, int NX, const void* code
     return TL_OK;
 }
 
-template <int NX>
+template <int NX, bool F16>
 tl_status launch_tc(DevState& d, tl::TcParams& p, cudaStream_t stream) {
     using C = tl::TcCfg<NX>;
     // the attribute is per function; set for both variants on first use (idempotent, cheap)
-    TL_CUDA(cudaFuncSetAttribute(tl::gemm_tc_kernel<NX>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
+    TL_CUDA(cudaFuncSetAttribute(tl::gemm_tc_kernel<NX, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::SMEM_BYTES));
     const long long grid = p.total_tiles < d.num_sms ? p.total_tiles : d.num_sms;
     p.partials = d.partials;
     p.counters = d.counters;
     p.err = d.err;
     p.spread_mul = 0x1040u;
     p.scale_mul = 0x00100010u;
-    tl::gemm_tc_kernel<NX><<<(unsigned)grid, tl::TC_THREADS, C::SMEM_BYTES, stream>>>(p);
+    tl::gemm_tc_kernel<NX, F16><<<(unsigned)grid, tl::TC_THREADS, C::SMEM_BYTES, stream>>>(p);
     TL_CUDA(cudaGetLastError());
     return TL_OK;
 }
 
-tl_status launch_tc_any(DevState& d, tl::TcParams& p, cudaStream_t stream) {
-    return (p.M <= 16) ? launch_tc<16>(d, p, stream) : launch_tc<32>(d, p, stream);
+// The exact paths. bf16 decode: one GEMM launch on X as given. f16 decode: the X preparation
+// (one CTA per matrix), the GEMM on the prepared X, then the fallback for flagged rows (it
+// returns at once when no row is flagged).
+tl_status launch_tc_any(DevState& d, tl::TcParams& p, bool f16, cudaStream_t stream) {
+    if (!f16) return (p.M <= 16) ? launch_tc<16, false>(d, p, stream) : launch_tc<32, false>(d, p, stream);
+    tl::x_prep_kernel<<<(unsigned)p.n_mats, tl::XP_THREADS, 0, stream>>>(p);
+    TL_CUDA(cudaGetLastError());
+    tl_status st = (p.M <= 16) ? launch_tc<16, true>(d, p, stream) : launch_tc<32, true>(d, p, stream);
+    if (st != TL_OK) return st;
+    tl::fallback_rows_kernel<<<(unsigned)d.num_sms, tl::FB_THREADS, 0, stream>>>(p);
+    TL_CUDA(cudaGetLastError());
+    return TL_OK;
 }
 
 // Rows one launch serves: the block-scaled GEMM 64, the exact and CUDA-core kernels 32. Calls with
@@ -243,7 +290,13 @@ tl_status check_M(int M, int limit = TL_NVFP4_MAX_M) {
 }
 
 // Device copy of a stack's descriptor table (host bytes `key`): reused while the same
-// matrices come back.
+// matrices come back. On a miss the least recently used slot is refilled with an asynchronous
+// copy on `stream` from the slot's pinned staging buffer. The slot's previous table may still be
+// read by a kernel queued earlier: calls of one device are serialised on one stream (see the
+// header), so that kernel runs before the copy. The staging buffer is rewritten only after its
+// previous copy has executed (its event). A slot allocates (device and pinned host memory, after
+// synchronising the device) only when it must grow: once the slots have held the largest table
+// the caller uses, a miss neither allocates nor synchronises the device.
 tl_status device_table(DevState& d, const void* key_, size_t bytes, cudaStream_t stream, const void** out) {
     const unsigned char* key = static_cast<const unsigned char*>(key_);
     std::lock_guard<std::mutex> lk(g_mu);
@@ -262,13 +315,32 @@ tl_status device_table(DevState& d, const void* key_, size_t bytes, cudaStream_t
     StackCacheEntry* victim = &d.cache[0];
     for (auto& e : d.cache)
         if (!e.table || e.last_use < victim->last_use) victim = &e;
-    if (victim->table) {
-        TL_CUDA(cudaDeviceSynchronize());   // the old table may be read by a kernel in flight
-        TL_CUDA(cudaFree(victim->table));
-        victim->table = nullptr;
+    if (victim->cap < bytes) {
+        if (victim->table) {
+            TL_CUDA(cudaDeviceSynchronize());   // the old table may be read by a kernel in flight
+            TL_CUDA(cudaFree(victim->table));
+            TL_CUDA(cudaFreeHost(victim->staging));
+            victim->table = nullptr;
+            victim->staging = nullptr;
+            victim->cap = 0;
+            victim->key.clear();
+        }
+        if (!victim->copied) TL_CUDA(cudaEventCreateWithFlags(&victim->copied, cudaEventDisableTiming));
+        const size_t cap = (bytes + 4095) & ~size_t(4095);
+        TL_CUDA(cudaMalloc(&victim->table, cap));
+        if (cudaMallocHost(&victim->staging, cap) != cudaSuccess) {
+            cudaFree(victim->table);
+            victim->table = nullptr;
+            return fail(TL_ERR_CUDA, "cudaMallocHost of a descriptor staging buffer failed");
+        }
+        victim->cap = cap;
+    } else {
+        TL_CUDA(cudaEventSynchronize(victim->copied));   // its last refill copy has run
     }
-    TL_CUDA(cudaMalloc(&victim->table, bytes));
-    TL_CUDA(cudaMemcpy(victim->table, key, bytes, cudaMemcpyHostToDevice));
+    victim->key.clear();   // the slot holds no valid table until the copy is queued
+    memcpy(victim->staging, key, bytes);
+    TL_CUDA(cudaMemcpyAsync(victim->table, victim->staging, bytes, cudaMemcpyHostToDevice, stream));
+    TL_CUDA(cudaEventRecord(victim->copied, stream));
     victim->key.assign(key, key + bytes);
     victim->last_use = d.use_clock;
     *out = victim->table;
@@ -286,9 +358,20 @@ tl_status stack_table(DevState& d, const std::vector<tl::TcMat>& mats, cudaStrea
 // state lookup). `table_out` receives the TcMat array when n_mats > 1.
 // path: the GEMM path the parameters are for (the caller's copy of the setting, so that one
 // call or plan never mixes two paths).
+size_t xh_bytes_total(const tl_nvfp4_matrix* mats, int n_mats, int M) {
+    size_t t = 0;
+    for (int i = 0; i < n_mats; ++i) t += xh_bytes_of(M, mats[i].K);
+    return t;
+}
+
+tl_status ensure_xh(DevState& d, size_t bytes, cudaStream_t stream);
+
+// xh: the exact path's scratch for the whole stack (xh_bytes_total bytes); nullptr means the
+// per-device buffer (grown here if needed). Unused on the other paths.
 tl_status build_params(const tl_nvfp4_matrix* mats, int n_mats, int M, const unsigned char* x_dev,
                        unsigned char* y_dev, int path, DevState** dstate, tl::TcParams* p,
-                       std::vector<tl::TcMat>* table_out) {
+                       std::vector<tl::TcMat>* table_out, unsigned char* xh = nullptr,
+                       cudaStream_t stream = nullptr) {
     tl_status st = check_M(M, path == TL_PATH_BLOCK_SCALED ? kBsMaxRows : kExactMaxRows);
     if (st != TL_OK) return st;
     if (!mats) return fail(TL_ERR_INVALID_VALUE, "mats is null");
@@ -313,7 +396,14 @@ tl_status build_params(const tl_nvfp4_matrix* mats, int n_mats, int M, const uns
     st = current_state(dstate);
     if (st != TL_OK) return st;
     if (path == TL_PATH_BLOCK_SCALED) return TL_OK;     // the block-scaled launch builds its own tables
+    const bool f16 = (path == TL_PATH_EXACT);
+    if (f16 && !xh) {
+        st = ensure_xh(**dstate, xh_bytes_total(mats, n_mats, M), stream);
+        if (st != TL_OK) return st;
+        xh = (*dstate)->xh_buf;
+    }
     const int NX = M <= 16 ? 16 : 32;
+    size_t hoff = 0;
     std::vector<tl::TcMat>& tbl = *table_out;
     tbl.assign(n_mats, tl::TcMat());
     long long tiles = 0;
@@ -323,8 +413,10 @@ tl_status build_params(const tl_nvfp4_matrix* mats, int n_mats, int M, const uns
         const tl_nvfp4_matrix& m = mats[i];
         const void* x = x_dev ? static_cast<const void*>(x_dev + xoff) : m.x;
         void* y = y_dev ? static_cast<void*>(y_dev + yoff) : m.y;
-        st = build_mat(&tbl[i], x, M, NX, m.w_codes, m.w_scales, m.global_scale, y, m.N, m.K, tiles);
+        st = build_mat(&tbl[i], x, M, NX, m.w_codes, m.w_scales, m.global_scale, y, m.N, m.K, tiles,
+                       f16 ? xh + hoff : nullptr);
         if (st != TL_OK) return st;
+        if (f16) hoff += xh_bytes_of(M, m.K);
         tiles += (long long)tbl[i].n_tiles * tbl[i].k_tiles;
         xoff += (size_t)2 * M * m.K;
         yoff += (size_t)2 * M * m.N;
@@ -389,15 +481,15 @@ tl_status run_stack_rows(const tl_nvfp4_matrix* mats, int n_mats, int M, const u
     tl::TcParams p;
     std::vector<tl::TcMat> tbl;
     const int path = current_path();
-    tl_status st = build_params(mats, n_mats, M, x_dev, y_dev, path, &d, &p, &tbl);
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    tl_status st = build_params(mats, n_mats, M, x_dev, y_dev, path, &d, &p, &tbl, nullptr, stream);
     if (st != TL_OK || M == 0) return st;
     if (path == TL_PATH_BLOCK_SCALED) return run_stack_bs(mats, n_mats, M, x_dev, y_dev, stream_, d);
-    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
     if (n_mats > 1) {
         st = stack_table(*d, tbl, stream, &p.mats);
         if (st != TL_OK) return st;
     }
-    return launch_tc_any(*d, p, stream);
+    return launch_tc_any(*d, p, path == TL_PATH_EXACT, stream);
 }
 
 
@@ -637,7 +729,7 @@ tl_status build_bs(const tl_nvfp4_matrix* mats, int n_mats, int M, const unsigne
     L->bp.mats = nullptr;
     L->grid = (int)std::min<long long>(bs_unit_ktiles(mats, n_mats), num_sms);
     build_schedule(mats, n_mats, L->grid, &L->sched, tile_rows);
-    if (L->sched.slots > 4 * num_sms || L->sched.splits > 2 * num_sms)
+    if (L->sched.slots > 4 * num_sms || (size_t)L->sched.splits * kCountersPerSplit > counter_words(num_sms))
         return fail(TL_ERR_DEVICE_FAULT, "internal: schedule needs %d partial slots and %d splits", L->sched.slots,
                     L->sched.splits);
     if (n_mats == 1) L->bp.one = L->tbl[0];
@@ -707,6 +799,26 @@ tl_status ensure_xs(DevState& d, size_t bytes, cudaStream_t stream) {
     return TL_OK;
 }
 
+// Grow the per-device prepared-X scratch of the exact path to `bytes` (never inside a graph
+// capture). It only grows: once it has the largest size the caller uses, no call allocates.
+tl_status ensure_xh(DevState& d, size_t bytes, cudaStream_t stream) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (d.xh_cap >= bytes) return TL_OK;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    TL_CUDA(cudaStreamIsCapturing(stream, &cs));
+    if (cs != cudaStreamCaptureStatusNone)
+        return fail(TL_ERR_UNSUPPORTED, "the exact path must run once at this size before graph capture");
+    if (d.xh_buf) {
+        TL_CUDA(cudaDeviceSynchronize());   // a kernel in flight may still use the old buffer
+        TL_CUDA(cudaFree(d.xh_buf));
+        d.xh_buf = nullptr;
+        d.xh_cap = 0;
+    }
+    TL_CUDA(cudaMalloc(&d.xh_buf, bytes));
+    d.xh_cap = bytes;
+    return TL_OK;
+}
+
 tl_status run_stack_bs(const tl_nvfp4_matrix* mats, int n_mats, int M, const unsigned char* x_dev,
                        unsigned char* y_dev, void* stream_, DevState* d) {
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
@@ -744,8 +856,13 @@ tl_status run_stack_bs(const tl_nvfp4_matrix* mats, int n_mats, int M, const uns
 // engine that hands all free HBM to its KV-cache pool at start-up has nothing left
 // for a first-call workspace, and some host runtimes route every device allocation
 // through their own pool and forbid libraries from calling cudaMalloc. For them,
-// tl_nvfp4_verify_gemm_noalloc() runs the same tensor-core kernel with its split-K
-// scratch in the static array below, which the CUDA module reserves when it loads.
+// tl_nvfp4_verify_gemm_noalloc() runs the exact bf16-decode kernel (TL_PATH_BF16_EXACT) with
+// its split-K scratch in the static array below. The array is device memory of this
+// library's CUDA module: with lazy module loading (the default since CUDA 12.2) the module,
+// and so the array, is loaded on a device the first time the library touches it there, which
+// for a caller that only uses this entry point is the set-up inside its first call. That first
+// call is therefore the one that takes device memory (the array and the module's code); later
+// calls take none.
 
 // Room for the split-K partials of up to kNoAllocMaxCtas CTAs (two 32 x 128 fp32 tiles
 // each, 5 MiB in all), their counters (must be zero when a launch starts) and a status word.
@@ -785,9 +902,9 @@ tl_status noalloc_setup(int device, NoAllocDevice** out) {
             return fail(TL_ERR_CUDA, "cudaGetSymbolAddress of the static scratch failed: %s", cudaGetErrorString(e));
         tl_status st = load_encode_fn();
         if (st != TL_OK) return st;
-        TL_CUDA(cudaFuncSetAttribute(tl::gemm_tc_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        TL_CUDA(cudaFuncSetAttribute(tl::gemm_tc_kernel<16, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      tl::TcCfg<16>::SMEM_BYTES));
-        TL_CUDA(cudaFuncSetAttribute(tl::gemm_tc_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        TL_CUDA(cudaFuncSetAttribute(tl::gemm_tc_kernel<32, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      tl::TcCfg<32>::SMEM_BYTES));
         nd.num_sms = sms;
         nd.scratch = static_cast<NoAllocScratch*>(ptr);
@@ -827,15 +944,16 @@ extern "C" tl_status tl_nvfp4_verify_gemm_noalloc(const void* x, int M, const vo
     p.spread_mul = 0x1040u;
     p.scale_mul = 0x00100010u;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    // the counters must start at zero; a launch that gave up could have left them raised
+    // the counters must start at zero; a launch that gave up could have left them raised. The
+    // status word is not cleared here: it keeps a timeout until tl_noalloc_check_error() reads it.
     TL_CUDA(cudaMemsetAsync(p.counters, 0, sizeof(nd->scratch->counters), s));
     long long grid = p.total_tiles;
     if (grid > nd->num_sms) grid = nd->num_sms;
     if (grid > kNoAllocMaxCtas) grid = kNoAllocMaxCtas;
     if (NX == 16)
-        tl::gemm_tc_kernel<16><<<(unsigned)grid, tl::TC_THREADS, tl::TcCfg<16>::SMEM_BYTES, s>>>(p);
+        tl::gemm_tc_kernel<16, false><<<(unsigned)grid, tl::TC_THREADS, tl::TcCfg<16>::SMEM_BYTES, s>>>(p);
     else
-        tl::gemm_tc_kernel<32><<<(unsigned)grid, tl::TC_THREADS, tl::TcCfg<32>::SMEM_BYTES, s>>>(p);
+        tl::gemm_tc_kernel<32, false><<<(unsigned)grid, tl::TC_THREADS, tl::TcCfg<32>::SMEM_BYTES, s>>>(p);
     TL_CUDA(cudaGetLastError());
     return TL_OK;
 }
@@ -843,7 +961,7 @@ extern "C" tl_status tl_nvfp4_verify_gemm_noalloc(const void* x, int M, const vo
 struct tl_nvfp4_plan_st {
     int device = 0;
     DevState* d = nullptr;
-    int path = TL_PATH_BLOCK_SCALED;  // fixed when the plan is made
+    int path = TL_PATH_EXACT;         // fixed when the plan is made
     tl::TcParams params;
     tl::TcMat* table = nullptr;       // device copy when n_mats > 1
     tl::BsParams bparams;             // block-scaled path
@@ -851,6 +969,7 @@ struct tl_nvfp4_plan_st {
     int grid = 0;                     // CTAs of the block-scaled GEMM
     void* bs_tables = nullptr;        // device copies of the BsMat and XSplitMat tables (n_mats > 1) and the schedule
     unsigned char* xs = nullptr;      // the plan's own X-piece scratch
+    unsigned char* xh = nullptr;      // the plan's own prepared-X scratch (exact path)
     const void* x_base = nullptr;     // packed X_i buffer (or nullptr if not packed)
     void* y_base = nullptr;           // packed Y_i buffer (or nullptr if not packed)
     size_t x_bytes = 0, y_bytes = 0;
@@ -905,7 +1024,7 @@ tl_status plan_launch(tl_nvfp4_plan plan, cudaStream_t s) {
     if (plan->params.n_mats < 1 || plan->params.total_tiles < 1 || (plan->params.n_mats > 1 && !plan->params.mats))
         return fail(TL_ERR_DEVICE_FAULT, "internal: plan without descriptors");
     tl::TcParams p = plan->params;
-    return launch_tc_any(*plan->d, p, s);
+    return launch_tc_any(*plan->d, p, plan->path == TL_PATH_EXACT, s);
 }
 
 tl_status plan_create_path(const tl_nvfp4_matrix* mats, int n_mats, int M, int path, tl_nvfp4_plan* plan_out);
@@ -996,9 +1115,22 @@ tl_status plan_create_path(const tl_nvfp4_matrix* mats, int n_mats, int M, int p
     DevState* d = nullptr;
     tl::TcParams p;
     std::vector<tl::TcMat> tbl;
-    tl_status st = build_params(mats, n_mats, M, nullptr, nullptr, path, &d, &p, &tbl);
+    // the exact path's scratch belongs to the plan: validate first (the bf16 decode builds no
+    // scratch), then allocate it and build the descriptors over it
+    tl_status st = build_params(mats, n_mats, M, nullptr, nullptr, path == TL_PATH_EXACT ? TL_PATH_BF16_EXACT : path,
+                                &d, &p, &tbl);
     if (st != TL_OK) return st;
+    unsigned char* xh = nullptr;
+    if (path == TL_PATH_EXACT) {
+        TL_CUDA(cudaMalloc(&xh, xh_bytes_total(mats, n_mats, M)));
+        st = build_params(mats, n_mats, M, nullptr, nullptr, path, &d, &p, &tbl, xh);
+        if (st != TL_OK) {
+            cudaFree(xh);
+            return st;
+        }
+    }
     tl_nvfp4_plan plan = new tl_nvfp4_plan_st();
+    plan->xh = xh;
     TL_CUDA(cudaGetDevice(&plan->device));
     plan->d = d;
     plan->params = p;
@@ -1080,22 +1212,36 @@ tl_status tl_nvfp4_plan_run_host(tl_nvfp4_plan plan, const void* x_host, void* y
     TL_CUDA(cudaEventRecord(e_start, s));
     TL_CUDA(cudaStreamWaitEvent(plan->s_in, e_start, 0));
     TL_CUDA(cudaStreamWaitEvent(plan->s_out, e_start, 0));
-    for (size_t c = 0; c < C; ++c) {
-        TL_CUDA(cudaMemcpyAsync(xd + plan->cx_off[c], xh + plan->cx_off[c], plan->cx_len[c], cudaMemcpyHostToDevice,
-                                plan->s_in));
-        TL_CUDA(cudaEventRecord(plan->ev[2 + 2 * c], plan->s_in));
+    // From here on both internal streams are forked from `s`: every return joins them back
+    // (s_in into s_out, s_out into s), so that later work on `s` is ordered after everything
+    // queued and a stream capture of the call stays closed.
+    tl_status st = TL_OK;
+    for (size_t c = 0; c < C && st == TL_OK; ++c) {
+        if (cudaMemcpyAsync(xd + plan->cx_off[c], xh + plan->cx_off[c], plan->cx_len[c], cudaMemcpyHostToDevice,
+                            plan->s_in) != cudaSuccess ||
+            cudaEventRecord(plan->ev[2 + 2 * c], plan->s_in) != cudaSuccess)
+            st = fail(TL_ERR_CUDA, "queueing the X copy of chunk %zu failed", c);
     }
-    for (size_t c = 0; c < C; ++c) {
-        TL_CUDA(cudaStreamWaitEvent(s, plan->ev[2 + 2 * c], 0));
-        tl_status st = plan_launch(plan->chunks[c], s);
-        if (st != TL_OK) return st;
-        TL_CUDA(cudaEventRecord(plan->ev[3 + 2 * c], s));
-        TL_CUDA(cudaStreamWaitEvent(plan->s_out, plan->ev[3 + 2 * c], 0));
-        TL_CUDA(cudaMemcpyAsync(yh + plan->cy_off[c], yd + plan->cy_off[c], plan->cy_len[c], cudaMemcpyDeviceToHost,
-                                plan->s_out));
+    for (size_t c = 0; c < C && st == TL_OK; ++c) {
+        if (cudaStreamWaitEvent(s, plan->ev[2 + 2 * c], 0) != cudaSuccess) {
+            st = fail(TL_ERR_CUDA, "ordering chunk %zu after its X copy failed", c);
+            break;
+        }
+        st = plan_launch(plan->chunks[c], s);
+        if (st != TL_OK) break;
+        if (cudaEventRecord(plan->ev[3 + 2 * c], s) != cudaSuccess ||
+            cudaStreamWaitEvent(plan->s_out, plan->ev[3 + 2 * c], 0) != cudaSuccess ||
+            cudaMemcpyAsync(yh + plan->cy_off[c], yd + plan->cy_off[c], plan->cy_len[c], cudaMemcpyDeviceToHost,
+                            plan->s_out) != cudaSuccess)
+            st = fail(TL_ERR_CUDA, "queueing the Y copy of chunk %zu failed", c);
     }
-    TL_CUDA(cudaEventRecord(e_done, plan->s_out));
-    TL_CUDA(cudaStreamWaitEvent(s, e_done, 0));
+    // join: s_in -> s_out (e_start is free again once recorded here), s_out -> s
+    const bool joined = cudaEventRecord(e_start, plan->s_in) == cudaSuccess &&
+                        cudaStreamWaitEvent(plan->s_out, e_start, 0) == cudaSuccess &&
+                        cudaEventRecord(e_done, plan->s_out) == cudaSuccess &&
+                        cudaStreamWaitEvent(s, e_done, 0) == cudaSuccess;
+    if (st != TL_OK) return st;
+    if (!joined) return fail(TL_ERR_CUDA, "joining the host-buffer run's copy streams failed");
     return TL_OK;
 }
 
@@ -1113,7 +1259,7 @@ tl_status tl_nvfp4_plan_destroy(tl_nvfp4_plan plan) {
         if (plan->s_out) cudaStreamDestroy(plan->s_out);
         cudaSetDevice(prev);
     }
-    if (plan->table || plan->bs_tables || plan->xs) {
+    if (plan->table || plan->bs_tables || plan->xs || plan->xh) {
         int prev = 0;
         cudaGetDevice(&prev);
         cudaSetDevice(plan->device);
@@ -1121,6 +1267,7 @@ tl_status tl_nvfp4_plan_destroy(tl_nvfp4_plan plan) {
         if (plan->table) cudaFree(plan->table);
         if (plan->bs_tables) cudaFree(plan->bs_tables);
         if (plan->xs) cudaFree(plan->xs);
+        if (plan->xh) cudaFree(plan->xh);
         cudaSetDevice(prev);
     }
     delete plan;
@@ -1128,7 +1275,7 @@ tl_status tl_nvfp4_plan_destroy(tl_nvfp4_plan plan) {
 }
 
 tl_status tl_set_gemm_path(int path) {
-    if (path != TL_PATH_BLOCK_SCALED && path != TL_PATH_BF16_EXACT)
+    if (path != TL_PATH_BLOCK_SCALED && path != TL_PATH_BF16_EXACT && path != TL_PATH_EXACT)
         return fail(TL_ERR_INVALID_VALUE, "unknown GEMM path %d", path);
     std::lock_guard<std::mutex> lk(g_mu);
     g_path = path;
@@ -1160,9 +1307,13 @@ void tl_shutdown(void) {
         cudaFree(d.partials);
         cudaFree(d.counters);
         cudaFree(d.qscratch);
-        for (auto& e : d.cache)
+        for (auto& e : d.cache) {
             if (e.table) cudaFree(e.table);
+            if (e.staging) cudaFreeHost(e.staging);
+            if (e.copied) cudaEventDestroy(e.copied);
+        }
         if (d.xs_buf) cudaFree(d.xs_buf);
+        if (d.xh_buf) cudaFree(d.xh_buf);
         d = DevState();
     }
     cudaSetDevice(prev);
@@ -1286,21 +1437,58 @@ tl_status tl_nvfp4_quantize(const float* w, int N, int K, void* w_codes, void* w
     return TL_OK;
 }
 
+// The status word of the no-allocation entry point's static scratch on the current device:
+// read, and cleared when set (no allocation; only the static array is touched).
+static tl_status noalloc_take_error(int* code_out) {
+    *code_out = 0;
+    int dev = 0;
+    TL_CUDA(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) return fail(TL_ERR_INVALID_VALUE, "device %d out of range", dev);
+    NoAllocScratch* sc = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (g_noalloc[dev].ready) sc = g_noalloc[dev].scratch;
+    }
+    if (!sc) return TL_OK;   // never used on this device
+    int code = 0;
+    TL_CUDA(cudaMemcpy(&code, sc->err, sizeof code, cudaMemcpyDeviceToHost));
+    if (code != 0) TL_CUDA(cudaMemset(sc->err, 0, sizeof code));
+    *code_out = code;
+    return TL_OK;
+}
+
+static tl_status status_of_code(int code) {
+    if (code == 0) return TL_OK;
+    if ((code & 0xF00) == 0x100) return fail(TL_ERR_TIMEOUT, "a device-side wait ran past its limit (code 0x%x)", code);
+    return fail(TL_ERR_DEVICE_FAULT, "device status word 0x%x", code);
+}
+
+tl_status tl_noalloc_check_error(void* stream) {
+    TL_CUDA(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+    int code = 0;
+    tl_status st = noalloc_take_error(&code);
+    if (st != TL_OK) return st;
+    return status_of_code(code);
+}
+
 tl_status tl_check_device_error(void* stream) {
     DevState* d = nullptr;
     tl_status st = current_state(&d);
     if (st != TL_OK) return st;
     TL_CUDA(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+    int na_code = 0;
+    st = noalloc_take_error(&na_code);
+    if (st != TL_OK) return st;
     int code = 0;
     TL_CUDA(cudaMemcpy(&code, d->err, sizeof code, cudaMemcpyDeviceToHost));
+    if (code == 0 && na_code != 0) return status_of_code(na_code);
     if (code == 0) return TL_OK;
-    // a kernel that gave up may have left split-K counters raised: clear them for the next launch
+    // a kernel that gave up may have left split-K counters raised: clear all of them (up to
+    // 2 * SMs splits of four counters each, kCounterWords) for the next launch
     TL_CUDA(cudaMemset(d->err, 0, sizeof code));
-    TL_CUDA(cudaMemset(d->counters, 0, (size_t)4 * d->num_sms * sizeof(unsigned)));
+    TL_CUDA(cudaMemset(d->counters, 0, counter_words(d->num_sms) * sizeof(unsigned)));
     TL_CUDA(cudaDeviceSynchronize());
-    if ((code & 0xF00) == 0x100)
-        return fail(TL_ERR_TIMEOUT, "a device-side wait ran past its limit (code 0x%x)", code);
-    return fail(TL_ERR_DEVICE_FAULT, "device status word 0x%x", code);
+    return status_of_code(code);
 }
 
 tl_status tl_selftest_bounded_wait(unsigned iterations, void* stream) {
