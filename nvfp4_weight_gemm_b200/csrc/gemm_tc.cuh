@@ -73,15 +73,15 @@ struct alignas(64) TcMat {
     CUtensorMap tm_x;       // bf16 X as 3-D {64, M, K/64}, box {64, NX, 4}: the four 64-k slices of a
                             // tile, 128-byte swizzle (rows >= M read 0)
     __nv_bfloat16* y;
-    float g_out;            // bf16 decode: epilogue multiplier global_scale * 2^7
+    float g_out;            // epilogue multiplier: global_scale * 2^7
     int N;
     int k_tiles;            // K / 256
     int n_tiles;            // ceil(N / 128)
     long long tile_begin;   // first global tile index of this matrix
-    // f16 decode only (tm_x then maps xh, the prepared copy of X; see xprep.cuh)
+    // the exact f16 path only (gemm_ex.cuh, xprep.cuh; tm_x then maps xh, the prepared copy of X)
     const __nv_bfloat16* x; // X as given, bf16 [M][K]
     __half* xh;             // X row m times 2^-e_m in f16, [M][K]
-    float* rowfac;          // 2^e_m per row; the epilogue multiplies by global_scale * 2^e_m
+    float* rowfac;          // 2^e_m per row; that path's epilogue multiplies by global_scale * 2^e_m
     unsigned* rowmask;      // bit m set: row m is not exact in f16 (recomputed by the fallback)
     const uint8_t* codes;   // the weights as given (fallback rows)
     const uint8_t* scales;
@@ -116,9 +116,7 @@ struct TcCfg {
     static constexpr int X_RING = W_STAGES * W_STAGE_BYTES;            // offset of the X ring
     static constexpr int NUM_A = 3;                                    // tile slots: A buffer + X stage
     static constexpr int SMEM_BYTES = X_RING + NUM_A * X_BYTES + 1024 /*align*/ + 512 /*barriers*/;
-    // operand type: bf16 (decode to bf16, X as given) or f16 (decode to f16, X prepared)
-    static constexpr uint32_t IDESC_BF16 = idesc_f16(1u, 128u, (uint32_t)NX);
-    static constexpr uint32_t IDESC_F16 = idesc_f16(0u, 128u, (uint32_t)NX);
+    static constexpr uint32_t IDESC = idesc_f16(1u, 128u, (uint32_t)NX);
     // tensor memory: three A buffers (128 columns each) so a tile set never waits for the
     // MMAs of its own previous tile, then ACC_BUFS accumulator buffers of TC_NISSUE
     // accumulators of NX fp32 columns each (one buffer at NX = 32: the MMAs then wait for
@@ -191,12 +189,6 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     return d;
 }
 
-__device__ __forceinline__ uint32_t hmul2_f16(uint32_t a, uint32_t b) {
-    uint32_t d;
-    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-
 __device__ __forceinline__ uint32_t hmul2_bf16(uint32_t a, uint32_t b) {
     uint32_t d;
     asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
@@ -253,62 +245,17 @@ __device__ __forceinline__ void decode8(uint32_t q, uint32_t S, uint32_t spread,
     }
 }
 
-// f16 decode. Four scale bytes of `sc` -> four words holding e4m3(s) in both halves (exact:
-// every E4M3 value, subnormals, signs and NaN included, is an f16 value; hardware convert).
-__device__ __forceinline__ void scales4_f16(uint32_t sc, uint32_t (&S)[4]) {
-#pragma unroll
-    for (int p = 0; p < 2; ++p) {
-        uint32_t h;
-        asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}"
-            : "=r"(h) : "r"(sc >> (16 * p)));
-        S[2 * p] = prmt(h, 0u, 0x1010u);
-        S[2 * p + 1] = prmt(h, 0u, 0x3232u);
-    }
-}
-
-// f16 decode. Sixteen code bytes (32 weights, k order) -> sixteen f16x2 words W' in k order:
-// the hardware converts each byte's two E2M1 codes to f16 (low nibble to the low half), and
-// one f16 multiply by the block's scale gives W' = e2m1 * e4m3 exactly (at most six
-// significant bits, inside the f16 normal range: 2^-10 <= |W'| <= 2688). Bytes 0..7 belong to
-// the block of S0, bytes 8..15 to the block of S1. The bytes are unpacked with one vector move
-// per word, which the converts read in place.
-__device__ __forceinline__ void decode16_f16(uint4 q, uint32_t S0, uint32_t S1, uint32_t* out) {
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        uint32_t c0, c1, c2, c3;
-        asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %4;\n\t"
-            "cvt.rn.f16x2.e2m1x2 %0, b0;\n\tcvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
-            "cvt.rn.f16x2.e2m1x2 %2, b2;\n\tcvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
-            : "=r"(c0), "=r"(c1), "=r"(c2), "=r"(c3) : "r"(w[j]));
-        const uint32_t S = (j < 2) ? S0 : S1;
-        out[4 * j + 0] = hmul2_f16(c0, S);
-        out[4 * j + 1] = hmul2_f16(c1, S);
-        out[4 * j + 2] = hmul2_f16(c2, S);
-        out[4 * j + 3] = hmul2_f16(c3, S);
-    }
-}
-
-// Epilogue multiplier of X row i: global_scale * 2^7 (bf16 decode, W' scaled by 2^-7), or
-// global_scale * 2^e_i (f16 decode, X row i prepared as x * 2^-e_i; both factors exact).
-template <bool F16>
-__device__ __forceinline__ float out_factor(float g, const float* rowfac, int i) {
-    if constexpr (F16) return g * __ldg(rowfac + i);
-    else return g;
-}
-
 // MMA issuer J (a whole warp, converged; one elected lane issues): k-steps
 // [tc_ks_begin(J), tc_ks_begin(J + 1)) of every tile into accumulator J. A tile slot (A buffer +
 // X stage) is ready when the 8 warps of its tile set have arrived and its X bytes have landed;
 // the slot is handed back by one commit per issuer.
-template <int NX, bool F16, int J>
+template <int NX, int J>
 __device__ __forceinline__ void tc_mma_issuer(const TcParams& p, const TcMat* mats, long long t_begin, long long t_end,
                                               uint8_t* smem, uint32_t tmem, uint64_t* ready, uint64_t* tfree,
                                               uint64_t* accfull, uint64_t* accempty, uint64_t* drain,
                                               volatile int* abort_flag) {
     using C = TcCfg<NX>;
     constexpr int I0 = tc_ks_begin(J), I1 = tc_ks_begin(J + 1);
-    constexpr uint32_t IDESC = F16 ? C::IDESC_F16 : C::IDESC_BF16;
     const bool leader = elect_one();   // issues every MMA and commit of this issuer
     int a = 0, acc = 0;
     uint32_t aph = 0, accph = 0;
@@ -339,7 +286,7 @@ __device__ __forceinline__ void tc_mma_issuer(const TcParams& p, const TcMat* ma
 #pragma unroll
                 for (int i = I0; i < I1; ++i)
                     mma_ts_f16(d_tmem, a_tmem + 8u * (i - I0),
-                               bdesc0 + (uint64_t)((((i >> 2) * C::X_SUB + (i & 3) * 32)) >> 4), IDESC,
+                               bdesc0 + (uint64_t)((((i >> 2) * C::X_SUB + (i & 3) * 32)) >> 4), C::IDESC,
                                (i == I0) ? (first ^ 1u) : 1u);
                 mma_commit(&tfree[a]);
             }
@@ -357,7 +304,7 @@ __device__ __forceinline__ void tc_mma_issuer(const TcParams& p, const TcMat* ma
     __syncwarp();
 }
 
-template <int NX, bool F16>
+template <int NX>
 __global__ void __launch_bounds__(TC_THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ TcParams p) {
     using C = TcCfg<NX>;
@@ -484,13 +431,13 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
         // ------------------------------------------------------------ MMA issuers
         const int j = tc_issuer_of_warp(warp);
         if (j == 0)
-            tc_mma_issuer<NX, F16, 0>(p, mats, t_begin, t_end, smem, tmem, ready, tfree, accfull, accempty, drain, abort_flag);
+            tc_mma_issuer<NX, 0>(p, mats, t_begin, t_end, smem, tmem, ready, tfree, accfull, accempty, drain, abort_flag);
         else if (j == 1)
-            tc_mma_issuer<NX, F16, 1>(p, mats, t_begin, t_end, smem, tmem, ready, tfree, accfull, accempty, drain, abort_flag);
+            tc_mma_issuer<NX, 1>(p, mats, t_begin, t_end, smem, tmem, ready, tfree, accfull, accempty, drain, abort_flag);
         else if (j == 2)
-            tc_mma_issuer<NX, F16, 2>(p, mats, t_begin, t_end, smem, tmem, ready, tfree, accfull, accempty, drain, abort_flag);
+            tc_mma_issuer<NX, 2>(p, mats, t_begin, t_end, smem, tmem, ready, tfree, accfull, accempty, drain, abort_flag);
         else
-            tc_mma_issuer<NX, F16, 3>(p, mats, t_begin, t_end, smem, tmem, ready, tfree, accfull, accempty, drain, abort_flag);
+            tc_mma_issuer<NX, 3>(p, mats, t_begin, t_end, smem, tmem, ready, tfree, accfull, accempty, drain, abort_flag);
         if (warp == 1 && !__all_sync(0xFFFFFFFFu, mbar_wait(drain, 0, TL_WAIT_LIMIT)) && lane == 0)
             tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_DRAIN);
     } else if (warp >= 4 && warp < 20) {
@@ -549,24 +496,18 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
             // one vote when both are ready, the usual case; each is waited for on its own otherwise
             const bool both_ready = __all_sync(0xFFFFFFFFu, (!has_next || mbar_test(&wfull[s], ph)) &&
                                                              mbar_test(&tfree[a], aph ^ 1u));
-            const bool fast = F16 || scales_fast_ok(sc);
+            const bool fast = scales_fast_ok(sc);
             uint32_t S[4];
+            if (fast) scales4_fast(sc.x, smul, S); else scales4_exact(sc.x, S);
             uint32_t out[32];
-            if (F16) {
-                scales4_f16(sc.x, S);
-                decode16_f16(cw0, S[0], S[1], &out[0]);
-                decode16_f16(cw1, S[2], S[3], &out[16]);
-            } else {
-                if (fast) scales4_fast(sc.x, smul, S); else scales4_exact(sc.x, S);
-                decode8(cw0.x, S[0], spread, &out[0]);
-                decode8(cw0.y, S[0], spread, &out[4]);
-                decode8(cw0.z, S[1], spread, &out[8]);
-                decode8(cw0.w, S[1], spread, &out[12]);
-                decode8(cw1.x, S[2], spread, &out[16]);
-                decode8(cw1.y, S[2], spread, &out[20]);
-                decode8(cw1.z, S[3], spread, &out[24]);
-                decode8(cw1.w, S[3], spread, &out[28]);
-            }
+            decode8(cw0.x, S[0], spread, &out[0]);
+            decode8(cw0.y, S[0], spread, &out[4]);
+            decode8(cw0.z, S[1], spread, &out[8]);
+            decode8(cw0.w, S[1], spread, &out[12]);
+            decode8(cw1.x, S[2], spread, &out[16]);
+            decode8(cw1.y, S[2], spread, &out[20]);
+            decode8(cw1.z, S[3], spread, &out[24]);
+            decode8(cw1.w, S[3], spread, &out[28]);
             // second chunk's codes: in flight while the first chunk is stored
             cw0 = *reinterpret_cast<const uint4*>(st_cur + cw_off[2]);
             cw1 = *reinterpret_cast<const uint4*>(st_cur + cw_off[3]);
@@ -580,21 +521,15 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
             tmem_st32(col, out);
             __syncwarp();
             if (lane == 0) mbar_arrive(&wempty[s_cur]);   // every byte of the stage this warp needs is in registers
-            if (F16) {
-                scales4_f16(sc.y, S);
-                decode16_f16(cw0, S[0], S[1], &out[0]);
-                decode16_f16(cw1, S[2], S[3], &out[16]);
-            } else {
-                if (fast) scales4_fast(sc.y, smul, S); else scales4_exact(sc.y, S);
-                decode8(cw0.x, S[0], spread, &out[0]);
-                decode8(cw0.y, S[0], spread, &out[4]);
-                decode8(cw0.z, S[1], spread, &out[8]);
-                decode8(cw0.w, S[1], spread, &out[12]);
-                decode8(cw1.x, S[2], spread, &out[16]);
-                decode8(cw1.y, S[2], spread, &out[20]);
-                decode8(cw1.z, S[3], spread, &out[24]);
-                decode8(cw1.w, S[3], spread, &out[28]);
-            }
+            if (fast) scales4_fast(sc.y, smul, S); else scales4_exact(sc.y, S);
+            decode8(cw0.x, S[0], spread, &out[0]);
+            decode8(cw0.y, S[0], spread, &out[4]);
+            decode8(cw0.z, S[1], spread, &out[8]);
+            decode8(cw0.w, S[1], spread, &out[12]);
+            decode8(cw1.x, S[2], spread, &out[16]);
+            decode8(cw1.y, S[2], spread, &out[20]);
+            decode8(cw1.z, S[3], spread, &out[24]);
+            decode8(cw1.w, S[3], spread, &out[28]);
             tmem_st32(col + 32u, out);
             // the next tile's scales and first-chunk codes: in flight while the stores complete
             if (has_next) {
@@ -636,8 +571,7 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
             const TcMat& m = mats[sg.mat];
             // the matrix's fields in registers: stores to Y must not force them to be re-read
             __nv_bfloat16* const yp = m.y;
-            const float g_out = F16 ? m.g : m.g_out;
-            const float* const rowfac = m.rowfac;
+            const float g_out = m.g_out;
             const int N = m.N;
             const int n = sg.ntile * TC_BLOCK_N + r;
             const bool whole = (sg.k0 == 0 && sg.k1 == m.k_tiles);
@@ -668,7 +602,7 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
                 if (n < N) {
 #pragma unroll
                     for (int i = 0; i < NX; ++i)
-                        if (i < M) yp[(long long)i * N + n] = __float2bfloat16_rn(v[i] * out_factor<F16>(g_out, rowfac, i));
+                        if (i < M) yp[(long long)i * N + n] = __float2bfloat16_rn(v[i] * g_out);
                 }
             } else {
 #pragma unroll
@@ -705,9 +639,7 @@ gemm_tc_kernel(const __grid_constant__ TcParams p) {
                     if (n < N) {
 #pragma unroll
                         for (int i = 0; i < 16; ++i)
-                            if (c0 + i < M)
-                                yp[(long long)(c0 + i) * N + n] =
-                                    __float2bfloat16_rn(v[i] * out_factor<F16>(g_out, rowfac, c0 + i));
+                            if (c0 + i < M) yp[(long long)(c0 + i) * N + n] = __float2bfloat16_rn(v[i] * g_out);
                     }
                 }
                 if (lane == 0) p.counters[4 * f + q] = 0u;   // ready for the next launch

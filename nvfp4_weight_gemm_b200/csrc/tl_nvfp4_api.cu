@@ -21,6 +21,7 @@
 
 #include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
+#include "gemm_ex.cuh"
 #include "xprep.cuh"
 #include "gemm_bs.cuh"
 #include "kernels_aux.cuh"
@@ -247,31 +248,44 @@ tl_status build_mat(tl::TcMat* m, const void* x, int M, int NX, const void* code
     return TL_OK;
 }
 
-template <int NX, bool F16>
+template <int NX>
 tl_status launch_tc(DevState& d, tl::TcParams& p, cudaStream_t stream) {
     using C = tl::TcCfg<NX>;
     // the attribute is per function; set for both variants on first use (idempotent, cheap)
-    TL_CUDA(cudaFuncSetAttribute(tl::gemm_tc_kernel<NX, F16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::SMEM_BYTES));
+    TL_CUDA(cudaFuncSetAttribute(tl::gemm_tc_kernel<NX>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
     const long long grid = p.total_tiles < d.num_sms ? p.total_tiles : d.num_sms;
     p.partials = d.partials;
     p.counters = d.counters;
     p.err = d.err;
     p.spread_mul = 0x1040u;
     p.scale_mul = 0x00100010u;
-    tl::gemm_tc_kernel<NX, F16><<<(unsigned)grid, tl::TC_THREADS, C::SMEM_BYTES, stream>>>(p);
+    tl::gemm_tc_kernel<NX><<<(unsigned)grid, tl::TC_THREADS, C::SMEM_BYTES, stream>>>(p);
+    TL_CUDA(cudaGetLastError());
+    return TL_OK;
+}
+
+template <int NX>
+tl_status launch_ex(DevState& d, tl::TcParams& p, cudaStream_t stream) {
+    using C = tl::ExCfg<NX>;
+    TL_CUDA(cudaFuncSetAttribute(tl::gemm_ex_kernel<NX>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
+    const long long grid = p.total_tiles < d.num_sms ? p.total_tiles : d.num_sms;
+    p.partials = d.partials;
+    p.counters = d.counters;
+    p.err = d.err;
+    tl::gemm_ex_kernel<NX><<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, stream>>>(p);
     TL_CUDA(cudaGetLastError());
     return TL_OK;
 }
 
 // The exact paths. bf16 decode: one GEMM launch on X as given. f16 decode: the X preparation
-// (one CTA per matrix), the GEMM on the prepared X, then the fallback for flagged rows (it
+// (one CTA per matrix and group of 8 rows), the GEMM on the prepared X, then the fallback for flagged rows (it
 // returns at once when no row is flagged).
 tl_status launch_tc_any(DevState& d, tl::TcParams& p, bool f16, cudaStream_t stream) {
-    if (!f16) return (p.M <= 16) ? launch_tc<16, false>(d, p, stream) : launch_tc<32, false>(d, p, stream);
-    tl::x_prep_kernel<<<(unsigned)p.n_mats, tl::XP_THREADS, 0, stream>>>(p);
+    if (!f16) return (p.M <= 16) ? launch_tc<16>(d, p, stream) : launch_tc<32>(d, p, stream);
+    tl::x_prep_kernel<<<dim3((unsigned)p.n_mats, (unsigned)((p.M + tl::XP_ROWS - 1) / tl::XP_ROWS)), tl::XP_THREADS, 0,
+                        stream>>>(p);
     TL_CUDA(cudaGetLastError());
-    tl_status st = (p.M <= 16) ? launch_tc<16, true>(d, p, stream) : launch_tc<32, true>(d, p, stream);
+    tl_status st = (p.M <= 16) ? launch_ex<16>(d, p, stream) : launch_ex<32>(d, p, stream);
     if (st != TL_OK) return st;
     tl::fallback_rows_kernel<<<(unsigned)d.num_sms, tl::FB_THREADS, 0, stream>>>(p);
     TL_CUDA(cudaGetLastError());
@@ -902,9 +916,9 @@ tl_status noalloc_setup(int device, NoAllocDevice** out) {
             return fail(TL_ERR_CUDA, "cudaGetSymbolAddress of the static scratch failed: %s", cudaGetErrorString(e));
         tl_status st = load_encode_fn();
         if (st != TL_OK) return st;
-        TL_CUDA(cudaFuncSetAttribute(tl::gemm_tc_kernel<16, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        TL_CUDA(cudaFuncSetAttribute(tl::gemm_tc_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      tl::TcCfg<16>::SMEM_BYTES));
-        TL_CUDA(cudaFuncSetAttribute(tl::gemm_tc_kernel<32, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        TL_CUDA(cudaFuncSetAttribute(tl::gemm_tc_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      tl::TcCfg<32>::SMEM_BYTES));
         nd.num_sms = sms;
         nd.scratch = static_cast<NoAllocScratch*>(ptr);
@@ -951,9 +965,9 @@ extern "C" tl_status tl_nvfp4_verify_gemm_noalloc(const void* x, int M, const vo
     if (grid > nd->num_sms) grid = nd->num_sms;
     if (grid > kNoAllocMaxCtas) grid = kNoAllocMaxCtas;
     if (NX == 16)
-        tl::gemm_tc_kernel<16, false><<<(unsigned)grid, tl::TC_THREADS, tl::TcCfg<16>::SMEM_BYTES, s>>>(p);
+        tl::gemm_tc_kernel<16><<<(unsigned)grid, tl::TC_THREADS, tl::TcCfg<16>::SMEM_BYTES, s>>>(p);
     else
-        tl::gemm_tc_kernel<32, false><<<(unsigned)grid, tl::TC_THREADS, tl::TcCfg<32>::SMEM_BYTES, s>>>(p);
+        tl::gemm_tc_kernel<32><<<(unsigned)grid, tl::TC_THREADS, tl::TcCfg<32>::SMEM_BYTES, s>>>(p);
     TL_CUDA(cudaGetLastError());
     return TL_OK;
 }
