@@ -268,6 +268,38 @@ tl_status tl_nvfp4_dequant(const void* w_codes, const void* w_scales, float glob
 tl_status tl_nvfp4_quantize(const float* w, int N, int K, void* w_codes, void* w_scales,
                             float* global_scale_out, void* stream);
 
+/* FP8 output head of the verify pass, with its greedy top-2 (the next row of the path).
+ *
+ * The pages keep the model's output head in FP8 while the projections are NVFP4 (TandemLLM docs
+ * v0.12.0, "What TandemLLM is", section 1.2), and the agreement rule looks at the two best
+ * logits, a near tie being a gap within one unit in the last place (same page, section 1.5). For
+ * M tree rows:
+ *     logits[m][n] = (sum_k x[m][k] * e4m3(w[n][k])) * s_n
+ *     token = argmax_n (the lowest n among equal maxima), top1, top2 = the largest logit of the
+ *     row without the token's entry, gap_ulp = (top1 - top2) / ulp_bf16(top1)
+ * where ulp_bf16(v) = 2^(e - 7) for 2^e <= |v| < 2^(e + 1) (2^-133 below 2^-126).
+ *   x            device bf16 [M][K], 16-byte aligned
+ *   M            0..TL_HEAD_MAX_M (0 is a no-op)
+ *   w_fp8        device uint8 [N][K] E4M3 ("fn") bytes, 16-byte aligned; 0x7F / 0xFF are NaN
+ *   N            >= 2 (vocabulary rows);  K > 0 and K % 256 == 0
+ *   tensor_scale s_n for every n when row_scales is NULL (finite)
+ *   row_scales   NULL, or device float [N]: s_n per output row (the pages do not say which)
+ *   logits       device float [M][N], 16-byte aligned, output (fp32, rounded once)
+ *   top2         device tl_head_top2 [M], output; token -1 and NaN values for a row with a NaN
+ * Arithmetic: exact f16 operands on the tensor cores (every E4M3 value is an f16 value; X rows
+ * prepared as for TL_PATH_EXACT, with the same fp64 fallback for rows outside f16), fp32
+ * accumulation. Same scratch, allocation and serialisation rules as the calls without a plan
+ * (the prepared-X buffer of the device). Asynchronous on `stream`. */
+#define TL_HEAD_MAX_M 32
+typedef struct {
+    int token;
+    float top1;
+    float top2;
+    float gap_ulp;
+} tl_head_top2;
+tl_status tl_fp8_head(const void* x, int M, const void* w_fp8, int N, int K, float tensor_scale,
+                      const float* row_scales, float* logits, tl_head_top2* top2, void* stream);
+
 /* Synchronise `stream`, then report and clear the device status word:
  * TL_OK, TL_ERR_TIMEOUT (a bounded wait ran out) or TL_ERR_DEVICE_FAULT. Also reads and
  * clears the status word of tl_nvfp4_verify_gemm_noalloc()'s static scratch on the current

@@ -14,7 +14,7 @@ from ._lib import Matrix, TlError, check
 
 __all__ = ["verify_gemm", "verify_gemm_simt", "set_gemm_path", "get_gemm_path", "gemm_path", "PATH_BLOCK_SCALED",
            "PATH_BF16_EXACT", "PATH_EXACT", "verify_stack", "verify_stack_host", "Plan", "dequant",
-           "quantize", "check_device_error", "noalloc_check_error", "init", "num_sms", "Matrix", "TlError"]
+           "quantize", "check_device_error", "noalloc_check_error", "fp8_head", "init", "num_sms", "Matrix", "TlError"]
 
 
 def _stream(stream):
@@ -170,3 +170,30 @@ def check_device_error(stream=None) -> None:
 def noalloc_check_error(stream=None) -> None:
     """Status word of the no-allocation entry point's static scratch (allocation-free)."""
     check(_lib.lib().tl_noalloc_check_error(_stream(stream)))
+
+
+def fp8_head(x, w_fp8, scale, logits=None, stream=None):
+    """FP8 output head: x bf16 [M, K]; w_fp8 uint8 [N, K] (E4M3 bytes); scale a float (per tensor)
+    or a float32 device tensor [N] (per row). Returns (logits float32 [M, N], top2 int32/float32
+    tensor [M, 4] viewed as (token, top1, top2, gap_ulp): the token as int32 bits in column 0)."""
+    import torch
+    M, K = x.shape
+    N = w_fp8.shape[0]
+    if logits is None:
+        logits = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    top2 = torch.empty((M, 4), dtype=torch.int32, device=x.device)
+    if isinstance(scale, (float, int)):
+        ts, rs = float(scale), None
+    else:
+        ts, rs = 0.0, ctypes.c_void_p(scale.data_ptr())
+    check(_lib.lib().tl_fp8_head(_ptr(x), M, _ptr(w_fp8), N, K, ctypes.c_float(ts), rs, _ptr(logits), _ptr(top2),
+                                 _stream(stream)))
+    return logits, top2
+
+
+def head_top2_fields(top2):
+    """(token int64[M], top1, top2, gap float64[M]) from fp8_head's top2 tensor (on the host)."""
+    import numpy as np
+    t = top2.cpu().numpy()
+    return (t[:, 0].astype(np.int64), t[:, 1].view(np.float32).astype(np.float64),
+            t[:, 2].view(np.float32).astype(np.float64), t[:, 3].view(np.float32).astype(np.float64))

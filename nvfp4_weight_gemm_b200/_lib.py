@@ -26,13 +26,18 @@ EXPORTS = (
     "tl_nvfp4_verify_stack", "tl_nvfp4_verify_stack_host", "tl_nvfp4_plan_create",
     "tl_nvfp4_plan_run", "tl_nvfp4_plan_run_host", "tl_nvfp4_plan_destroy", "tl_nvfp4_dequant",
     "tl_nvfp4_quantize", "tl_check_device_error", "tl_selftest_bounded_wait", "tl_num_sms", "tl_status_string",
-    "tl_last_error_message", "tl_set_gemm_path", "tl_get_gemm_path", "tl_noalloc_check_error",
+    "tl_last_error_message", "tl_set_gemm_path", "tl_get_gemm_path", "tl_noalloc_check_error", "tl_fp8_head",
 )
 
 # Tensor-core paths (tl_set_gemm_path).
 TL_PATH_BLOCK_SCALED = 0
 TL_PATH_BF16_EXACT = 1
 TL_PATH_EXACT = 2
+
+
+class HeadTop2(ctypes.Structure):
+    """tl_head_top2."""
+    _fields_ = [("token", ctypes.c_int), ("top1", ctypes.c_float), ("top2", ctypes.c_float), ("gap_ulp", ctypes.c_float)]
 
 
 class TlError(RuntimeError):
@@ -76,6 +81,7 @@ def lib() -> ctypes.CDLL:
             "tl_nvfp4_quantize": [vp, i, i, vp, vp, ctypes.POINTER(f), vp],
             "tl_check_device_error": [vp],
             "tl_noalloc_check_error": [vp],
+            "tl_fp8_head": [vp, i, vp, i, i, f, vp, vp, vp, vp],
             "tl_selftest_bounded_wait": [ctypes.c_uint, vp],
             "tl_num_sms": [i],
             "tl_status_string": [i],

@@ -22,6 +22,7 @@
 #include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
 #include "gemm_ex.cuh"
+#include "gemm_head.cuh"
 #include "xprep.cuh"
 #include "gemm_bs.cuh"
 #include "kernels_aux.cuh"
@@ -1185,6 +1186,20 @@ tl_status plan_create_path(const tl_nvfp4_matrix* mats, int n_mats, int M, int p
 
 }  // namespace
 
+namespace {
+
+template <int NX>
+tl_status launch_head(DevState& d, tl::HeadParams& hp, cudaStream_t stream) {
+    using C = tl::HeadCfg<NX>;
+    TL_CUDA(cudaFuncSetAttribute(tl::gemm_head_kernel<NX>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES));
+    const long long grid = hp.total_tiles < d.num_sms ? hp.total_tiles : d.num_sms;
+    tl::gemm_head_kernel<NX><<<(unsigned)grid, C::THREADS, C::SMEM_BYTES, stream>>>(hp);
+    TL_CUDA(cudaGetLastError());
+    return TL_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 tl_status tl_nvfp4_plan_create(const tl_nvfp4_matrix* mats, int n_mats, int M, tl_nvfp4_plan* plan_out) {
@@ -1401,6 +1416,75 @@ tl_status tl_nvfp4_verify_stack_host(const tl_nvfp4_matrix* mats, int n_mats, in
                    stream);
     if (st != TL_OK) return st;
     TL_CUDA(cudaMemcpyAsync(y_host, y_dev, yb, cudaMemcpyDeviceToHost, s));
+    return TL_OK;
+}
+
+tl_status tl_fp8_head(const void* x, int M, const void* w_fp8, int N, int K, float tensor_scale,
+                      const float* row_scales, float* logits, tl_head_top2* top2, void* stream) {
+    if (M < 0 || M > TL_HEAD_MAX_M) return fail(M < 0 ? TL_ERR_INVALID_VALUE : TL_ERR_UNSUPPORTED,
+                                                "M = %d outside 0..%d rows", M, TL_HEAD_MAX_M);
+    if (N < 2) return fail(TL_ERR_INVALID_VALUE, "N = %d: the head needs at least two rows", N);
+    if (K <= 0 || K % TL_NVFP4_K_ALIGN != 0)
+        return fail(TL_ERR_INVALID_VALUE, "K = %d must be a positive multiple of %d", K, TL_NVFP4_K_ALIGN);
+    if (!x || !w_fp8 || !logits || !top2) return fail(TL_ERR_INVALID_VALUE, "null pointer");
+    if (!aligned16(x) || !aligned16(w_fp8) || !aligned16(logits) || (row_scales && !aligned16(row_scales)))
+        return fail(TL_ERR_MISALIGNED, "x, w, logits and row_scales must be 16-byte aligned");
+    if (!row_scales && !std::isfinite(tensor_scale)) return fail(TL_ERR_INVALID_VALUE, "tensor_scale is not finite");
+    if (overlap(logits, (size_t)4 * M * N, x, (size_t)2 * M * K) || overlap(logits, (size_t)4 * M * N, w_fp8, (size_t)N * K))
+        return fail(TL_ERR_INVALID_VALUE, "logits overlap x or the weights");
+    if (M == 0) return TL_OK;
+    DevState* d = nullptr;
+    tl_status st = current_state(&d);
+    if (st != TL_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = ensure_xh(*d, xh_bytes_of(M, K), s);
+    if (st != TL_OK) return st;
+    // the X preparation: a one-matrix TcParams over the per-device scratch
+    const int NX = M <= 16 ? 16 : 32;
+    tl::TcParams pp;
+    memset(&pp, 0, sizeof pp);
+    unsigned char* xh = d->xh_buf;
+    pp.one.x = static_cast<const __nv_bfloat16*>(x);
+    pp.one.xh = reinterpret_cast<__half*>(xh);
+    pp.one.rowfac = reinterpret_cast<float*>(xh + (((size_t)2 * M * K + 255) & ~size_t(255)));
+    pp.one.rowmask = reinterpret_cast<unsigned*>(reinterpret_cast<unsigned char*>(pp.one.rowfac) +
+                                                 (((size_t)4 * M + 255) & ~size_t(255)));
+    pp.one.K = K;
+    pp.n_mats = 1;
+    pp.M = M;
+    tl::HeadParams hp;
+    memset(&hp, 0, sizeof hp);
+    const cuuint64_t n = (cuuint64_t)N, k = (cuuint64_t)K;
+    st = encode_3d(&hp.tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_fp8, {128, n, k / 128}, {k, 128},
+                   {128, tl::TC_BLOCK_N, 2}, CU_TENSOR_MAP_SWIZZLE_128B, "head weights");
+    if (st != TL_OK) return st;
+    st = encode_3d(&hp.tm_x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xh, {64, (cuuint64_t)M, k / 64}, {k * 2, 128},
+                   {64, (cuuint32_t)NX, 4}, CU_TENSOR_MAP_SWIZZLE_128B, "head X");
+    if (st != TL_OK) return st;
+    hp.w = static_cast<const uint8_t*>(w_fp8);
+    hp.row_scale = row_scales;
+    hp.tensor_scale = tensor_scale;
+    hp.logits = logits;
+    hp.rowfac = pp.one.rowfac;
+    hp.rowmask = pp.one.rowmask;
+    hp.x = static_cast<const __nv_bfloat16*>(x);
+    hp.M = M;
+    hp.N = N;
+    hp.K = K;
+    hp.k_tiles = K / tl::TC_BLOCK_K;
+    hp.n_tiles = (N + tl::TC_BLOCK_N - 1) / tl::TC_BLOCK_N;
+    hp.total_tiles = (long long)hp.k_tiles * hp.n_tiles;
+    hp.partials = d->partials;
+    hp.counters = d->counters;
+    hp.err = d->err;
+    tl::x_prep_kernel<<<dim3(1u, (unsigned)((M + tl::XP_ROWS - 1) / tl::XP_ROWS)), tl::XP_THREADS, 0, s>>>(pp);
+    TL_CUDA(cudaGetLastError());
+    st = (NX == 16) ? launch_head<16>(*d, hp, s) : launch_head<32>(*d, hp, s);
+    if (st != TL_OK) return st;
+    tl::head_fallback_kernel<<<(unsigned)d->num_sms, tl::HEAD_FB_THREADS, 0, s>>>(hp);
+    TL_CUDA(cudaGetLastError());
+    tl::head_top2_kernel<<<(unsigned)M, tl::HEAD_TOP2_THREADS, 0, s>>>(logits, N, reinterpret_cast<tl::HeadTop2*>(top2));
+    TL_CUDA(cudaGetLastError());
     return TL_OK;
 }
 
