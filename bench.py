@@ -45,7 +45,7 @@ WORKLOAD = ("64-layer verify-pass weight stream: 64 x {QKV 5120->7168, O 5120->5
 # exact, so it meets the per-element tolerance on every input; "block-scaled" is approximate
 # (X rewritten as FP4 pieces) and is reported only as a separately labelled run.
 PATHS = {"exact": 2, "bf16-exact": 1, "block-scaled": 0}
-KERNELS = {"exact": "x_prep_kernel + gemm_tc_kernel<NX, f16> + fallback_rows_kernel (three launches per stack pass, "
+KERNELS = {"exact": "x_prep_kernel + gemm_ex_kernel<NX> + fallback_rows_kernel (three launches per stack pass, "
                     "timed together)",
            "bf16-exact": "gemm_tc_kernel<NX, bf16> (one launch per stack pass)",
            "block-scaled": "x_split_kernel + gemm_bs_kernel (two launches per stack pass, timed together)"}
@@ -390,6 +390,9 @@ def main_gpu(args):
     # ---- the benchmarked stack against the oracle, sampled: every matrix, at M = 8, 16, 24, 32
     parity = sampled_parity(tl, stack, xs, ys, plans, stream, rank) if rank == 0 else None
 
+    # ---- the FP8 output head after the stack: vocabulary-sized logits + greedy top-2 per M
+    head = head_figure(tl, dev, stream, rank) if rank == 0 else None
+
     # ---- reduce over ranks: max time, summed bytes
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev, world)
 
@@ -427,6 +430,7 @@ def main_gpu(args):
             "m_invariance_row_fraction": inv,
             "parity_sampled": parity,
             "staircut": cut,
+            "fp8_head": head,
             "cpu_baseline": {"value": round(cb / cs / 1e9, 4), "unit": "GB/s", "cores": cthreads, "kind": "oracle",
                              "sample": CPU_SAMPLE_DESC},
             "e2e": {"value": round(job_gbs(world, bytes_step, e2e_ms), 1), "unit": "GB/s",
@@ -444,7 +448,84 @@ def main_gpu(args):
         print(f"sampled parity: {parity['outside']} of {parity['checked']} outputs outside the tolerance",
               file=sys.stderr, flush=True)
         return 1
+    if head is not None and head["parity_sampled"]["outside"] > 0:
+        print(f"FP8 head sampled parity: {head['parity_sampled']['outside']} logits outside the tolerance",
+              file=sys.stderr, flush=True)
+        return 1
     return 0
+
+
+HEAD_N, HEAD_K = 151936, 5120     # a vocabulary-sized head on the stack's hidden size
+HEAD_M = (1, 8, 16, 17, 24, 32)
+HEAD_REPS = 20
+
+
+def head_bytes(M):
+    """Algorithmic bytes of one head call: E4M3 weights, per-row scales, X, fp32 logits, top-2 records."""
+    return HEAD_N * HEAD_K + 4 * HEAD_N + 2 * M * HEAD_K + 4 * M * HEAD_N + 16 * M
+
+
+def head_figure(tl, dev, stream, rank):
+    """Time tl_fp8_head (X prep + head GEMM + fp64 fallback + top-2: four launches) at a
+    151,936 x 5,120 FP8 head with per-row scales, per M, with CUDA events on the launching stream
+    (the 0.78 GB weight is over six times L2, so no flush), then check sampled logits against the
+    oracle and the top-2 against the kernel's own logits."""
+    import numpy as np
+    import torch
+    import oracle
+    import synth
+    peak, _ = load_peaks()
+    w = synth.w_f32_torch(HEAD_N, HEAD_K, rank, 9000, dev)
+    sc = (w.abs().amax(dim=1) / 448.0).clamp_min(1e-30)
+    wq = (w / sc[:, None]).to(torch.float8_e4m3fn).view(torch.uint8).contiguous()
+    sc = sc.float().contiguous()
+    del w
+    torch.cuda.empty_cache()
+    per_M = {}
+    with torch.cuda.stream(stream):
+        x = synth.x_bf16_torch(max(HEAD_M), HEAD_K, rank, synth.X_ID_BASE + 9000, dev)
+        logits = torch.empty((max(HEAD_M), HEAD_N), dtype=torch.float32, device=dev)
+        for M in HEAD_M:
+            for _ in range(3):
+                tl.fp8_head(x[:M], wq, sc, logits=logits[:M], stream=stream)
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(HEAD_REPS)]
+            for e0, e1 in evs:
+                e0.record(stream)
+                tl.fp8_head(x[:M], wq, sc, logits=logits[:M], stream=stream)
+                e1.record(stream)
+            stream.synchronize()
+            ms = statistics.median(e0.elapsed_time(e1) for e0, e1 in evs)
+            gbs = head_bytes(M) / (ms * 1e-3) / 1e9
+            per_M[str(M)] = {"us": round(ms * 1e3, 1), "gbs": round(gbs, 1), "frac": round(gbs / peak, 4)}
+        # sampled parity at M = 32: 512 seeded columns + the last 16, every row
+        M = max(HEAD_M)
+        lg, top2 = tl.fp8_head(x[:M], wq, sc, logits=logits[:M], stream=stream)
+        stream.synchronize()
+    tl.check_device_error(stream)
+    rng = np.random.default_rng(9000)
+    cols = np.unique(np.concatenate([rng.integers(0, HEAD_N, 512), np.arange(HEAD_N - 16, HEAD_N)]))
+    idx = torch.from_numpy(cols).to(dev)
+    w_s = wq.index_select(0, idx).cpu().numpy()
+    s_s = sc.index_select(0, idx).cpu().numpy().astype(np.float64)
+    xb = x[:M].cpu().view(torch.int16).numpy().view(np.uint16)
+    ref = oracle.fp8_head_logits(xb, w_s, s_s)
+    table = np.array([oracle.e4m3_decode(b) for b in range(256)], dtype=np.float64)
+    xa = np.abs((xb.astype(np.uint32) << 16).view(np.float32).astype(np.float64))
+    tol = 1e-3 * (xa @ np.abs(np.nan_to_num(table[w_s])).T) * np.abs(s_s)[None, :] + 2.0 ** -22 * np.abs(ref)
+    got = lg.index_select(1, idx).cpu().numpy().astype(np.float64)
+    with np.errstate(invalid="ignore"):
+        outside = int((~(np.abs(got - ref) <= tol)).sum())
+    tok, t1, t2, gap = tl.head_top2_fields(top2)
+    o_idx, o_t1, o_t2, _ = oracle.greedy_top2(lg.cpu().numpy().astype(np.float64))
+    top2_ok = bool(np.array_equal(tok, o_idx) and np.array_equal(t1, o_t1) and np.array_equal(t2, o_t2))
+    outside += 0 if top2_ok else 1
+    return {"N": HEAD_N, "K": HEAD_K, "weights": "E4M3, per-row fp32 scale", "per_M": per_M,
+            "min_frac_over_M": round(min(v["frac"] for v in per_M.values()), 4),
+            "bytes": "N*K + 4N + 2MK + 4MN + 16M per call",
+            "kernels": "x_prep_kernel + gemm_head_kernel<NX> + head_fallback_kernel + head_top2_kernel (timed together)",
+            "gap_ulp_at_M32": [round(float(v), 3) for v in gap],
+            "parity_sampled": {"checked": int(got.size), "outside": outside, "top2_matches_own_logits": top2_ok,
+                               "sample": "528 weight rows (512 seeded + last 16), all 32 rows, vs fp64 oracle"}}
 
 
 PARITY_M = (8, 16, 24, 32)
