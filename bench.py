@@ -466,7 +466,7 @@ def head_bytes(M):
 
 
 def head_figure(tl, dev, stream, rank):
-    """Time tl_fp8_head (X prep + head GEMM + fp64 fallback + top-2: four launches) at a
+    """Time tl_fp8_head (X prep + head GEMM + fp64 fallback + two top-2 stages: five launches) at a
     151,936 x 5,120 FP8 head with per-row scales, per M, with CUDA events on the launching stream
     (the 0.78 GB weight is over six times L2, so no flush), then check sampled logits against the
     oracle and the top-2 against the kernel's own logits."""
@@ -522,7 +522,7 @@ def head_figure(tl, dev, stream, rank):
     return {"N": HEAD_N, "K": HEAD_K, "weights": "E4M3, per-row fp32 scale", "per_M": per_M,
             "min_frac_over_M": round(min(v["frac"] for v in per_M.values()), 4),
             "bytes": "N*K + 4N + 2MK + 4MN + 16M per call",
-            "kernels": "x_prep_kernel + gemm_head_kernel<NX> + head_fallback_kernel + head_top2_kernel (timed together)",
+            "kernels": "x_prep_kernel + gemm_head_kernel<NX> + head_fallback_kernel + head_top2_part_kernel + head_top2_final_kernel (timed together)",
             "gap_ulp_at_M32": [round(float(v), 3) for v in gap],
             "parity_sampled": {"checked": int(got.size), "outside": outside, "top2_matches_own_logits": top2_ok,
                                "sample": "528 weight rows (512 seeded + last 16), all 32 rows, vs fp64 oracle"}}
@@ -569,8 +569,9 @@ def sampled_parity(tl, stack, xs, ys, plans, stream, rank):
 
 
 def run_profile_case(args):
-    """Small case for ncu: one matrix (--profile-matrix NxK) or the first L layers of the stack
-    (--profile-layers L), `--reps` launches of one plan at --M rows.
+    """Small case for ncu: one matrix (--profile-matrix NxK), the first L layers of the stack
+    (--profile-layers L), `--reps` launches of one plan at --M rows; or `--reps` calls of the FP8
+    output head (--profile-head) at --M rows.
 
     Inputs are drawn and packed on the device like the stack's; prints one summary line."""
     import torch
@@ -580,6 +581,20 @@ def run_profile_case(args):
     torch.cuda.set_device(dev)
     tl.init(0)
     tl.set_gemm_path(PATHS[args.path])
+    if args.profile_head:
+        w = synth.w_f32_torch(HEAD_N, HEAD_K, 0, 9000, dev)
+        sc = (w.abs().amax(dim=1) / 448.0).clamp_min(1e-30)
+        wq = (w / sc[:, None]).to(torch.float8_e4m3fn).view(torch.uint8).contiguous()
+        sc = sc.float().contiguous()
+        del w
+        x = synth.x_bf16_torch(args.M, HEAD_K, 0, synth.X_ID_BASE + 9000, dev)
+        for _ in range(args.reps):
+            tl.fp8_head(x, wq, sc)
+        torch.cuda.synchronize()
+        tl.check_device_error()
+        print(json.dumps({"profile_case": f"FP8 head {HEAD_N}x{HEAD_K}", "w_bytes": HEAD_N * HEAD_K, "M": args.M,
+                          "reps": args.reps}), flush=True)
+        return 0
     if args.profile_matrix:
         N, K = (int(v) for v in args.profile_matrix.lower().split("x"))
         shapes = [(N, K, "normal")]
@@ -610,6 +625,7 @@ def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--profile-matrix", default=None, help="NxK: run one matrix --reps times (for ncu)")
     ap.add_argument("--profile-layers", type=int, default=0, help="L: run the first L layers of the stack (for ncu)")
+    ap.add_argument("--profile-head", action="store_true", help="run the FP8 output head --reps times (for ncu)")
     ap.add_argument("--M", type=int, default=32)
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--gpus", type=int, default=1)
@@ -624,7 +640,7 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
-    if args.profile_matrix or args.profile_layers:
+    if args.profile_matrix or args.profile_layers or args.profile_head:
         return run_profile_case(args)
     return main_gpu(args)
 

@@ -13,7 +13,8 @@
 // E4M3 value is an f16 normal, so exact), written into tensor memory by CUDA cores; B = X
 // prepared by xprep.cuh (row m times 2^-e_m in f16, exact); fp32 accumulation in tensor memory.
 // The epilogue writes fp32 logits acc * 2^e_m * s_n; rows xprep flags are recomputed in fp64
-// (head_fallback_kernel) and head_top2_kernel reduces every row of logits in a fixed order.
+// (head_fallback_kernel), and two small kernels reduce every row of logits to its top two
+// (head_top2_part_kernel over chunks of the row, head_top2_final_kernel over the chunks).
 //
 // Tile: 128 weight rows x 256 k (32 KiB of E4M3 bytes, two 128-byte swizzled slices per row);
 // roles and stream-K split as in gemm_ex.cuh (weight producer, X producer, 4 MMA issuers,
@@ -444,7 +445,7 @@ struct HeadTop2 {
     float top1, top2, gap_ulp;
 };
 
-constexpr int HEAD_TOP2_THREADS = 512;
+constexpr int HEAD_TOP2_THREADS = 256;
 
 struct T2 {
     float v1, v2;
@@ -472,16 +473,7 @@ __device__ __forceinline__ float bf16_ulp_f(float v) {
     return ldexpf(1.0f, e - 7);
 }
 
-__global__ void __launch_bounds__(HEAD_TOP2_THREADS) head_top2_kernel(const float* logits, int N, HeadTop2* out) {
-    const int m = blockIdx.x;
-    const float* row = logits + (size_t)m * N;
-    T2 t = {-INFINITY, -INFINITY, 0x7FFFFFFF, 0};
-    for (int n = threadIdx.x; n < N; n += HEAD_TOP2_THREADS) {
-        const float v = row[n];
-        if (isnan(v)) { t.nan = 1; continue; }
-        T2 e = {v, -INFINITY, n, 0};
-        t = t2_merge(t, e);
-    }
+__device__ __forceinline__ T2 t2_warp_merge(T2 t) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         T2 u;
@@ -491,22 +483,53 @@ __global__ void __launch_bounds__(HEAD_TOP2_THREADS) head_top2_kernel(const floa
         u.nan = __shfl_xor_sync(0xFFFFFFFFu, t.nan, o);
         t = t2_merge(t, u);
     }
-    __shared__ T2 part[HEAD_TOP2_THREADS / 32];
+    return t;
+}
+
+// Stage 1: grid (chunks, M); CTA (c, m) reduces logits[m][c * chunk, (c + 1) * chunk) to one
+// partial. The merge keeps the largest value (lowest index among equal ones) and the largest of
+// the rest, so the two stages give the same answer in any order of merging.
+__global__ void __launch_bounds__(HEAD_TOP2_THREADS) head_top2_part_kernel(const float* logits, int N, int chunk,
+                                                                           T2* part) {
+    const int c = blockIdx.x, m = blockIdx.y;
+    const float* row = logits + (size_t)m * N;
+    const int n0 = c * chunk, n1 = min(N, n0 + chunk);
+    T2 t = {-INFINITY, -INFINITY, 0x7FFFFFFF, 0};
+    for (int n = n0 + (int)threadIdx.x; n < n1; n += HEAD_TOP2_THREADS) {
+        const float v = __ldcg(row + n);
+        if (isnan(v)) { t.nan = 1; continue; }
+        const T2 e = {v, -INFINITY, n, 0};
+        t = t2_merge(t, e);
+    }
+    t = t2_warp_merge(t);
+    __shared__ T2 ws[HEAD_TOP2_THREADS / 32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (lane == 0) part[warp] = t;
+    if (lane == 0) ws[warp] = t;
     __syncthreads();
     if (threadIdx.x == 0) {
-        T2 r = part[0];
-        for (int w = 1; w < HEAD_TOP2_THREADS / 32; ++w) r = t2_merge(r, part[w]);
+        T2 r = ws[0];
+        for (int w = 1; w < HEAD_TOP2_THREADS / 32; ++w) r = t2_merge(r, ws[w]);
+        part[(size_t)m * gridDim.x + c] = r;
+    }
+}
+
+// Stage 2: one warp per row merges the row's partials and writes the token, the two best values
+// and their gap in bf16 units in the last place at the largest (token -1 and NaN for a row with a NaN).
+__global__ void __launch_bounds__(32) head_top2_final_kernel(const T2* part, int chunks, HeadTop2* out) {
+    const int m = blockIdx.x, lane = threadIdx.x;
+    T2 t = {-INFINITY, -INFINITY, 0x7FFFFFFF, 0};
+    for (int c = lane; c < chunks; c += 32) t = t2_merge(t, part[(size_t)m * chunks + c]);
+    t = t2_warp_merge(t);
+    if (lane == 0) {
         HeadTop2 o;
-        if (r.nan) {
+        if (t.nan) {
             o.token = -1;
             o.top1 = o.top2 = o.gap_ulp = __int_as_float(0x7FC00000);
         } else {
-            o.token = r.i1;
-            o.top1 = r.v1;
-            o.top2 = r.v2;
-            o.gap_ulp = (r.v1 - r.v2) / bf16_ulp_f(r.v1);
+            o.token = t.i1;
+            o.top1 = t.v1;
+            o.top2 = t.v2;
+            o.gap_ulp = (t.v1 - t.v2) / bf16_ulp_f(t.v1);
         }
         out[m] = o;
     }

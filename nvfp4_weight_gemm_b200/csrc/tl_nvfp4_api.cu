@@ -279,12 +279,11 @@ tl_status launch_ex(DevState& d, tl::TcParams& p, cudaStream_t stream) {
 }
 
 // The exact paths. bf16 decode: one GEMM launch on X as given. f16 decode: the X preparation
-// (one CTA per matrix and group of 8 rows), the GEMM on the prepared X, then the fallback for flagged rows (it
+// (one CTA per matrix and row), the GEMM on the prepared X, then the fallback for flagged rows (it
 // returns at once when no row is flagged).
 tl_status launch_tc_any(DevState& d, tl::TcParams& p, bool f16, cudaStream_t stream) {
     if (!f16) return (p.M <= 16) ? launch_tc<16>(d, p, stream) : launch_tc<32>(d, p, stream);
-    tl::x_prep_kernel<<<dim3((unsigned)p.n_mats, (unsigned)((p.M + tl::XP_ROWS - 1) / tl::XP_ROWS)), tl::XP_THREADS, 0,
-                        stream>>>(p);
+    tl::x_prep_kernel<<<dim3((unsigned)p.n_mats, (unsigned)p.M), tl::XP_THREADS, 0, stream>>>(p);
     TL_CUDA(cudaGetLastError());
     tl_status st = (p.M <= 16) ? launch_ex<16>(d, p, stream) : launch_ex<32>(d, p, stream);
     if (st != TL_OK) return st;
@@ -1477,13 +1476,22 @@ tl_status tl_fp8_head(const void* x, int M, const void* w_fp8, int N, int K, flo
     hp.partials = d->partials;
     hp.counters = d->counters;
     hp.err = d->err;
-    tl::x_prep_kernel<<<dim3(1u, (unsigned)((M + tl::XP_ROWS - 1) / tl::XP_ROWS)), tl::XP_THREADS, 0, s>>>(pp);
+    tl::x_prep_kernel<<<dim3(1u, (unsigned)M), tl::XP_THREADS, 0, s>>>(pp);
     TL_CUDA(cudaGetLastError());
     st = (NX == 16) ? launch_head<16>(*d, hp, s) : launch_head<32>(*d, hp, s);
     if (st != TL_OK) return st;
     tl::head_fallback_kernel<<<(unsigned)d->num_sms, tl::HEAD_FB_THREADS, 0, s>>>(hp);
     TL_CUDA(cudaGetLastError());
-    tl::head_top2_kernel<<<(unsigned)M, tl::HEAD_TOP2_THREADS, 0, s>>>(logits, N, reinterpret_cast<tl::HeadTop2*>(top2));
+    // top-2 in two stages over at most 1024 chunks of a row (the partials reuse the split-K scratch,
+    // free again once the GEMM has run on this stream)
+    int chunk = (N + 1023) / 1024;
+    chunk = ((chunk < 4096 ? 4096 : chunk) + 255) & ~255;
+    const int chunks = (N + chunk - 1) / chunk;
+    tl::T2* part = reinterpret_cast<tl::T2*>(d->partials);
+    tl::head_top2_part_kernel<<<dim3((unsigned)chunks, (unsigned)M), tl::HEAD_TOP2_THREADS, 0, s>>>(logits, N, chunk,
+                                                                                               part);
+    TL_CUDA(cudaGetLastError());
+    tl::head_top2_final_kernel<<<(unsigned)M, 32, 0, s>>>(part, chunks, reinterpret_cast<tl::HeadTop2*>(top2));
     TL_CUDA(cudaGetLastError());
     return TL_OK;
 }

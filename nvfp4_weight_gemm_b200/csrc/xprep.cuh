@@ -35,77 +35,75 @@ constexpr int XP_EMIN = -60, XP_EMAX = 60;   // e_m range with a normal epilogue
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// Grid (matrices, ceil(M / 8)): CTA (i, g) prepares rows 8g .. 8g + 7 of matrix i, one warp per
-// row, and writes byte g of the matrix's row mask (bit j: row 8g + j flagged). Every lane keeps
-// four 16-byte loads in flight.
-constexpr int XP_ROWS = XP_THREADS / 32;
-constexpr int XP_UNROLL = 4;
-
+// Grid (matrices, M): CTA (i, r) prepares row r of matrix i, its 256 threads over the row's
+// 16-byte chunks. A first pass finds the row's largest |x| (and any NaN or infinity), a second
+// re-reads the row (from L1) and writes it scaled; the CTA then sets or clears bit r of the
+// matrix's row mask with one atomic, so concurrent rows of one matrix never race on it.
 __global__ void __launch_bounds__(XP_THREADS) x_prep_kernel(const __grid_constant__ TcParams p) {
     const TcMat& m = p.mats ? p.mats[blockIdx.x] : p.one;
-    __shared__ unsigned mask_s;
-    if (threadIdx.x == 0) mask_s = 0u;
-    __syncthreads();
+    constexpr int W = XP_THREADS / 32;
+    __shared__ float amax_s[W];
+    __shared__ int bad_s[W], inexact_s[W];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int r = blockIdx.y * XP_ROWS + warp;
-    const int K = m.K, chunks = K / 8;   // K is a multiple of 256: chunks is a multiple of 32
-    if (r < p.M) {
-        const uint4* xr = reinterpret_cast<const uint4*>(m.x + (size_t)r * K);
-        float amax = 0.0f;
-        bool bad = false;
-        for (int c0 = lane; c0 < chunks; c0 += 32 * XP_UNROLL) {
-            uint4 v[XP_UNROLL];
+    const int r = blockIdx.y;
+    const int K = m.K, chunks = K / 8;   // K is a multiple of 256
+    const uint4* xr = reinterpret_cast<const uint4*>(m.x + (size_t)r * K);
+    float amax = 0.0f;
+    bool bad = false;
+    for (int c = threadIdx.x; c < chunks; c += XP_THREADS) {
+        const uint4 v = __ldg(xr + c);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int u = 0; u < XP_UNROLL; ++u) v[u] = (c0 + 32 * u < chunks) ? __ldg(xr + c0 + 32 * u) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-            for (int u = 0; u < XP_UNROLL; ++u) {
-                const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float a = bf16_lo(w[j]), b = bf16_hi(w[j]);
-                    bad |= !isfinite(a) || !isfinite(b);
-                    amax = fmaxf(amax, fmaxf(fabsf(a), fabsf(b)));
-                }
-            }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-        bad = __any_sync(0xFFFFFFFFu, bad);
-        int e = 0;
-        if (!bad && amax > 0.0f) {
-            e = ilogbf(amax) - 15;   // largest |x| * 2^-e in [2^15, 2^16)
-            if (e < XP_EMIN || e > XP_EMAX) bad = true;
-        }
-        if (bad) e = 0;
-        const float down = ldexpf(1.0f, -e);
-        uint4* xo = reinterpret_cast<uint4*>(m.xh + (size_t)r * K);
-        bool inexact = false;
-        for (int c0 = lane; c0 < chunks; c0 += 32 * XP_UNROLL) {
-            uint4 v[XP_UNROLL];
-#pragma unroll
-            for (int u = 0; u < XP_UNROLL; ++u) v[u] = (c0 + 32 * u < chunks) ? __ldg(xr + c0 + 32 * u) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-            for (int u = 0; u < XP_UNROLL; ++u) {
-                const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-                uint32_t o[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float a = bf16_lo(w[j]) * down, b = bf16_hi(w[j]) * down;   // exact (power of two)
-                    const __half ha = __float2half_rn(a), hb = __float2half_rn(b);
-                    inexact |= (__half2float(ha) != a) || (__half2float(hb) != b);
-                    o[j] = (uint32_t)__half_as_ushort(ha) | ((uint32_t)__half_as_ushort(hb) << 16);
-                }
-                if (c0 + 32 * u < chunks) xo[c0 + 32 * u] = make_uint4(o[0], o[1], o[2], o[3]);
-            }
-        }
-        inexact = __any_sync(0xFFFFFFFFu, inexact);
-        if (lane == 0) {
-            m.rowfac[r] = ldexpf(1.0f, e);
-            if (bad || inexact) atomicOr(&mask_s, 1u << warp);
+        for (int j = 0; j < 4; ++j) {
+            const float a = bf16_lo(w[j]), b = bf16_hi(w[j]);
+            bad |= !isfinite(a) || !isfinite(b);
+            amax = fmaxf(amax, fmaxf(fabsf(a), fabsf(b)));
         }
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+    bad = __any_sync(0xFFFFFFFFu, bad);
+    if (lane == 0) { amax_s[warp] = amax; bad_s[warp] = bad ? 1 : 0; }
     __syncthreads();
-    if (threadIdx.x == 0) reinterpret_cast<uint8_t*>(m.rowmask)[blockIdx.y] = (uint8_t)mask_s;
+    amax = amax_s[0];
+    int anybad = bad_s[0];
+#pragma unroll
+    for (int i = 1; i < W; ++i) { amax = fmaxf(amax, amax_s[i]); anybad |= bad_s[i]; }
+    bad = anybad != 0;
+    int e = 0;
+    if (!bad && amax > 0.0f) {
+        e = ilogbf(amax) - 15;   // largest |x| * 2^-e in [2^15, 2^16)
+        if (e < XP_EMIN || e > XP_EMAX) bad = true;
+    }
+    if (bad) e = 0;
+    const float down = ldexpf(1.0f, -e);
+    uint4* xo = reinterpret_cast<uint4*>(m.xh + (size_t)r * K);
+    bool inexact = false;
+    for (int c = threadIdx.x; c < chunks; c += XP_THREADS) {
+        const uint4 v = __ldg(xr + c);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float a = bf16_lo(w[j]) * down, b = bf16_hi(w[j]) * down;   // exact (power of two)
+            const __half ha = __float2half_rn(a), hb = __float2half_rn(b);
+            inexact |= (__half2float(ha) != a) || (__half2float(hb) != b);
+            o[j] = (uint32_t)__half_as_ushort(ha) | ((uint32_t)__half_as_ushort(hb) << 16);
+        }
+        xo[c] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    inexact = __any_sync(0xFFFFFFFFu, inexact);
+    if (lane == 0) inexact_s[warp] = inexact ? 1 : 0;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int flagged = bad ? 1 : 0;
+#pragma unroll
+        for (int i = 0; i < W; ++i) flagged |= inexact_s[i];
+        m.rowfac[r] = ldexpf(1.0f, e);
+        const unsigned bit = 1u << r;
+        if (flagged) atomicOr(m.rowmask, bit);
+        else atomicAnd(m.rowmask, ~bit);
+    }
 }
 
 // Recompute the flagged rows: y[r][n] = bf16( g * sum_b e4m3(s[n][b]) * sum_{k in b} x[r][k] * e2m1(c[n][k]) )
@@ -122,7 +120,7 @@ __global__ void __launch_bounds__(FB_THREADS) fallback_rows_kernel(const __grid_
         if (i < p.n_mats) {
             const TcMat& mm = p.mats ? p.mats[i] : p.one;
             mk = __ldcg(mm.rowmask);
-            // bytes of the mask past the launch's row groups can hold another call's bits
+            // bits of rows past M can hold another call's flags
             if (p.M < 32) mk &= (1u << p.M) - 1u;
         }
         unsigned any = __ballot_sync(0xFFFFFFFFu, mk != 0u);
