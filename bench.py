@@ -20,7 +20,6 @@ from __future__ import annotations
 
 import argparse
 import ctypes
-import glob
 import hashlib
 import json
 import os
@@ -86,10 +85,18 @@ def load_peaks():
     return 6650.0, "fallback"
 
 
-def source_hash():
+# the device code of each path: a recorded DRAM figure holds while these files are unchanged
+PATH_SOURCES = {
+    "exact": ("gemm_ex.cuh", "gemm_tc.cuh", "xprep.cuh", "ptx.cuh", "nvfp4_format.cuh"),
+    "bf16-exact": ("gemm_tc.cuh", "ptx.cuh", "nvfp4_format.cuh"),
+    "block-scaled": ("gemm_bs.cuh", "xsplit.cuh", "ptx.cuh", "nvfp4_format.cuh"),
+}
+
+
+def source_hash(path="exact"):
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "nvfp4_weight_gemm_b200", "csrc", "*"))):
-        h.update(open(f, "rb").read())
+    for f in PATH_SOURCES[path]:
+        h.update(open(os.path.join(ROOT, "nvfp4_weight_gemm_b200", "csrc", f), "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -101,7 +108,7 @@ def profiled_traffic(shapes, path):
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
-    if d.get("source_hash") != source_hash() or not d.get("kernels", "").startswith(KERNELS[path].split(" (")[0]):
+    if d.get("source_hash") != source_hash(path) or not d.get("kernels", "").startswith(KERNELS[path].split(" (")[0]):
         return None
     pts = sorted((int(m), v["ratio"]) for m, v in d["per_M"].items())
 

@@ -209,12 +209,16 @@ __global__ void __launch_bounds__(HeadCfg<NX>::THREADS, 1) gemm_head_kernel(cons
         }
     } else if (head_issuer_of_warp(warp) >= 0) {
         // ------------------------------------------------------------ MMA issuers (k-steps 4j .. 4j + 3)
-        const int j = head_issuer_of_warp(warp);
+        // warp-uniform operands (lane-0 shuffles), as in gemm_ex_kernel
+        const int j = __shfl_sync(0xFFFFFFFFu, head_issuer_of_warp(warp), 0);
         const int i0 = 4 * j;
         const bool leader = elect_one();
         int a = 0, acc = 0;
         uint32_t aph = 0, accph = 0;
-        const uint64_t bdesc_base = smem_desc_k_sw128(smem_u32(smem + C::X_RING));
+        const uint32_t tmem_u = __shfl_sync(0xFFFFFFFFu, tmem, 0);
+        const uint64_t bdesc_raw = smem_desc_k_sw128(smem_u32(smem + C::X_RING));
+        const uint64_t bdesc_base = ((uint64_t)__shfl_sync(0xFFFFFFFFu, (uint32_t)(bdesc_raw >> 32), 0) << 32) |
+                                    (uint64_t)__shfl_sync(0xFFFFFFFFu, (uint32_t)bdesc_raw, 0);
         HeadSegIter it(p.k_tiles, t_begin, t_end);
         HeadSeg sg;
         bool ok = true;
@@ -224,7 +228,7 @@ __global__ void __launch_bounds__(HeadCfg<NX>::THREADS, 1) gemm_head_kernel(cons
                 break;
             }
             tc_fence_after();
-            const uint32_t d_tmem = tmem + (uint32_t)(C::ACC_COL0 + C::ACC_BUF_COLS * acc + NX * j);
+            const uint32_t d_tmem = tmem_u + (uint32_t)(C::ACC_COL0 + C::ACC_BUF_COLS * acc + NX * j);
             uint32_t first = 1;
             for (int kt = sg.k0; kt < sg.k1; ++kt) {
                 if (!__all_sync(0xFFFFFFFFu, tc_wait(&ready[a], aph, abort_flag))) {
@@ -234,7 +238,7 @@ __global__ void __launch_bounds__(HeadCfg<NX>::THREADS, 1) gemm_head_kernel(cons
                 }
                 tc_fence_after();
                 const uint64_t bdesc0 = bdesc_base + (uint64_t)((a * C::X_BYTES) >> 4);
-                const uint32_t a_tmem = tmem + (uint32_t)(128 * a + 8 * i0);
+                const uint32_t a_tmem = tmem_u + (uint32_t)(128 * a + 8 * i0);
                 if (leader) {
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
