@@ -195,6 +195,16 @@ CPU_SAMPLE_DESC = (f"{CPU_ROWS} weight rows of each layer shape (QKV, O, gate+up
                    f"fp64 oracle GEMM, GB/s over the same algorithmic bytes")
 
 
+def arm_config(path, world):
+    """The `config` of the bench line; the reference arm prints the same one (its sample of the
+    workload is named in its `cpu_baseline`)."""
+    shapes = stack_shapes()
+    return {"workload": WORKLOAD, "path": path, "arithmetic": ARITHMETIC[path], "matrices": len(shapes),
+            "weights": sum(N * K for (_, _, _, N, K, _) in shapes), "w_bytes": w_bytes(shapes),
+            "M": "1..32 (one pass each per step)", "l2": "working set 11.9 GB >> 126 MB L2; no flush needed",
+            "parallelism": f"replicas x{world}"}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -213,7 +223,7 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "sample": CPU_SAMPLE_DESC},
+        "config": arm_config(args.path, int(os.environ.get("WORLD_SIZE", "1"))),
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": CPU_SAMPLE_DESC},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -426,9 +436,7 @@ def main_gpu(args):
             "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": DTYPES[args.path], "data": "synthetic",
-            "config": {"workload": WORKLOAD, "path": args.path, "arithmetic": ARITHMETIC[args.path], "matrices": len(shapes), "weights": sum(N * K for (_, _, _, N, K, _) in shapes),
-                       "w_bytes": w_bytes(shapes), "M": "1..32 (one pass each per step)",
-                       "l2": "working set 11.9 GB >> 126 MB L2; no flush needed", "parallelism": f"replicas x{world}"},
+            "config": arm_config(args.path, world),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": traffic, "peak_kind": peak_kind,
                          "kernel": KERNELS[args.path]},
