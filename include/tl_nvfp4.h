@@ -97,7 +97,7 @@ typedef enum {
  *
  * TL_PATH_BF16_EXACT. The same exact arithmetic with the bf16 MMA: CUDA cores decode each
  * weight to bf16 with integer bit operations and X is used as given (no preparation, no
- * scratch). About half as fast: its decode is bound by the integer pipe.
+ * scratch). Slower: its decode is bound by the integer pipe.
  *
  * TL_PATH_BLOCK_SCALED (approximate; not the default). Before the GEMM, a small kernel
  * writes each row of X as a power of two times a sum of four NVFP4-shaped pieces (E2M1
