@@ -4,8 +4,10 @@ TEST INFRASTRUCTURE ONLY. Only the tests, ``__graft_entry__.smoke()`` and the
 benchmark's CPU-baseline leg may import this package. The GPU library never
 imports it and shares no code with it.
 
-It also holds, in numpy fp64, the oracle of the next row: the FP8 output head's logits and the
-greedy top-2 / near-tie statistic (end of this file).
+It also holds, in numpy fp64, the oracles of two next rows: the FP8 output head's logits and the
+greedy top-2 / near-tie statistic, and the closed-form commit of an accepted draft path through a
+Gated DeltaNet state (end of this file; that one's parity against the pages is unpinned, as they
+print no equation).
 
 The C source computes everything in fp64 from the format definitions:
 E2M1 codes (two per byte, low nibble = even k), one E4M3 scale per 16-element
@@ -233,3 +235,67 @@ def greedy_top2(logits: np.ndarray):
         top2[m] = rest.max()
         gap[m] = (top1[m] - top2[m]) / bf16_ulp(top1[m])
     return idx, top1, top2, gap
+
+
+# ---------------------------------------------------------------- GDN closed-form commit (next row)
+#
+# 48 of the served model's 64 layers are Gated DeltaNet layers whose recurrent state cannot step
+# back after a wrong guess, so the engine commits the state of the accepted path in closed form
+# (TandemLLM docs v0.12.0, "What TandemLLM is", section 1.7; the author's "Research" page,
+# StairCut abstract). The pages give no equations. Reading taken here: the state of one head is
+# S (d_v x d_k) and one token with key k, value v, gate alpha in (0, 1] and step beta in [0, 1]
+# updates it by the gated delta rule
+#
+#     S_t = alpha_t * S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
+#
+# and "committing the accepted path" means producing S_L, the state after the path's L tokens
+# (taken in order from the draft tree's nodes), from S_0 in one batched step instead of L
+# sequential updates. PARITY UNPINNED against the pages (they print no equation or value); the
+# functions below are pinned against each other, against exact rational arithmetic and against
+# the properties of the rule in tests/test_oracle_pins.py.
+
+def gdn_sequential(S0: np.ndarray, K: np.ndarray, V: np.ndarray, alpha: np.ndarray, beta: np.ndarray) -> np.ndarray:
+    """The definition: L sequential gated-delta updates of S0 (d_v x d_k) in fp64, token t with
+    key K[t] (d_k), value V[t] (d_v), gate alpha[t], step beta[t]."""
+    S = np.array(S0, dtype=np.float64)
+    for k, v, a, b in zip(np.asarray(K, np.float64), np.asarray(V, np.float64), np.asarray(alpha, np.float64),
+                          np.asarray(beta, np.float64)):
+        S = a * (S - b * np.outer(S @ k, k)) + b * np.outer(v, k)
+    return S
+
+
+def gdn_commit_closed_form(S0: np.ndarray, K: np.ndarray, V: np.ndarray, alpha: np.ndarray,
+                           beta: np.ndarray) -> np.ndarray:
+    """The same state in closed form, in fp64.
+
+    Write the rule as S_t = alpha_t S_{t-1} + u_t k_t^T with u_t = beta_t (v_t - alpha_t S_{t-1} k_t),
+    and let g_t = alpha_1 ... alpha_t (g_0 = 1). Unrolling S_{t-1} gives, for the columns u_t of U:
+        u_t + sum_{s<t} beta_t (g_t / g_s) (k_s . k_t) u_s = beta_t (v_t - g_t S_0 k_t),
+    a unit lower-triangular system (I + A) in the path's order, so
+        U = ((V^T - S_0 K^T G) B) (I + A)^-T,      S_L = g_L S_0 + U diag(g_L / g_t) K
+    with G = diag(g), B = diag(beta) and K holding one key per row. The triangular solve is a
+    library routine; everything else is written out."""
+    S0 = np.asarray(S0, np.float64)
+    K = np.asarray(K, np.float64)
+    V = np.asarray(V, np.float64)
+    a = np.asarray(alpha, np.float64)
+    b = np.asarray(beta, np.float64)
+    L = K.shape[0]
+    if L == 0:
+        return S0.copy()
+    g = np.cumprod(a)                                   # g_t, t = 1..L
+    A = np.zeros((L, L))
+    for t in range(L):
+        for s in range(t):
+            A[t, s] = b[t] * (np.prod(a[s + 1:t + 1])) * float(K[s] @ K[t])
+    R = (V.T - (S0 @ K.T) * g[None, :]) * b[None, :]    # d_v x L: beta_t (v_t - g_t S0 k_t)
+    # U (I + A)^T = R  <=>  (I + A) U^T = R^T
+    U = np.linalg.solve(np.eye(L) + A, R.T).T
+    decay = np.array([np.prod(a[t + 1:]) for t in range(L)])   # g_L / g_t
+    return g[-1] * S0 + (U * decay[None, :]) @ K
+
+
+def gdn_path_inputs(K_nodes, V_nodes, alpha_nodes, beta_nodes, path):
+    """Gather one head's path inputs from per-node arrays of a draft tree (node-major)."""
+    p = np.asarray(path, dtype=np.int64)
+    return (np.asarray(K_nodes)[p], np.asarray(V_nodes)[p], np.asarray(alpha_nodes)[p], np.asarray(beta_nodes)[p])

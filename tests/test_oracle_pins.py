@@ -415,3 +415,112 @@ def test_greedy_top2_hand_worked(orc):
     assert math.isnan(gap[4]) and math.isnan(t1[4])
     with pytest.raises(ValueError):
         orc.greedy_top2(np.zeros((2, 1)))
+
+
+# ---------------------------------------------------------------- GDN closed-form commit
+
+def _gdn_cases():
+    rows = read_golden("gdn_worked.txt")
+    cases, cur = [], None
+    for r in rows:
+        if r[0] == "case":
+            cur = {"alpha": float(r[2]), "beta": float(r[3])}
+            cases.append(cur)
+        else:
+            cur[r[0]] = np.array([float(x) for x in r[1:]])
+    return cases
+
+
+def test_gdn_one_token_hand_worked(orc):
+    for c in _gdn_cases():
+        S0 = c["S0"].reshape(2, 2)
+        K, V = c["k"][None, :], c["v"][None, :]
+        for fn in (orc.gdn_sequential, orc.gdn_commit_closed_form):
+            S1 = fn(S0, K, V, [c["alpha"]], [c["beta"]])
+            assert np.allclose(S1.reshape(-1), c["S1"], rtol=0, atol=1e-12), (fn.__name__, S1)
+
+
+def _gdn_exact(S0, K, V, alpha, beta):
+    # the rule token by token in exact rational arithmetic
+    S = [[Fraction(x) for x in row] for row in S0]
+    for k, v, a, b in zip(K, V, alpha, beta):
+        k = [Fraction(x) for x in k]
+        Sk = [sum(S[i][j] * k[j] for j in range(len(k))) for i in range(len(S))]
+        S = [[Fraction(a) * (S[i][j] - Fraction(b) * Sk[i] * k[j]) + Fraction(b) * Fraction(v[i]) * k[j]
+              for j in range(len(k))] for i in range(len(S))]
+    return np.array([[float(x) for x in row] for row in S])
+
+
+def test_gdn_closed_form_matches_exact_rationals(orc):
+    # small dyadic inputs: every step is exact in rationals; the closed form (a triangular solve
+    # in fp64) must land on the same state
+    rng = np.random.default_rng(11)
+    for L, dk, dv in ((1, 2, 2), (3, 3, 2), (4, 2, 3), (6, 4, 4)):
+        S0 = rng.integers(-4, 5, (dv, dk)) / 4.0
+        K = rng.integers(-2, 3, (L, dk)) / 2.0
+        V = rng.integers(-4, 5, (L, dv)) / 4.0
+        alpha = rng.choice([0.5, 0.75, 1.0], L)
+        beta = rng.choice([0.0, 0.25, 0.5, 1.0], L)
+        ref = _gdn_exact(S0, K, V, alpha, beta)
+        got = orc.gdn_commit_closed_form(S0, K, V, alpha, beta)
+        assert np.allclose(got, ref, rtol=1e-12, atol=1e-12 * max(1.0, np.abs(ref).max()))
+        assert np.allclose(orc.gdn_sequential(S0, K, V, alpha, beta), ref, rtol=0, atol=1e-12 * max(1.0, np.abs(ref).max()))
+
+
+def test_gdn_special_cases(orc):
+    rng = np.random.default_rng(12)
+    dk, dv, L = 16, 8, 7
+    S0 = rng.standard_normal((dv, dk))
+    K = rng.standard_normal((L, dk))
+    V = rng.standard_normal((L, dv))
+    alpha = rng.uniform(0.5, 1.0, L)
+    # beta = 0: only the gates act, S_L = (alpha_1 ... alpha_L) S_0
+    got = orc.gdn_commit_closed_form(S0, K, V, alpha, np.zeros(L))
+    assert np.allclose(got, np.prod(alpha) * S0, rtol=1e-14, atol=0)
+    # beta = 0 and alpha = 1: nothing changes; an empty path changes nothing either
+    assert np.array_equal(orc.gdn_commit_closed_form(S0, K, V, np.ones(L), np.zeros(L)), S0)
+    assert np.array_equal(orc.gdn_commit_closed_form(S0, K[:0], V[:0], alpha[:0], alpha[:0]), S0)
+
+
+def test_gdn_orthonormal_keys_write_their_values(orc):
+    # alpha = beta = 1 with orthonormal keys: the delta rule stores v_t at k_t exactly and leaves
+    # every direction orthogonal to the keys as it was
+    rng = np.random.default_rng(13)
+    dk, dv, L = 32, 16, 12
+    Q, _ = np.linalg.qr(rng.standard_normal((dk, dk)))
+    K = Q[:, :L].T
+    V = rng.standard_normal((L, dv))
+    S0 = rng.standard_normal((dv, dk))
+    SL = orc.gdn_commit_closed_form(S0, K, V, np.ones(L), np.ones(L))
+    assert np.allclose(SL @ K.T, V.T, atol=1e-12)
+    q = Q[:, L]
+    assert np.allclose(SL @ q, S0 @ q, atol=1e-12)
+
+
+def test_gdn_commit_composes_and_matches_the_recurrence(orc):
+    rng = np.random.default_rng(14)
+    dk, dv, L = 128, 128, 32
+    S0 = rng.standard_normal((dv, dk)) * 0.1
+    K = rng.standard_normal((L, dk))
+    K /= np.linalg.norm(K, axis=1, keepdims=True)
+    V = rng.standard_normal((L, dv))
+    alpha = rng.uniform(0.9, 1.0, L)
+    beta = rng.uniform(0.0, 1.0, L)
+    full = orc.gdn_commit_closed_form(S0, K, V, alpha, beta)
+    seq = orc.gdn_sequential(S0, K, V, alpha, beta)
+    assert np.allclose(full, seq, rtol=0, atol=1e-12)
+    a = 13
+    first = orc.gdn_commit_closed_form(S0, K[:a], V[:a], alpha[:a], beta[:a])
+    both = orc.gdn_commit_closed_form(first, K[a:], V[a:], alpha[a:], beta[a:])
+    assert np.allclose(both, full, rtol=0, atol=1e-12)
+
+
+def test_gdn_path_gather(orc):
+    # a draft tree of 5 nodes; the accepted path 0 -> 2 -> 4 takes those nodes' inputs in order
+    rng = np.random.default_rng(15)
+    Kn, Vn = rng.standard_normal((5, 4)), rng.standard_normal((5, 3))
+    an, bn = rng.uniform(0.5, 1, 5), rng.uniform(0, 1, 5)
+    K, V, a, b = orc.gdn_path_inputs(Kn, Vn, an, bn, [0, 2, 4])
+    assert np.array_equal(K, Kn[[0, 2, 4]]) and np.array_equal(b, bn[[0, 2, 4]])
+    S0 = rng.standard_normal((3, 4))
+    assert np.allclose(orc.gdn_commit_closed_form(S0, K, V, a, b), orc.gdn_sequential(S0, K, V, a, b), atol=1e-13)
