@@ -409,6 +409,8 @@ def main_gpu(args):
 
     # ---- the FP8 output head after the stack: vocabulary-sized logits + greedy top-2 per M
     head = head_figure(tl, dev, stream, rank) if rank == 0 else None
+    # ---- the closed-form commit of the accepted path through the GDN layers' states
+    gdn = gdn_figure(tl, dev, stream, rank) if rank == 0 else None
 
     # ---- reduce over ranks: max time, summed bytes
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev, world)
@@ -446,6 +448,7 @@ def main_gpu(args):
             "parity_sampled": parity,
             "staircut": cut,
             "fp8_head": head,
+            "gdn_commit": gdn,
             "cpu_baseline": {"value": round(cb / cs / 1e9, 4), "unit": "GB/s", "cores": cthreads, "kind": "oracle",
                              "sample": CPU_SAMPLE_DESC},
             "e2e": {"value": round(job_gbs(world, bytes_step, e2e_ms), 1), "unit": "GB/s",
@@ -463,11 +466,76 @@ def main_gpu(args):
         print(f"sampled parity: {parity['outside']} of {parity['checked']} outputs outside the tolerance",
               file=sys.stderr, flush=True)
         return 1
+    if gdn is not None and gdn["parity_sampled"]["outside"] > 0:
+        print(f"GDN commit sampled parity: {gdn['parity_sampled']['outside']} heads outside the bar",
+              file=sys.stderr, flush=True)
+        return 1
     if head is not None and head["parity_sampled"]["outside"] > 0:
         print(f"FP8 head sampled parity: {head['parity_sampled']['outside']} logits outside the tolerance",
               file=sys.stderr, flush=True)
         return 1
     return 0
+
+
+GDN_H, GDN_D, GDN_NODES = 48 * 32, 128, 32   # 48 GDN layers x 32 heads of 128 x 128 states; a 32-node tree
+GDN_L = (1, 4, 8, 16, 32)
+FP32_FMA_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # 148 SMs x 128 fp32 FMA lanes x 2 flops at 1,965 MHz
+
+
+def gdn_figure(tl, dev, stream, rank):
+    """Time tl_gdn_commit over 1,536 heads of 128 x 128 fp32 states for accepted paths of L = 1..32
+    tokens, CUDA events on the launching stream, with a 256 MB write between launches so the
+    100 MB of states come from HBM every time; then check 4 heads against the oracle."""
+    import numpy as np
+    import torch
+    import oracle
+    import synth
+    peak, _ = load_peaks()
+    S0, K, V, a, b = synth.gdn_inputs_torch(GDN_H, GDN_D, GDN_D, GDN_NODES, rank, dev)
+    state = S0.clone()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    per_L = {}
+    with torch.cuda.stream(stream):
+        for L in GDN_L:
+            path = list(range(L))
+            for _ in range(3):
+                tl.gdn_commit(state, K, V, a, b, path, stream=stream)
+            times = []
+            for _ in range(10):
+                flush.fill_(1)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                tl.gdn_commit(state, K, V, a, b, path, stream=stream)
+                e1.record(stream)
+                times.append((e0, e1))
+            stream.synchronize()
+            ms = statistics.median(e0.elapsed_time(e1) for e0, e1 in times)
+            byts = 2 * GDN_H * GDN_D * GDN_D * 4 + L * GDN_H * (2 * GDN_D + 2) * 4
+            flops = 4 * GDN_H * GDN_D * GDN_D * L + GDN_H * L * L * GDN_D
+            per_L[str(L)] = {"us": round(ms * 1e3, 1), "gbs": round(byts / (ms * 1e-3) / 1e9, 1),
+                             "frac_hbm": round(byts / (ms * 1e-3) / 1e9 / peak, 4),
+                             "tflops": round(flops / (ms * 1e-3) / 1e12, 2),
+                             "frac_fp32_fma": round(flops / (ms * 1e-3) / 1e12 / FP32_FMA_PEAK_TFLOPS, 4)}
+        # sampled parity: the longest path from the initial states, 4 heads
+        state.copy_(S0)
+        path = [0, 2, 3, 5, 8, 9, 13, 14, 17, 19, 20, 24, 26, 27, 30, 31]
+        tl.gdn_commit(state, K, V, a, b, path, stream=stream)
+        stream.synchronize()
+    tl.check_device_error(stream)
+    heads = [0, 511, 1024, GDN_H - 1]
+    outside = 0
+    S0h, Kh, Vh, ah, bh = (t.cpu().numpy() for t in (S0, K, V, a, b))
+    got = state.cpu().numpy().astype(np.float64)
+    for h in heads:
+        Kp, Vp, ap, bp = oracle.gdn_path_inputs(Kh[:, h], Vh[:, h], ah[:, h], bh[:, h], path)
+        ref = oracle.gdn_commit_closed_form(S0h[h], Kp, Vp, ap, bp)
+        outside += int(np.abs(got[h] - ref).max() > 1e-4 * max(1.0, float(np.abs(ref).max())))
+    return {"heads": GDN_H, "d_k": GDN_D, "d_v": GDN_D, "tree_nodes": GDN_NODES, "per_L": per_L,
+            "bytes": "2 * H * d_v * d_k * 4 (state in and out) + L * H * (d_k + d_v + 2) * 4 per commit",
+            "flops": "4 * H * d_v * d_k * L + H * L^2 * d_k", "fp32_fma_peak_tflops": round(FP32_FMA_PEAK_TFLOPS, 1),
+            "kernel": "gdn_commit_kernel<128, 128> (one launch)",
+            "parity_sampled": {"heads": len(heads), "outside": outside,
+                               "sample": "4 heads after a 16-token path, vs the fp64 oracle (bar 1e-4 of the state)"}}
 
 
 HEAD_N, HEAD_K = 151936, 5120     # a vocabulary-sized head on the stack's hidden size

@@ -300,6 +300,33 @@ typedef struct {
 tl_status tl_fp8_head(const void* x, int M, const void* w_fp8, int N, int K, float tensor_scale,
                       const float* row_scales, float* logits, tl_head_top2* top2, void* stream);
 
+/* Closed-form commit of an accepted draft path through Gated DeltaNet states (a next row).
+ *
+ * 48 of the served model's 64 layers carry a recurrent state that cannot step back after a wrong
+ * guess, so the engine commits the state of the accepted path in closed form (TandemLLM docs
+ * v0.12.0, "What TandemLLM is", section 1.7; the author's "Research" page, StairCut abstract).
+ * The pages print no equation; the rule taken is the gated delta rule, one token (key k, value v,
+ * gate a, step b) mapping a head's state S (d_v x d_k) to
+ *     S' = a S (I - b k k^T) + b v k^T,
+ * and the call replaces every head's S by its state after the L tokens of the path, in order, in
+ * one launch (a forward substitution over the path instead of L dependent updates).
+ *   state     device float [H][d_v][d_k], 16-byte aligned; read and overwritten in place
+ *   H         number of independent heads (layers x heads), >= 1
+ *   d_k, d_v  64 or 128 each
+ *   k         device float [n_nodes][H][d_k]: each draft-tree node's key per head
+ *   v         device float [n_nodes][H][d_v]
+ *   alpha     device float [n_nodes][H]: the gate a of each node and head
+ *   beta      device float [n_nodes][H]: the step b
+ *   path      HOST int [L]: the accepted nodes in path order, each in 0..n_nodes-1
+ *   L         0..TL_GDN_MAX_PATH (0 is a no-op)
+ * fp32 arithmetic on CUDA cores; no workspace, no allocation. Asynchronous on `stream`; the
+ * host path array is copied into the launch and may be reused at once. Errors: a size out of
+ * range, a node index outside 0..n_nodes-1, a null or misaligned pointer -> the status, nothing
+ * launched. */
+#define TL_GDN_MAX_PATH 32
+tl_status tl_gdn_commit(float* state, int H, int d_k, int d_v, const float* k, const float* v, const float* alpha,
+                        const float* beta, int n_nodes, const int* path, int L, void* stream);
+
 /* Synchronise `stream`, then report and clear the device status word:
  * TL_OK, TL_ERR_TIMEOUT (a bounded wait ran out) or TL_ERR_DEVICE_FAULT. Also reads and
  * clears the status word of tl_nvfp4_verify_gemm_noalloc()'s static scratch on the current

@@ -14,7 +14,7 @@ from ._lib import Matrix, TlError, check
 
 __all__ = ["verify_gemm", "verify_gemm_simt", "set_gemm_path", "get_gemm_path", "gemm_path", "PATH_BLOCK_SCALED",
            "PATH_BF16_EXACT", "PATH_EXACT", "verify_stack", "verify_stack_host", "Plan", "dequant",
-           "quantize", "check_device_error", "noalloc_check_error", "fp8_head", "init", "num_sms", "Matrix", "TlError"]
+           "quantize", "check_device_error", "noalloc_check_error", "fp8_head", "gdn_commit", "init", "num_sms", "Matrix", "TlError"]
 
 
 def _stream(stream):
@@ -197,3 +197,18 @@ def head_top2_fields(top2):
     t = top2.cpu().numpy()
     return (t[:, 0].astype(np.int64), t[:, 1].view(np.float32).astype(np.float64),
             t[:, 2].view(np.float32).astype(np.float64), t[:, 3].view(np.float32).astype(np.float64))
+
+
+def gdn_commit(state, k, v, alpha, beta, path, stream=None):
+    """Closed-form commit of an accepted draft path through Gated DeltaNet states, in place.
+
+    state float32 [H, d_v, d_k] (device); k float32 [n_nodes, H, d_k]; v float32 [n_nodes, H, d_v];
+    alpha, beta float32 [n_nodes, H]; path: the accepted node indices in order (a host sequence
+    of at most 32 ints). Returns `state`."""
+    H, d_v, d_k = state.shape
+    n_nodes = k.shape[0]
+    p = [int(t) for t in path]
+    arr = (ctypes.c_int * max(1, len(p)))(*p)
+    check(_lib.lib().tl_gdn_commit(_ptr(state), H, d_k, d_v, _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), n_nodes, arr,
+                                   len(p), _stream(stream)))
+    return state

@@ -27,6 +27,7 @@ EXPORTS = (
     "tl_nvfp4_plan_run", "tl_nvfp4_plan_run_host", "tl_nvfp4_plan_destroy", "tl_nvfp4_dequant",
     "tl_nvfp4_quantize", "tl_check_device_error", "tl_selftest_bounded_wait", "tl_num_sms", "tl_status_string",
     "tl_last_error_message", "tl_set_gemm_path", "tl_get_gemm_path", "tl_noalloc_check_error", "tl_fp8_head",
+    "tl_gdn_commit",
 )
 
 # Tensor-core paths (tl_set_gemm_path).
@@ -82,6 +83,7 @@ def lib() -> ctypes.CDLL:
             "tl_check_device_error": [vp],
             "tl_noalloc_check_error": [vp],
             "tl_fp8_head": [vp, i, vp, i, i, f, vp, vp, vp, vp],
+            "tl_gdn_commit": [vp, i, i, i, vp, vp, vp, vp, i, ctypes.POINTER(i), i, vp],
             "tl_selftest_bounded_wait": [ctypes.c_uint, vp],
             "tl_num_sms": [i],
             "tl_status_string": [i],

@@ -22,6 +22,7 @@
 #include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
 #include "gemm_ex.cuh"
+#include "gdn_commit.cuh"
 #include "gemm_head.cuh"
 #include "xprep.cuh"
 #include "gemm_bs.cuh"
@@ -1197,6 +1198,18 @@ tl_status launch_head(DevState& d, tl::HeadParams& hp, cudaStream_t stream) {
     return TL_OK;
 }
 
+template <int DK, int DV>
+tl_status launch_gdn(float* state, int H, const float* k, const float* v, const float* alpha, const float* beta,
+                     const tl::GdnPath& p, int L, cudaStream_t stream) {
+    using C = tl::GdnCfg<DK, DV>;
+    TL_CUDA(cudaFuncSetAttribute(tl::gdn_commit_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::SMEM_BYTES));
+    tl::gdn_commit_kernel<DK, DV><<<(unsigned)H, tl::GDN_THREADS, C::SMEM_BYTES, stream>>>(state, H, k, v, alpha, beta,
+                                                                                          p, L);
+    TL_CUDA(cudaGetLastError());
+    return TL_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -1494,6 +1507,35 @@ tl_status tl_fp8_head(const void* x, int M, const void* w_fp8, int N, int K, flo
     tl::head_top2_final_kernel<<<(unsigned)M, 32, 0, s>>>(part, chunks, reinterpret_cast<tl::HeadTop2*>(top2));
     TL_CUDA(cudaGetLastError());
     return TL_OK;
+}
+
+tl_status tl_gdn_commit(float* state, int H, int d_k, int d_v, const float* k, const float* v, const float* alpha,
+                        const float* beta, int n_nodes, const int* path, int L, void* stream) {
+    if (H < 1) return fail(TL_ERR_INVALID_VALUE, "H = %d must be >= 1", H);
+    if ((d_k != 64 && d_k != 128) || (d_v != 64 && d_v != 128))
+        return fail(TL_ERR_UNSUPPORTED, "d_k = %d, d_v = %d: each must be 64 or 128", d_k, d_v);
+    if (L < 0 || L > TL_GDN_MAX_PATH) return fail(TL_ERR_INVALID_VALUE, "L = %d outside 0..%d", L, TL_GDN_MAX_PATH);
+    if (n_nodes < 1) return fail(TL_ERR_INVALID_VALUE, "n_nodes = %d must be >= 1", n_nodes);
+    if (!state || !k || !v || !alpha || !beta || (L > 0 && !path)) return fail(TL_ERR_INVALID_VALUE, "null pointer");
+    if (!aligned16(state)) return fail(TL_ERR_MISALIGNED, "state must be 16-byte aligned");
+    tl::GdnPath p;
+    memset(&p, 0, sizeof p);
+    for (int t = 0; t < L; ++t) {
+        if (path[t] < 0 || path[t] >= n_nodes)
+            return fail(TL_ERR_INVALID_VALUE, "path[%d] = %d outside 0..%d", t, path[t], n_nodes - 1);
+        p.idx[t] = path[t];
+    }
+    if (L == 0) return TL_OK;
+    DevState* d = nullptr;
+    tl_status st = current_state(&d);
+    if (st != TL_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (d_k == 128 && d_v == 128) st = launch_gdn<128, 128>(state, H, k, v, alpha, beta, p, L, s);
+    else if (d_k == 128) st = launch_gdn<128, 64>(state, H, k, v, alpha, beta, p, L, s);
+    else if (d_v == 128) st = launch_gdn<64, 128>(state, H, k, v, alpha, beta, p, L, s);
+    else st = launch_gdn<64, 64>(state, H, k, v, alpha, beta, p, L, s);
+    (void)d;
+    return st;
 }
 
 tl_status tl_nvfp4_dequant(const void* w_codes, const void* w_scales, float global_scale, float* w_out, int N, int K,

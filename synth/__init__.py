@@ -118,3 +118,33 @@ def w_f32_torch(N: int, K: int, seed: int, tensor_id: int, device, dist: str = "
             del e
         return z.div_(v.mul_(0.25).sqrt_()).mul_(std)
     raise ValueError(f"unknown weight distribution {dist!r}")
+
+
+# ---------------------------------------------------------------------------
+# Gated DeltaNet commit inputs: per-head states and per-node key/value/gate/step of a draft tree.
+
+def gdn_inputs(H: int, d_k: int, d_v: int, n_nodes: int, seed: int = 0):
+    """(S0 [H, d_v, d_k], K [n_nodes, H, d_k], V [n_nodes, H, d_v], alpha [n_nodes, H], beta [n_nodes, H]),
+    all float32: S0 ~ N(0, 0.1); keys N(0, 1) scaled to unit length (as the layer normalises them);
+    V ~ N(0, 1); gates alpha ~ U(0.9, 1); steps beta ~ U(0, 1)."""
+    g = _rng(seed, 2_000_000 + H)
+    S0 = (g.standard_normal((H, d_v, d_k), dtype=np.float32) * np.float32(0.1)).astype(np.float32)
+    K = g.standard_normal((n_nodes, H, d_k), dtype=np.float32)
+    K = (K / np.linalg.norm(K, axis=2, keepdims=True)).astype(np.float32)
+    V = g.standard_normal((n_nodes, H, d_v), dtype=np.float32)
+    alpha = g.uniform(0.9, 1.0, (n_nodes, H)).astype(np.float32)
+    beta = g.uniform(0.0, 1.0, (n_nodes, H)).astype(np.float32)
+    return S0, K, V, alpha, beta
+
+
+def gdn_inputs_torch(H: int, d_k: int, d_v: int, n_nodes: int, seed: int, device):
+    """The same recipe drawn on `device` with torch (for the bench's 1,536 heads)."""
+    import torch
+    gen = _torch_gen(seed, 2_000_000 + H, device)
+    S0 = torch.randn((H, d_v, d_k), generator=gen, device=device) * 0.1
+    K = torch.randn((n_nodes, H, d_k), generator=gen, device=device)
+    K = K / K.norm(dim=2, keepdim=True)
+    V = torch.randn((n_nodes, H, d_v), generator=gen, device=device)
+    alpha = torch.rand((n_nodes, H), generator=gen, device=device) * 0.1 + 0.9
+    beta = torch.rand((n_nodes, H), generator=gen, device=device)
+    return S0, K.contiguous(), V, alpha, beta

@@ -83,3 +83,16 @@ def test_dequant_and_quantize_validate(L):
     g = ctypes.c_float()
     assert L.tl_nvfp4_quantize(A, 0, 256, A, A, ctypes.byref(g), None) == 1
     assert L.tl_nvfp4_quantize(A, 4, 24, A, A, ctypes.byref(g), None) == 1
+
+
+def test_gdn_commit_validates(L):
+    path = (ctypes.c_int * 4)(0, 1, 2, 3)
+    def call(H=4, dk=128, dv=128, state=A, n_nodes=8, p=path, n=4):
+        return L.tl_gdn_commit(state, H, dk, dv, A, A, A, A, n_nodes, p, n, None)
+    assert call(H=0) == 1
+    assert call(dk=96) == 3 and call(dv=32) == 3
+    assert call(n=33) == 1 and call(n=-1) == 1
+    assert call(n_nodes=3) == 1                 # node index 3 is outside 0..2
+    assert call(state=A + 4) == 2
+    assert call(state=0) == 1
+    assert call(n=0) == 0                       # an empty path is a no-op and never reaches CUDA
