@@ -313,7 +313,7 @@ tl_status tl_fp8_head(const void* x, int M, const void* w_fp8, int N, int K, flo
  *   state     device float [H][d_v][d_k], 16-byte aligned; read and overwritten in place
  *   H         number of independent heads (layers x heads), >= 1
  *   d_k, d_v  64 or 128 each
- *   k         device float [n_nodes][H][d_k]: each draft-tree node's key per head
+ *   k         device float [n_nodes][H][d_k], 16-byte aligned: each draft-tree node's key per head
  *   v         device float [n_nodes][H][d_v]
  *   alpha     device float [n_nodes][H]: the gate a of each node and head
  *   beta      device float [n_nodes][H]: the step b

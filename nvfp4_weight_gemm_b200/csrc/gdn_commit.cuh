@@ -16,8 +16,8 @@
 //
 // so one launch computes P = S_0 K^T, solves the unit lower-triangular system for U by forward
 // substitution (one thread per state row), and writes S_L = g_L S_0 + U' K, all in fp32 on CUDA
-// cores. One CTA per head; S_0 is read once from HBM into shared memory and S_L written back in
-// place, coalesced. Bound: HBM for the state (2 * DV * DK * 4 bytes per head) against the fp32
+// cores. One CTA per head (about 106 KB of shared memory at d_k = d_v = 128, two per SM); S_0 is
+// read once from HBM into shared memory and S_L written back in place, coalesced. Bound: HBM for the state (2 * DV * DK * 4 bytes per head) against the fp32
 // FMA pipe for the 2 * DV * DK * L multiply-adds per head.
 #pragma once
 #include <cstdint>
@@ -34,18 +34,21 @@ struct GdnPath {
 
 template <int DK, int DV>
 struct GdnCfg {
-    static constexpr int SP = DK + 1;                    // padded row of S in shared memory
+    static constexpr int SP = DK + 4;                    // padded row (16-byte steps, conflict-free float4)
     static constexpr int G = GDN_THREADS / DV;           // thread groups over the rows of S
+    static constexpr int PL = GDN_MAX_L + 1;
     static constexpr int SMEM_FLOATS = DV * SP           // S_0, then S_L
-                                     + GDN_MAX_L * DK    // keys of the path
-                                     + DV * (GDN_MAX_L + 1)   // P, then U'
-                                     + GDN_MAX_L * (GDN_MAX_L + 1)   // A
+                                     + GDN_MAX_L * SP    // keys of the path
+                                     + DV * PL           // R, then U
+                                     + GDN_MAX_L * PL    // A
                                      + 4 * GDN_MAX_L;    // g, decay, beta, alpha
     static constexpr int SMEM_BYTES = SMEM_FLOATS * 4;
     static_assert(GDN_THREADS % DV == 0 && DK % (4 * G) == 0, "thread layout");
 };
 
-template <int DK, int DV>
+// One CTA per head; LMAX (8, 16 or 32) bounds the path length, so the substitution's unrolled
+// loops run no further than needed.
+template <int DK, int DV, int LMAX>
 __global__ void __launch_bounds__(GDN_THREADS) gdn_commit_kernel(float* __restrict__ state, int H,
                                                                  const float* __restrict__ k,
                                                                  const float* __restrict__ v,
@@ -53,31 +56,38 @@ __global__ void __launch_bounds__(GDN_THREADS) gdn_commit_kernel(float* __restri
                                                                  const float* __restrict__ beta,
                                                                  const GdnPath path, int L) {
     using C = GdnCfg<DK, DV>;
+    constexpr int SP = C::SP, PL = C::PL;
     extern __shared__ float sm[];
     float* Ss = sm;                                  // [DV][SP]
-    float* Ks = Ss + DV * C::SP;                     // [L][DK]
-    float* Ps = Ks + GDN_MAX_L * DK;                 // [DV][L + 1]: P, then U'
-    float* As = Ps + DV * (GDN_MAX_L + 1);           // [L][L + 1]
-    float* gs = As + GDN_MAX_L * (GDN_MAX_L + 1);    // g_t
+    float* Ks = Ss + DV * SP;                        // [L][SP]
+    float* Rs = Ks + GDN_MAX_L * SP;                 // [DV][PL]: R, then U (in place)
+    float* As = Rs + DV * PL;                        // [L][PL]
+    float* gs = As + GDN_MAX_L * PL;                 // g_t
     float* ds = gs + GDN_MAX_L;                      // a_{t+1} ... a_L
     float* bs = ds + GDN_MAX_L;                      // beta_t
     float* as = bs + GDN_MAX_L;                      // alpha_t
-    constexpr int PL = GDN_MAX_L + 1;
 
     const int h = blockIdx.x;
     const int tid = threadIdx.x;
     float* S = state + (size_t)h * DV * DK;
 
-    // S_0 into shared memory (coalesced), the path's keys, gates and steps
-    for (int e = tid; e < DV * DK / 4; e += GDN_THREADS) {
-        const float4 q = reinterpret_cast<const float4*>(S)[e];
-        const int i = (4 * e) / DK, j = (4 * e) % DK;
-        float* row = Ss + i * C::SP + j;
-        row[0] = q.x; row[1] = q.y; row[2] = q.z; row[3] = q.w;
+    // S_0 into shared memory (coalesced; a thread's loads all in flight at once), the path's keys,
+    // gates and steps
+    constexpr int NQ = DV * DK / 4 / GDN_THREADS;
+    {
+        float4 q[NQ];
+#pragma unroll
+        for (int u = 0; u < NQ; ++u) q[u] = __ldcs(reinterpret_cast<const float4*>(S) + tid + u * GDN_THREADS);
+#pragma unroll
+        for (int u = 0; u < NQ; ++u) {
+            const int e = tid + u * GDN_THREADS;
+            *reinterpret_cast<float4*>(Ss + ((4 * e) / DK) * SP + (4 * e) % DK) = q[u];
+        }
     }
-    for (int e = tid; e < L * DK; e += GDN_THREADS) {
-        const int t = e / DK, j = e % DK;
-        Ks[t * DK + j] = k[((size_t)path.idx[t] * H + h) * DK + j];
+    for (int e = tid; e < L * DK / 4; e += GDN_THREADS) {
+        const int t = (4 * e) / DK, j = (4 * e) % DK;
+        *reinterpret_cast<float4*>(Ks + t * SP + j) =
+            __ldg(reinterpret_cast<const float4*>(k + ((size_t)path.idx[t] * H + h) * DK + j));
     }
     if (tid < L) {
         as[tid] = alpha[(size_t)path.idx[tid] * H + h];
@@ -95,68 +105,92 @@ __global__ void __launch_bounds__(GDN_THREADS) gdn_commit_kernel(float* __restri
         const int t = p / L, s = p % L;
         if (s >= t) continue;
         float dot = 0.0f;
-#pragma unroll 8
-        for (int j = 0; j < DK; ++j) dot = fmaf(Ks[s * DK + j], Ks[t * DK + j], dot);
+#pragma unroll 4
+        for (int j = 0; j < DK; j += 4) {
+            const float4 x = *reinterpret_cast<const float4*>(Ks + s * SP + j);
+            const float4 y = *reinterpret_cast<const float4*>(Ks + t * SP + j);
+            dot = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, fmaf(x.w, y.w, dot))));
+        }
         float decay = 1.0f;
         for (int r = s + 1; r <= t; ++r) decay *= as[r];
         As[t * PL + s] = bs[t] * decay * dot;
     }
-    // P = S_0 K^T: thread (row i, group gi) takes t = gi, gi + G, ...
+    __syncthreads();
+    // R = B (V^T - S_0 K^T G): thread (row i, group gi) takes t = gi, gi + G, ..., four at a time;
+    // the values are loaded before the dot products so their latency overlaps them
     const int i = tid % DV, gi = tid / DV;
     {
-        float acc[GDN_MAX_L / C::G];
+        const float* srow = Ss + i * SP;
+        for (int t0 = gi; t0 < L; t0 += 4 * C::G) {
+            float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f}, vv[4];
 #pragma unroll
-        for (int u = 0; u < GDN_MAX_L / C::G; ++u) acc[u] = 0.0f;
-        const float* srow = Ss + i * C::SP;
-        for (int j = 0; j < DK; j += 4) {
-            const float s0 = srow[j], s1 = srow[j + 1], s2 = srow[j + 2], s3 = srow[j + 3];
+            for (int u = 0; u < 4; ++u) {
+                const int t = t0 + C::G * u;
+                vv[u] = (t < L) ? __ldg(v + ((size_t)path.idx[t] * H + h) * DV + i) : 0.0f;
+            }
+#pragma unroll 4
+            for (int j = 0; j < DK; j += 4) {
+                const float4 sv = *reinterpret_cast<const float4*>(srow + j);
 #pragma unroll
-            for (int u = 0; u < GDN_MAX_L / C::G; ++u) {
-                const int t = gi + C::G * u;
-                if (t < L) {
-                    const float4 kk = *reinterpret_cast<const float4*>(Ks + t * DK + j);
-                    acc[u] = fmaf(s0, kk.x, fmaf(s1, kk.y, fmaf(s2, kk.z, fmaf(s3, kk.w, acc[u]))));
+                for (int u = 0; u < 4; ++u) {
+                    const int t = t0 + C::G * u;
+                    if (t < L) {
+                        const float4 kk = *reinterpret_cast<const float4*>(Ks + t * SP + j);
+                        acc[u] = fmaf(sv.x, kk.x, fmaf(sv.y, kk.y, fmaf(sv.z, kk.z, fmaf(sv.w, kk.w, acc[u]))));
+                    }
                 }
             }
-        }
 #pragma unroll
-        for (int u = 0; u < GDN_MAX_L / C::G; ++u) {
-            const int t = gi + C::G * u;
-            if (t < L) Ps[i * PL + t] = acc[u];
+            for (int u = 0; u < 4; ++u) {
+                const int t = t0 + C::G * u;
+                if (t < L) Rs[i * PL + t] = bs[t] * (vv[u] - gs[t] * acc[u]);
+            }
         }
     }
     __syncthreads();
-    // forward substitution, one thread per row of S: u_t = r_t - sum_{s<t} A[t][s] u_s, with
-    // r_t = b_t (v_t[i] - g_t P[i][t]); then U'[i][t] = (a_{t+1} ... a_L) u_t
+    // forward substitution, one thread per row, in registers: u_t = r_t - sum_{s<t} A[t][s] u_s
+    // (the sum in four interleaved partial sums, added in a fixed order, to shorten the chain)
     if (tid < DV) {
-        float u[GDN_MAX_L];
+        float* row = Rs + i * PL;
+        float u[LMAX];
 #pragma unroll
-        for (int t = 0; t < GDN_MAX_L; ++t) {
+        for (int t = 0; t < LMAX; ++t) u[t] = (t < L) ? row[t] : 0.0f;
+#pragma unroll
+        for (int t = 1; t < LMAX; ++t) {
             if (t < L) {
-                const float vt = v[((size_t)path.idx[t] * H + h) * DV + i];
-                float r = bs[t] * (vt - gs[t] * Ps[i * PL + t]);
+                float p0 = 0.0f, p1 = 0.0f, p2 = 0.0f, p3 = 0.0f;
 #pragma unroll
-                for (int s = 0; s < t; ++s) r = fmaf(-As[t * PL + s], u[s], r);
-                u[t] = r;
+                for (int s = 0; s < t; ++s) {
+                    const float term = As[t * PL + s] * u[s];
+                    if ((s & 3) == 0) p0 += term;
+                    else if ((s & 3) == 1) p1 += term;
+                    else if ((s & 3) == 2) p2 += term;
+                    else p3 += term;
+                }
+                u[t] -= (p0 + p1) + (p2 + p3);
             }
         }
 #pragma unroll
-        for (int t = 0; t < GDN_MAX_L; ++t)
-            if (t < L) Ps[i * PL + t] = ds[t] * u[t];
+        for (int t = 0; t < LMAX; ++t)
+            if (t < L) row[t] = u[t];
     }
     __syncthreads();
-    // S_L = g_L S_0 + U' K: thread (row i, group gi) takes columns [gi * DK / G, (gi + 1) * DK / G)
+    // S_L = g_L S_0 + sum_t (a_{t+1} ... a_L) u_t k_t^T: thread (row i, group gi) takes columns
+    // [gi * DK / G, (gi + 1) * DK / G)
     {
         constexpr int NC = DK / C::G;
         const int j0 = gi * NC;
         float acc[NC];
         const float gL = (L > 0) ? gs[L - 1] : 1.0f;
-        float* srow = Ss + i * C::SP + j0;
+        float* srow = Ss + i * SP + j0;
 #pragma unroll
-        for (int c = 0; c < NC; ++c) acc[c] = gL * srow[c];
+        for (int c = 0; c < NC; c += 4) {
+            const float4 sv = *reinterpret_cast<const float4*>(srow + c);
+            acc[c] = gL * sv.x; acc[c + 1] = gL * sv.y; acc[c + 2] = gL * sv.z; acc[c + 3] = gL * sv.w;
+        }
         for (int t = 0; t < L; ++t) {
-            const float ut = Ps[i * PL + t];
-            const float* kr = Ks + t * DK + j0;
+            const float ut = ds[t] * Rs[i * PL + t];
+            const float* kr = Ks + t * SP + j0;
 #pragma unroll
             for (int c = 0; c < NC; c += 4) {
                 const float4 kk = *reinterpret_cast<const float4*>(kr + c);
@@ -166,15 +200,17 @@ __global__ void __launch_bounds__(GDN_THREADS) gdn_commit_kernel(float* __restri
                 acc[c + 3] = fmaf(ut, kk.w, acc[c + 3]);
             }
         }
-        __syncthreads();   // every thread has read its S_0 elements before any is overwritten
+        // each thread rewrites only the elements it read
 #pragma unroll
-        for (int c = 0; c < NC; ++c) srow[c] = acc[c];
+        for (int c = 0; c < NC; c += 4)
+            *reinterpret_cast<float4*>(srow + c) = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
     }
     __syncthreads();
-    for (int e = tid; e < DV * DK / 4; e += GDN_THREADS) {
-        const int r = (4 * e) / DK, j = (4 * e) % DK;
-        const float* row = Ss + r * C::SP + j;
-        reinterpret_cast<float4*>(S)[e] = make_float4(row[0], row[1], row[2], row[3]);
+#pragma unroll
+    for (int u = 0; u < NQ; ++u) {
+        const int e = tid + u * GDN_THREADS;
+        __stcs(reinterpret_cast<float4*>(S) + e,
+               *reinterpret_cast<const float4*>(Ss + ((4 * e) / DK) * SP + (4 * e) % DK));
     }
 }
 

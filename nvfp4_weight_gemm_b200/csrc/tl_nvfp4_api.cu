@@ -1198,16 +1198,24 @@ tl_status launch_head(DevState& d, tl::HeadParams& hp, cudaStream_t stream) {
     return TL_OK;
 }
 
+template <int DK, int DV, int LMAX>
+tl_status launch_gdn_l(float* state, int H, const float* k, const float* v, const float* alpha, const float* beta,
+                       const tl::GdnPath& p, int L, cudaStream_t stream) {
+    using C = tl::GdnCfg<DK, DV>;
+    TL_CUDA(cudaFuncSetAttribute(tl::gdn_commit_kernel<DK, DV, LMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::SMEM_BYTES));
+    tl::gdn_commit_kernel<DK, DV, LMAX><<<(unsigned)H, tl::GDN_THREADS, C::SMEM_BYTES, stream>>>(state, H, k, v, alpha,
+                                                                                                beta, p, L);
+    TL_CUDA(cudaGetLastError());
+    return TL_OK;
+}
+
 template <int DK, int DV>
 tl_status launch_gdn(float* state, int H, const float* k, const float* v, const float* alpha, const float* beta,
                      const tl::GdnPath& p, int L, cudaStream_t stream) {
-    using C = tl::GdnCfg<DK, DV>;
-    TL_CUDA(cudaFuncSetAttribute(tl::gdn_commit_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 C::SMEM_BYTES));
-    tl::gdn_commit_kernel<DK, DV><<<(unsigned)H, tl::GDN_THREADS, C::SMEM_BYTES, stream>>>(state, H, k, v, alpha, beta,
-                                                                                          p, L);
-    TL_CUDA(cudaGetLastError());
-    return TL_OK;
+    if (L <= 8) return launch_gdn_l<DK, DV, 8>(state, H, k, v, alpha, beta, p, L, stream);
+    if (L <= 16) return launch_gdn_l<DK, DV, 16>(state, H, k, v, alpha, beta, p, L, stream);
+    return launch_gdn_l<DK, DV, 32>(state, H, k, v, alpha, beta, p, L, stream);
 }
 
 }  // namespace
@@ -1517,7 +1525,7 @@ tl_status tl_gdn_commit(float* state, int H, int d_k, int d_v, const float* k, c
     if (L < 0 || L > TL_GDN_MAX_PATH) return fail(TL_ERR_INVALID_VALUE, "L = %d outside 0..%d", L, TL_GDN_MAX_PATH);
     if (n_nodes < 1) return fail(TL_ERR_INVALID_VALUE, "n_nodes = %d must be >= 1", n_nodes);
     if (!state || !k || !v || !alpha || !beta || (L > 0 && !path)) return fail(TL_ERR_INVALID_VALUE, "null pointer");
-    if (!aligned16(state)) return fail(TL_ERR_MISALIGNED, "state must be 16-byte aligned");
+    if (!aligned16(state) || !aligned16(k)) return fail(TL_ERR_MISALIGNED, "state and k must be 16-byte aligned");
     tl::GdnPath p;
     memset(&p, 0, sizeof p);
     for (int t = 0; t < L; ++t) {

@@ -94,5 +94,6 @@ def test_gdn_commit_validates(L):
     assert call(n=33) == 1 and call(n=-1) == 1
     assert call(n_nodes=3) == 1                 # node index 3 is outside 0..2
     assert call(state=A + 4) == 2
+    assert L.tl_gdn_commit(A, 4, 128, 128, A + 4, A, A, A, 8, path, 4, None) == 2   # misaligned keys
     assert call(state=0) == 1
     assert call(n=0) == 0                       # an empty path is a no-op and never reaches CUDA
