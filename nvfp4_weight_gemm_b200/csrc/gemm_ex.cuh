@@ -16,7 +16,7 @@
 //
 // Roles (one CTA per SM):
 //   * warp 0        weight producer: TMA copies of codes and scales into a ring of stages.
-//   * warp 16       X producer: one TMA copy of the X tile of each k-tile into the tile's slot.
+//   * warp 3        X producer: one TMA copy of the X tile of each k-tile into the tile's slot.
 //   * warps 4..11   dequantisers, two tile sets of four lane quarters; set t takes the tiles
 //                   with parity t. The warp of quarter q decodes weight rows 32q..32q+31 over the
 //                   whole 256 k of a tile: it loads its row's 128 code bytes and 16 scales from
@@ -24,9 +24,11 @@
 //                   the stage straight back (so nearly the whole ring is in flight from HBM); it
 //                   decodes the first 64-k chunk before waiting for the tile's slot, then writes
 //                   four chunks of 32 tensor-memory columns.
-//   * issuers       warps 1..3 and 17: issuer j issues k-steps 4j..4j+3 of every tile (half
-//                   j / 2) into its own accumulator; a thread keeps only about one MMA in flight
-//                   per ~80 cycles, so a tile's 16 MMAs are spread over four warps.
+//   * issuers       warps 1 and 2: issuer j issues k-steps 8j..8j+7 of every tile into its own
+//                   accumulator. Sixteen warps in all, so no SM sub-partition holds more than four
+//                   and every thread may use 128 registers (eighteen warps capped them at 96, with
+//                   spills at NX = 32); in paired timings this layout was 5% (M <= 16) to 8%
+//                   (M >= 17) faster than four issuer warps, and eight issuers were 23% slower.
 //   * warps 12..15  epilogue: add the issuers' accumulators in fixed order, write Y or a partial.
 //
 // Every mbarrier wait is bounded; a wait that runs out records TL_ERR_TIMEOUT in the device
@@ -43,11 +45,11 @@ namespace tl {
 
 template <int NX>
 struct ExCfg {
-    static constexpr int NISSUE = 4;
+    static constexpr int NISSUE = 2;
     static constexpr int KSTEPS = 16 / NISSUE;            // 16-k MMA steps per issuer per tile
-    static constexpr int WARPS = 14 + NISSUE;
+    static constexpr int WARPS = 16;                       // producer, 2 issuers, X producer, 8 + 4
     static constexpr int THREADS = 32 * WARPS;
-    static constexpr int DQ_FIRST = 4, DQ_WARPS = 8, EPI_FIRST = 12, XWARP = 16;
+    static constexpr int DQ_FIRST = 4, DQ_WARPS = 8, EPI_FIRST = 12, XWARP = 3;
     static constexpr int CODES_BYTES = TC_BLOCK_N * (TC_BLOCK_K / 2);   // 16384
     static constexpr int SCALES_BYTES = TC_BLOCK_N * (TC_BLOCK_K / 16); // 2048
     static constexpr int W_STAGE_BYTES = CODES_BYTES + SCALES_BYTES;   // 18432
@@ -60,18 +62,18 @@ struct ExCfg {
     static constexpr uint32_t IDESC = idesc_f16(0u /*f16*/, 128u, (uint32_t)NX);
     static constexpr int ACC_COL0 = 128 * NUM_A;                       // three A buffers, then the accumulators
     // accumulator buffers: two where tensor memory holds them (the next segment's MMAs then do not
-    // wait for the epilogue), one at NX = 32
+    // wait for the epilogue); with two issuers that is both NX = 16 and NX = 32
     static constexpr int ACC_BUF_COLS = NISSUE * NX;
     static constexpr int ACC_BUFS = (ACC_COL0 + 2 * ACC_BUF_COLS <= 512) ? 2 : 1;
     static constexpr int TMEM_COLS = 512;
     static_assert(ACC_COL0 + ACC_BUFS * ACC_BUF_COLS <= TMEM_COLS, "tensor memory budget");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-    static_assert((WARPS - 1) % 4 != 0 || true, "");
+    static_assert(WARPS * 32 <= 512, "16 warps: at most four per SM sub-partition, 128 registers a thread");
 };
 
 template <int NX>
 __host__ __device__ constexpr int ex_issuer_of_warp(int w) {
-    return (w >= 1 && w <= 3) ? w - 1 : (w >= 17 && w < 14 + ExCfg<NX>::NISSUE) ? w - 14 : -1;
+    return (w >= 1 && w <= 2) ? w - 1 : -1;
 }
 
 __device__ __forceinline__ uint32_t ex_hmul2_f16(uint32_t a, uint32_t b) {

@@ -17,7 +17,7 @@
 // (head_top2_part_kernel over chunks of the row, head_top2_final_kernel over the chunks).
 //
 // Tile: 128 weight rows x 256 k (32 KiB of E4M3 bytes, two 128-byte swizzled slices per row);
-// roles and stream-K split as in gemm_ex.cuh (weight producer, X producer, 4 MMA issuers,
+// roles and stream-K split as in gemm_ex.cuh (weight producer, X producer, 2 MMA issuers,
 // 8 dequantisers in two tile sets of four lane quarters, 4 epilogue warps).
 #pragma once
 #include <cstdint>
@@ -49,9 +49,10 @@ struct alignas(64) HeadParams {
 
 template <int NX>
 struct HeadCfg {
-    static constexpr int NISSUE = 4;
-    static constexpr int THREADS = 32 * 18;
-    static constexpr int DQ_FIRST = 4, EPI_FIRST = 12, XWARP = 16, ISSUER3 = 17;
+    static constexpr int NISSUE = 2;                       // k-steps 8j .. 8j + 7 for issuer j
+    static constexpr int KSTEPS = 16 / NISSUE;
+    static constexpr int THREADS = 32 * 16;                // 16 warps: 128 registers a thread
+    static constexpr int DQ_FIRST = 4, EPI_FIRST = 12, XWARP = 3;
     static constexpr int W_STAGE_BYTES = TC_BLOCK_N * TC_BLOCK_K;          // 32768
     static constexpr int X_SUB = NX * 128;
     static constexpr int X_BYTES = 4 * X_SUB;
@@ -68,7 +69,7 @@ struct HeadCfg {
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-__host__ __device__ constexpr int head_issuer_of_warp(int w) { return (w >= 1 && w <= 3) ? w - 1 : (w == 17 ? 3 : -1); }
+__host__ __device__ constexpr int head_issuer_of_warp(int w) { return (w == 1 || w == 2) ? w - 1 : -1; }
 
 // Sixteen E4M3 bytes (k order) -> eight f16x2 words (low byte in the low half), exact.
 __device__ __forceinline__ void head_decode16(uint4 q, uint32_t* out) {
@@ -211,7 +212,7 @@ __global__ void __launch_bounds__(HeadCfg<NX>::THREADS, 1) gemm_head_kernel(cons
         // ------------------------------------------------------------ MMA issuers (k-steps 4j .. 4j + 3)
         // warp-uniform operands (lane-0 shuffles), as in gemm_ex_kernel
         const int j = __shfl_sync(0xFFFFFFFFu, head_issuer_of_warp(warp), 0);
-        const int i0 = 4 * j;
+        const int i0 = C::KSTEPS * j;
         const bool leader = elect_one();
         int a = 0, acc = 0;
         uint32_t aph = 0, accph = 0;
@@ -241,7 +242,7 @@ __global__ void __launch_bounds__(HeadCfg<NX>::THREADS, 1) gemm_head_kernel(cons
                 const uint32_t a_tmem = tmem_u + (uint32_t)(128 * a + 8 * i0);
                 if (leader) {
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
+                    for (int u = 0; u < C::KSTEPS; ++u) {
                         const int i = i0 + u;
                         mma_ts_f16(d_tmem, a_tmem + 8u * u, bdesc0 + (uint64_t)((((i >> 2) * C::X_SUB + (i & 3) * 32)) >> 4),
                                    C::IDESC, (u == 0) ? (first ^ 1u) : 1u);
