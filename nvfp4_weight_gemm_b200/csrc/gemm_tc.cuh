@@ -1,4 +1,8 @@
-// gemm_tc.cuh -- tensor-core NVFP4 verify GEMM for sm_100a (tcgen05 + TMA + tensor memory).
+// gemm_tc.cuh -- the exact bf16 tensor-core NVFP4 verify GEMM for sm_100a (TL_PATH_BF16_EXACT and
+// the no-allocation entry point), and the structures every tensor-core path shares: the matrix
+// descriptor (TcMat), the launch parameters (TcParams), the stream-K work list (TcSegIter,
+// tc_range_start) and the bounded mbarrier wait (tc_wait). The default exact f16 path's GEMM
+// is gemm_ex.cuh.
 //
 // Y[M,N] = X[M,K] . dequant(W)[N,K]^T for M <= 32 draft-tree rows (TandemLLM docs v0.12.0,
 // "What TandemLLM is", section 1.2: one verify pass over all tree rows streams every 4-bit
@@ -11,7 +15,7 @@
 //     whose share starts or ends inside an n-tile writes an fp32 partial; the last of an
 //     n-tile's contributors (an atomic counter, no waiting) adds the partials in k order,
 //     so every output has one fixed reduction order.
-//   * Roles, 25 warps. Warp 0 streams codes and scales (TMA) into a ring of weight stages;
+//   * Roles, 26 warps. Warp 0 streams codes and scales (TMA) into a ring of weight stages;
 //     a stage is handed back as soon as the dequantisers hold its bytes in registers, so
 //     nearly the whole ring is in flight from HBM. Warp 24 loads the X tile of each k-tile
 //     into a separate, shorter ring (an L2 hit) that the MMAs release. Warps 4..19
@@ -23,7 +27,7 @@
 //     The dequantisers form two sets of eight warps that take alternate tiles, so four
 //     dequant warps share each scheduler and one set's waits overlap the other's decode. A single thread keeps
 //     only about one tcgen05.mma in flight per ~90 cycles at these small N, so warps 1..3
-//     each issue a third of every tile's 16 k-steps into their own accumulator.
+//     and 25 each issue a quarter of every tile's 16 k-steps into their own accumulator.
 //     Warps 20..23 read the accumulators and write Y (or a partial).
 //   * Dequantisation without a table. For code c = s e1 e0 m, the bf16 bit pattern
 //     (e1 e0 m) << 6 | s << 15 is exactly e2m1(c) * 2^-126 (code 1 lands on a bf16
