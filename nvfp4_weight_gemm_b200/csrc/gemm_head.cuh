@@ -209,7 +209,7 @@ __global__ void __launch_bounds__(HeadCfg<NX>::THREADS, 1) gemm_head_kernel(cons
                         tc_fail(p.err, abort_flag, TL_DEV_ERR_TIMEOUT_DRAIN);
         }
     } else if (head_issuer_of_warp(warp) >= 0) {
-        // ------------------------------------------------------------ MMA issuers (k-steps 4j .. 4j + 3)
+        // ------------------------------------------------------------ MMA issuers (k-steps 8j .. 8j + 7)
         // warp-uniform operands (lane-0 shuffles), as in gemm_ex_kernel
         const int j = __shfl_sync(0xFFFFFFFFu, head_issuer_of_warp(warp), 0);
         const int i0 = C::KSTEPS * j;
