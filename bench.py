@@ -549,7 +549,7 @@ def head_bytes(M):
 
 
 def head_figure(tl, dev, stream, rank):
-    """Time tl_fp8_head (X prep + head GEMM + fp64 fallback + two top-2 stages: five launches) at a
+    """Time tl_fp8_head (X prep, head GEMM, and one tail launch for fp64 rows and the top-2: three launches) at a
     151,936 x 5,120 FP8 head with per-row scales, per M, with CUDA events on the launching stream
     (the 0.78 GB weight is over six times L2, so no flush), then check sampled logits against the
     oracle and the top-2 against the kernel's own logits."""
@@ -605,7 +605,7 @@ def head_figure(tl, dev, stream, rank):
     return {"N": HEAD_N, "K": HEAD_K, "weights": "E4M3, per-row fp32 scale", "per_M": per_M,
             "min_frac_over_M": round(min(v["frac"] for v in per_M.values()), 4),
             "bytes": "N*K + 4N + 2MK + 4MN + 16M per call",
-            "kernels": "x_prep_kernel + gemm_head_kernel<NX> + head_fallback_kernel + head_top2_part_kernel + head_top2_final_kernel (timed together)",
+            "kernels": "x_prep_kernel + gemm_head_kernel<NX> + head_tail_kernel (timed together)",
             "gap_ulp_at_M32": [round(float(v), 3) for v in gap],
             "parity_sampled": {"checked": int(got.size), "outside": outside, "top2_matches_own_logits": top2_ok,
                                "sample": "528 weight rows (512 seeded + last 16), all 32 rows, vs fp64 oracle"}}

@@ -13,8 +13,8 @@
 // E4M3 value is an f16 normal, so exact), written into tensor memory by CUDA cores; B = X
 // prepared by xprep.cuh (row m times 2^-e_m in f16, exact); fp32 accumulation in tensor memory.
 // The epilogue writes fp32 logits acc * 2^e_m * s_n; rows xprep flags are recomputed in fp64
-// (head_fallback_kernel), and two small kernels reduce every row of logits to its top two
-// (head_top2_part_kernel over chunks of the row, head_top2_final_kernel over the chunks).
+// by head_tail_kernel, which also reduces every row of logits to its top two (partials over
+// chunks of the row, merged by the row's last CTA).
 //
 // Tile: 128 weight rows x 256 k (32 KiB of E4M3 bytes, two 128-byte swizzled slices per row);
 // roles and stream-K split as in gemm_ex.cuh (weight producer, X producer, 2 MMA issuers,
@@ -407,38 +407,24 @@ __global__ void __launch_bounds__(HeadCfg<NX>::THREADS, 1) gemm_head_kernel(cons
     }
 }
 
-// Rows the X preparation flagged: logits recomputed from the bf16 X as given, in fp64 (a warp
-// per weight row, lanes over k, fixed butterfly), then rounded to fp32 once.
-constexpr int HEAD_FB_THREADS = 256;
-__global__ void __launch_bounds__(HEAD_FB_THREADS) head_fallback_kernel(const __grid_constant__ HeadParams p) {
-    unsigned rows = __ldcg(p.rowmask);
-    if (p.M < 32) rows &= (1u << p.M) - 1u;
-    if (!rows) return;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long gw = (long long)blockIdx.x * (HEAD_FB_THREADS / 32) + warp;
-    const long long nw = (long long)gridDim.x * (HEAD_FB_THREADS / 32);
-    for (long long n = gw; n < p.N; n += nw) {
-        const uint8_t* wr = p.w + (size_t)n * p.K;
-        const double sn = p.row_scale ? (double)p.row_scale[n] : (double)p.tensor_scale;
-        unsigned todo = rows;
-        while (todo) {
-            const int m = __ffs(todo) - 1;
-            todo &= todo - 1u;
-            const __nv_bfloat16* xr = p.x + (size_t)m * p.K;
-            double acc = 0.0;
-            for (int k = 2 * lane; k < p.K; k += 64) {
-                const uint32_t two = (uint32_t)wr[k] | ((uint32_t)wr[k + 1] << 8);
-                uint32_t h;
-                asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(h) : "r"(two));
-                const __half2 hv = *reinterpret_cast<const __half2*>(&h);
-                acc += (double)__bfloat162float(xr[k]) * (double)__low2float(hv);
-                acc += (double)__bfloat162float(xr[k + 1]) * (double)__high2float(hv);
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
-            if (lane == 0) p.logits[(size_t)m * p.N + n] = (float)(acc * sn);
-        }
+// One logit of a row the X preparation flagged, recomputed from the bf16 X as given in fp64 by
+// one warp (lanes over k, a fixed butterfly) and rounded to fp32 once.
+__device__ __forceinline__ float head_logit_fp64(const HeadParams& p, int m, int n, int lane) {
+    const uint8_t* wr = p.w + (size_t)n * p.K;
+    const __nv_bfloat16* xr = p.x + (size_t)m * p.K;
+    const double sn = p.row_scale ? (double)p.row_scale[n] : (double)p.tensor_scale;
+    double acc = 0.0;
+    for (int k = 2 * lane; k < p.K; k += 64) {
+        const uint32_t two = (uint32_t)wr[k] | ((uint32_t)wr[k + 1] << 8);
+        uint32_t h;
+        asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(h) : "r"(two));
+        const __half2 hv = *reinterpret_cast<const __half2*>(&h);
+        acc += (double)__bfloat162float(xr[k]) * (double)__low2float(hv);
+        acc += (double)__bfloat162float(xr[k + 1]) * (double)__high2float(hv);
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+    return (float)(acc * sn);
 }
 
 // Greedy top-2 of each row of logits, one CTA per row, a fixed order of comparisons: token
@@ -491,14 +477,33 @@ __device__ __forceinline__ T2 t2_warp_merge(T2 t) {
     return t;
 }
 
-// Stage 1: grid (chunks, M); CTA (c, m) reduces logits[m][c * chunk, (c + 1) * chunk) to one
-// partial. The merge keeps the largest value (lowest index among equal ones) and the largest of
-// the rest, so the two stages give the same answer in any order of merging.
-__global__ void __launch_bounds__(HEAD_TOP2_THREADS) head_top2_part_kernel(const float* logits, int N, int chunk,
-                                                                           T2* part) {
-    const int c = blockIdx.x, m = blockIdx.y;
-    const float* row = logits + (size_t)m * N;
+// After the GEMM, one launch: grid (chunks, M); CTA (c, m) takes logits[m][c * chunk, (c + 1) * chunk).
+//   1. If the X preparation flagged row m, it first recomputes those logits in fp64 (a warp per
+//      weight row) and writes them.
+//   2. It reduces the chunk to one partial (best value, its lowest index, best of the rest, any
+//      NaN) and stores it.
+//   3. The last CTA of row m to finish (an atomic counter per row, reset by that CTA; nothing waits)
+//      merges the row's partials with one warp and writes the token, the two best values and their
+//      gap in bf16 units in the last place (token -1 and NaN for a row with a NaN).
+// The merge keeps the largest value with the lowest index and the largest of the rest, so the answer
+// does not depend on the order in which partials are merged.
+__global__ void __launch_bounds__(HEAD_TOP2_THREADS) head_tail_kernel(const __grid_constant__ HeadParams p, int chunk,
+                                                                      T2* part, unsigned* row_counters,
+                                                                      HeadTop2* out) {
+    const int c = blockIdx.x, m = blockIdx.y, chunks = gridDim.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int N = p.N;
+    float* row = p.logits + (size_t)m * N;
     const int n0 = c * chunk, n1 = min(N, n0 + chunk);
+    unsigned flagged = __ldcg(p.rowmask);
+    if (p.M < 32) flagged &= (1u << p.M) - 1u;
+    if ((flagged >> m) & 1u) {
+        for (int n = n0 + warp; n < n1; n += HEAD_TOP2_THREADS / 32) {
+            const float v = head_logit_fp64(p, m, n, lane);
+            if (lane == 0) row[n] = v;
+        }
+        __syncthreads();
+    }
     T2 t = {-INFINITY, -INFINITY, 0x7FFFFFFF, 0};
     for (int n = n0 + (int)threadIdx.x; n < n1; n += HEAD_TOP2_THREADS) {
         const float v = __ldcg(row + n);
@@ -508,35 +513,43 @@ __global__ void __launch_bounds__(HEAD_TOP2_THREADS) head_top2_part_kernel(const
     }
     t = t2_warp_merge(t);
     __shared__ T2 ws[HEAD_TOP2_THREADS / 32];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __shared__ int last;
     if (lane == 0) ws[warp] = t;
     __syncthreads();
     if (threadIdx.x == 0) {
         T2 r = ws[0];
         for (int w = 1; w < HEAD_TOP2_THREADS / 32; ++w) r = t2_merge(r, ws[w]);
-        part[(size_t)m * gridDim.x + c] = r;
+        part[(size_t)m * chunks + c] = r;
+        __threadfence();
+        last = (atomicAdd(row_counters + m, 1u) == (unsigned)(chunks - 1)) ? 1 : 0;
     }
-}
-
-// Stage 2: one warp per row merges the row's partials and writes the token, the two best values
-// and their gap in bf16 units in the last place at the largest (token -1 and NaN for a row with a NaN).
-__global__ void __launch_bounds__(32) head_top2_final_kernel(const T2* part, int chunks, HeadTop2* out) {
-    const int m = blockIdx.x, lane = threadIdx.x;
-    T2 t = {-INFINITY, -INFINITY, 0x7FFFFFFF, 0};
-    for (int c = lane; c < chunks; c += 32) t = t2_merge(t, part[(size_t)m * chunks + c]);
-    t = t2_warp_merge(t);
+    __syncthreads();
+    if (!last || warp != 0) return;
+    __threadfence();
+    T2 r = {-INFINITY, -INFINITY, 0x7FFFFFFF, 0};
+    for (int q = lane; q < chunks; q += 32) {
+        T2 e;
+        const T2* src = part + (size_t)m * chunks + q;
+        e.v1 = __ldcg(&src->v1);
+        e.v2 = __ldcg(&src->v2);
+        e.i1 = __ldcg(&src->i1);
+        e.nan = __ldcg(&src->nan);
+        r = t2_merge(r, e);
+    }
+    r = t2_warp_merge(r);
     if (lane == 0) {
         HeadTop2 o;
-        if (t.nan) {
+        if (r.nan) {
             o.token = -1;
             o.top1 = o.top2 = o.gap_ulp = __int_as_float(0x7FC00000);
         } else {
-            o.token = t.i1;
-            o.top1 = t.v1;
-            o.top2 = t.v2;
-            o.gap_ulp = (t.v1 - t.v2) / bf16_ulp_f(t.v1);
+            o.token = r.i1;
+            o.top1 = r.v1;
+            o.top2 = r.v2;
+            o.gap_ulp = (r.v1 - r.v2) / bf16_ulp_f(r.v1);
         }
         out[m] = o;
+        row_counters[m] = 0u;   // ready for the next call
     }
 }
 

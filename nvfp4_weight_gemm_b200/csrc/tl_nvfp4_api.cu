@@ -1501,18 +1501,16 @@ tl_status tl_fp8_head(const void* x, int M, const void* w_fp8, int N, int K, flo
     TL_CUDA(cudaGetLastError());
     st = (NX == 16) ? launch_head<16>(*d, hp, s) : launch_head<32>(*d, hp, s);
     if (st != TL_OK) return st;
-    tl::head_fallback_kernel<<<(unsigned)d->num_sms, tl::HEAD_FB_THREADS, 0, s>>>(hp);
-    TL_CUDA(cudaGetLastError());
-    // top-2 in two stages over at most 1024 chunks of a row (the partials reuse the split-K scratch,
-    // free again once the GEMM has run on this stream)
+    // fp64 rows, partials over chunks of at most 1024 per row and the per-row merge in one launch;
+    // the partials reuse the split-K scratch (free again once the GEMM has run on this stream), the
+    // per-row counters sit past the GEMM's in the counter array and are left at zero
     int chunk = (N + 1023) / 1024;
     chunk = ((chunk < 4096 ? 4096 : chunk) + 255) & ~255;
     const int chunks = (N + chunk - 1) / chunk;
     tl::T2* part = reinterpret_cast<tl::T2*>(d->partials);
-    tl::head_top2_part_kernel<<<dim3((unsigned)chunks, (unsigned)M), tl::HEAD_TOP2_THREADS, 0, s>>>(logits, N, chunk,
-                                                                                               part);
-    TL_CUDA(cudaGetLastError());
-    tl::head_top2_final_kernel<<<(unsigned)M, 32, 0, s>>>(part, chunks, reinterpret_cast<tl::HeadTop2*>(top2));
+    unsigned* row_counters = d->counters + counter_words(d->num_sms) - TL_HEAD_MAX_M;
+    tl::head_tail_kernel<<<dim3((unsigned)chunks, (unsigned)M), tl::HEAD_TOP2_THREADS, 0, s>>>(
+        hp, chunk, part, row_counters, reinterpret_cast<tl::HeadTop2*>(top2));
     TL_CUDA(cudaGetLastError());
     return TL_OK;
 }
