@@ -288,8 +288,11 @@ tl_status tl_nvfp4_quantize(const float* w, int N, int K, void* w_codes, void* w
  *   top2         device tl_head_top2 [M], output; token -1 and NaN values for a row with a NaN
  * Arithmetic: exact f16 operands on the tensor cores (every E4M3 value is an f16 value; X rows
  * prepared as for TL_PATH_EXACT, with the same fp64 fallback for rows outside f16), fp32
- * accumulation. Same scratch, allocation and serialisation rules as the calls without a plan
- * (the prepared-X buffer of the device). Asynchronous on `stream`. */
+ * accumulation. Three launches: X preparation, the GEMM, and one kernel that recomputes flagged
+ * rows in fp64 and reduces every row to its top two (partials in the device's split-K scratch,
+ * merged by the row's last CTA through a per-row counter it leaves at zero). Same scratch,
+ * allocation and serialisation rules as the calls without a plan (the prepared-X buffer, the
+ * split-K partials and counters of the device). Asynchronous on `stream`. */
 #define TL_HEAD_MAX_M 32
 typedef struct {
     int token;
