@@ -138,7 +138,9 @@ tl_status tl_init(int device);
 /* Free every per-device state. No call may be in flight. */
 void tl_shutdown(void);
 
-/* Y = X . dequant(W)^T for one weight matrix (see the top of this file).
+/* Y = X . dequant(W)^T for one weight matrix (see the top of this file): one projection of the
+ * verify pass, whose weights are four bits each with one scale per 16 (TandemLLM docs v0.12.0,
+ * "What TandemLLM is", section 1.2).
  *   x      device bf16 [M][K], 16-byte aligned
  *   M      0..TL_NVFP4_MAX_M (0 is a no-op returning TL_OK; more returns TL_ERR_UNSUPPORTED)
  *   w_codes, w_scales  device, 16-byte aligned, layouts above
@@ -202,7 +204,7 @@ typedef struct {
 } tl_nvfp4_matrix;
 
 /* The verify GEMM of `n_mats` independent matrices (e.g. QKV, O, gate+up and
- * down of 64 layers) in one persistent launch: all matrices' k-tiles form one
+ * down of the served model's 64 layers; "What TandemLLM is", section 1.1) in one persistent launch: all matrices' k-tiles form one
  * work list that is split evenly over the SMs, so no SM idles at a matrix
  * boundary. `mats` is a HOST array read during the call; each entry obeys the
  * rules of tl_nvfp4_verify_gemm(), with the same M for all. 1 <= n_mats <=
@@ -222,7 +224,8 @@ tl_status tl_nvfp4_verify_stack_host(const tl_nvfp4_matrix* mats, int n_mats, in
                                      const void* x_host, void* x_dev, void* y_host, void* y_dev,
                                      void* stream);
 
-/* Plans: the descriptors of a stack built once, launched many times.
+/* Plans: the descriptors of a stack built once, launched many times (the verify pass runs
+ * every decoding round over the same weights; "What TandemLLM is", section 1.2).
  *
  * tl_nvfp4_plan_create() validates `mats` (same rules as tl_nvfp4_verify_stack),
  * encodes the TMA descriptors of every matrix and uploads them to the device once
@@ -254,12 +257,14 @@ tl_status tl_nvfp4_plan_run_host(tl_nvfp4_plan plan, const void* x_host, void* y
 tl_status tl_nvfp4_plan_destroy(tl_nvfp4_plan plan);
 
 /* Parity hook: w_out[n][k] = fp32(e2m1 * e4m3 * global_scale), rounded once
- * (the product e2m1 * e4m3 is exact). w_out: device float [N][K], 16-byte
+ * (the product e2m1 * e4m3 is exact); the weight format of "What TandemLLM is", section 1.2. w_out: device float [N][K], 16-byte
  * aligned. Same size rules as tl_nvfp4_verify_gemm(). */
 tl_status tl_nvfp4_dequant(const void* w_codes, const void* w_scales, float global_scale,
                            float* w_out, int N, int K, void* stream);
 
-/* Round-to-nearest NVFP4 quantiser (weight-pack builder):
+/* Round-to-nearest NVFP4 quantiser (weight-pack builder). The pages build their packs with GPTQ
+ * ("Installing TandemLLM", section 3.12), which needs a checkpoint and calibration data; this is
+ * the plain round-to-nearest reading of the same format:
  *   g = fp32(absmax(w) / (6*448)); per 16-block s = E4M3_RNE_satfinite(absmax_block / 6 / g)
  *   in fp64; codes = E2M1_RNE(w / (e4m3(s) * g)) in fp64, ties to the even code, zero -> 0x0.
  * w: device float [N][K] (finite); codes/scales: device outputs as above.
