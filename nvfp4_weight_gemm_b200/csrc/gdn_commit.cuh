@@ -14,11 +14,12 @@
 //     u_t + sum_{s<t} b_t (a_{s+1} ... a_t) (k_s . k_t) u_s = b_t (v_t - g_t S_0 k_t)
 //     S_L = g_L S_0 + sum_t (a_{t+1} ... a_L) u_t k_t^T
 //
-// so one launch computes P = S_0 K^T, solves the unit lower-triangular system for U by forward
-// substitution (one thread per state row), and writes S_L = g_L S_0 + U' K, all in fp32 on CUDA
-// cores. One CTA per head (about 106 KB of shared memory at d_k = d_v = 128, two per SM); S_0 is
-// read once from HBM into shared memory and S_L written back in place, coalesced. Bound: HBM for the state (2 * DV * DK * 4 bytes per head) against the fp32
-// FMA pipe for the 2 * DV * DK * L multiply-adds per head.
+// so one launch forms the right-hand sides R = B (V^T - S_0 K^T G), solves the unit
+// lower-triangular system for U by forward substitution (one thread per state row), and writes
+// S_L = g_L S_0 + U' K, all in fp32 on CUDA cores. One CTA per head (about 106 KB of shared memory
+// at d_k = d_v = 128, two per SM); S_0 is read once from HBM into shared memory and S_L written
+// back in place, coalesced. Bound: HBM for the state (2 * DV * DK * 4 bytes per head) against the
+// fp32 FMA pipe for the 2 * DV * DK * L multiply-adds per head.
 #pragma once
 #include <cstdint>
 
