@@ -1450,8 +1450,9 @@ tl_status tl_fp8_head(const void* x, int M, const void* w_fp8, int N, int K, flo
     if (!aligned16(x) || !aligned16(w_fp8) || !aligned16(logits) || (row_scales && !aligned16(row_scales)))
         return fail(TL_ERR_MISALIGNED, "x, w, logits and row_scales must be 16-byte aligned");
     if (!row_scales && !std::isfinite(tensor_scale)) return fail(TL_ERR_INVALID_VALUE, "tensor_scale is not finite");
-    if (overlap(logits, (size_t)4 * M * N, x, (size_t)2 * M * K) || overlap(logits, (size_t)4 * M * N, w_fp8, (size_t)N * K))
-        return fail(TL_ERR_INVALID_VALUE, "logits overlap x or the weights");
+    if (overlap(logits, (size_t)4 * M * N, x, (size_t)2 * M * K) || overlap(logits, (size_t)4 * M * N, w_fp8, (size_t)N * K) ||
+        overlap(top2, sizeof(tl_head_top2) * (size_t)M, logits, (size_t)4 * M * N))
+        return fail(TL_ERR_INVALID_VALUE, "logits overlap x, the weights or top2");
     if (M == 0) return TL_OK;
     DevState* d = nullptr;
     tl_status st = current_state(&d);
@@ -1524,6 +1525,12 @@ tl_status tl_gdn_commit(float* state, int H, int d_k, int d_v, const float* k, c
     if (n_nodes < 1) return fail(TL_ERR_INVALID_VALUE, "n_nodes = %d must be >= 1", n_nodes);
     if (!state || !k || !v || !alpha || !beta || (L > 0 && !path)) return fail(TL_ERR_INVALID_VALUE, "null pointer");
     if (!aligned16(state) || !aligned16(k)) return fail(TL_ERR_MISALIGNED, "state and k must be 16-byte aligned");
+    {
+        const size_t sb = (size_t)H * d_v * d_k * 4, nh = (size_t)n_nodes * H;
+        if (overlap(state, sb, k, nh * d_k * 4) || overlap(state, sb, v, nh * d_v * 4) ||
+            overlap(state, sb, alpha, nh * 4) || overlap(state, sb, beta, nh * 4))
+            return fail(TL_ERR_INVALID_VALUE, "state overlaps the path inputs");
+    }
     tl::GdnPath p;
     memset(&p, 0, sizeof p);
     for (int t = 0; t < L; ++t) {

@@ -88,12 +88,29 @@ def test_dequant_and_quantize_validate(L):
 def test_gdn_commit_validates(L):
     path = (ctypes.c_int * 4)(0, 1, 2, 3)
     def call(H=4, dk=128, dv=128, state=A, n_nodes=8, p=path, n=4):
-        return L.tl_gdn_commit(state, H, dk, dv, A, A, A, A, n_nodes, p, n, None)
+        # fake, disjoint 16-byte aligned addresses; never dereferenced on these paths
+        return L.tl_gdn_commit(state, H, dk, dv, A + (1 << 24), A + (1 << 25), A + (1 << 26), A + (1 << 27),
+                               n_nodes, p, n, None)
     assert call(H=0) == 1
     assert call(dk=96) == 3 and call(dv=32) == 3
     assert call(n=33) == 1 and call(n=-1) == 1
     assert call(n_nodes=3) == 1                 # node index 3 is outside 0..2
     assert call(state=A + 4) == 2
-    assert L.tl_gdn_commit(A, 4, 128, 128, A + 4, A, A, A, 8, path, 4, None) == 2   # misaligned keys
+    assert L.tl_gdn_commit(A, 4, 128, 128, A + (1 << 24) + 4, A + (1 << 25), A + (1 << 26), A + (1 << 27), 8, path, 4,
+                           None) == 2   # misaligned keys
     assert call(state=0) == 1
     assert call(n=0) == 0                       # an empty path is a no-op and never reaches CUDA
+    # the state may not overlap the per-node inputs (state = keys)
+    assert L.tl_gdn_commit(A, 4, 128, 128, A, A + (1 << 24), A + (1 << 25), A + (1 << 26), 8, path, 4, None) == 1
+
+
+def test_fp8_head_validates(L):
+    def call(x=A, M=8, w=A + (1 << 24), N=1000, K=512, ts=1.0, rs=None, lg=A + (1 << 26), t2=A + (1 << 27)):
+        return L.tl_fp8_head(x, M, w, N, K, ctypes.c_float(ts), rs, lg, t2, None)
+    assert call(M=33) == 3 and call(M=-1) == 1
+    assert call(N=1) == 1 and call(K=100) == 1
+    assert call(x=A + 4) == 2 and call(lg=A + (1 << 26) + 4) == 2
+    assert call(ts=float("nan")) == 1
+    assert call(lg=A) == 1                       # logits over x
+    assert call(t2=A + (1 << 26)) == 1           # top2 over logits
+    assert call(M=0) == 0                        # no rows: a no-op before any CUDA call
