@@ -524,3 +524,26 @@ def test_gdn_path_gather(orc):
     assert np.array_equal(K, Kn[[0, 2, 4]]) and np.array_equal(b, bn[[0, 2, 4]])
     S0 = rng.standard_normal((3, 4))
     assert np.allclose(orc.gdn_commit_closed_form(S0, K, V, a, b), orc.gdn_sequential(S0, K, V, a, b), atol=1e-13)
+
+
+def test_gdn_closed_form_matches_transition_matrices(orc):
+    # a third formulation, written out with explicit d_k x d_k matrices: with
+    # T_t = a_t (I - b_t k_t k_t^T), S_L = S_0 T_1 ... T_L + sum_t b_t v_t k_t^T T_{t+1} ... T_L
+    rng = np.random.default_rng(16)
+    dk, dv, L = 12, 7, 9
+    S0 = rng.standard_normal((dv, dk))
+    K = rng.standard_normal((L, dk))
+    K /= np.linalg.norm(K, axis=1, keepdims=True)
+    V = rng.standard_normal((L, dv))
+    a = rng.uniform(0.6, 1.0, L)
+    b = rng.uniform(0.0, 1.0, L)
+    T = [a[t] * (np.eye(dk) - b[t] * np.outer(K[t], K[t])) for t in range(L)]
+
+    def chain(lo):
+        P = np.eye(dk)
+        for t in range(lo, L):
+            P = P @ T[t]
+        return P
+
+    ref = S0 @ chain(0) + sum(b[t] * np.outer(V[t], K[t]) @ chain(t + 1) for t in range(L))
+    assert np.allclose(orc.gdn_commit_closed_form(S0, K, V, a, b), ref, rtol=0, atol=1e-12)
