@@ -329,8 +329,8 @@ tl_status tl_fp8_head(const void* x, int M, const void* w_fp8, int N, int K, flo
  *   L         0..TL_GDN_MAX_PATH (0 is a no-op)
  * fp32 arithmetic on CUDA cores; no workspace, no allocation. Asynchronous on `stream`; the
  * host path array is copied into the launch and may be reused at once. Errors: a size out of
- * range, a node index outside 0..n_nodes-1, a null or misaligned pointer -> the status, nothing
- * launched. */
+ * range, a node index outside 0..n_nodes-1, a null or misaligned pointer, a state buffer that
+ * overlaps k, v, alpha or beta -> the status, nothing launched. */
 #define TL_GDN_MAX_PATH 32
 tl_status tl_gdn_commit(float* state, int H, int d_k, int d_v, const float* k, const float* v, const float* alpha,
                         const float* beta, int n_nodes, const int* path, int L, void* stream);
